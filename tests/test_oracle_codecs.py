@@ -1,0 +1,192 @@
+"""Pins of the oracle's key and value codecs and of the byte arithmetic: brute-force nearest-centroid
+search, hand-worked bit packing, the pages' packing order and byte formulas, worked value cases
+(constant group, two-value group, round-half-even ties), the measured MSE against the codebook's
+distortion, and the compression ratios the pages print."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import tq_oracle as o
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "pages_figures.json")))
+
+
+# ------------------------------------------------------------------------------------ key codec
+
+@pytest.mark.parametrize("d", [3, 4, 8])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_boundary_count_is_brute_force_argmin(d, bits):
+    rng = np.random.default_rng(d * 10 + bits)
+    x16 = rng.standard_normal((1000, d)).astype(np.float16)
+    pi = o.operational_rotation(d, 3)
+    c = o.to_fp16_values(o.sphere_codebook(d, bits))
+    t = o.boundaries_of(c)
+    idx, n, y = o.encode_k(x16, pi, t)
+    brute = np.argmin(np.abs(y[:, :, None] - c[None, None, :]), axis=-1)   # first occurrence
+    assert np.array_equal(idx, brute)
+    # exact ties go to the lower index, as argmin's first occurrence does
+    assert np.array_equal(o.nearest_index(t, t), np.arange(len(t)))
+    assert np.array_equal(np.argmin(np.abs(t[:, None] - c[None, :]), axis=1), np.arange(len(t)))
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_pack_is_little_endian_integer_of_the_bitstream(bits):
+    rng = np.random.default_rng(bits)
+    d = 40
+    idx = rng.integers(0, 1 << bits, size=(7, d))
+    packed = o.pack_lsb(idx, bits)
+    for r in range(7):
+        value = sum(int(idx[r, j]) << (bits * j) for j in range(d))
+        assert bytes(packed[r]) == value.to_bytes((d * bits + 7) // 8, "little")
+    assert np.array_equal(o.unpack_lsb(packed, bits, d), idx)
+
+
+def test_pack_3bit_worked_example():
+    # 5,3,7,1,0,6,2,4 -> sum idx_j 8^j = 9110493 = 0x8B03DD -> bytes DD 03 8B
+    assert list(o.pack_lsb(np.array([[5, 3, 7, 1, 0, 6, 2, 4]]), 3)[0]) == [0xDD, 0x03, 0x8B]
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_zero_vector(bits):
+    d = 128
+    pi = o.operational_rotation(d, 0)
+    c, t = o.operational_codebook(d, bits)
+    idx, n, _ = o.encode_k(np.zeros((2, d), np.float16), pi, t)
+    assert np.all(idx == (1 << (bits - 1)) - 1) and np.all(n == 0.0)
+    assert np.all(o.decode_k(idx, n, pi, c) == 0.0)
+
+
+def test_power_of_two_scaling_invariance():
+    d = 128
+    rng = np.random.default_rng(2)
+    x16 = rng.standard_normal((200, d)).astype(np.float16)
+    pi = o.operational_rotation(d, 0)
+    _, t = o.operational_codebook(d, 4)
+    i1, n1, _ = o.encode_k(x16, pi, t)
+    i2, n2, _ = o.encode_k((x16.astype(np.float32) * 4).astype(np.float16), pi, t)
+    # the 1e-8 guard changes y by ~1e-9 relative: only coordinates that close to a boundary may differ
+    assert np.mean(i1 != i2) < 1e-4 and np.allclose(n2, 4 * n1, rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_measured_mse_matches_distortion(bits):
+    # Workload of the K-only round trip: 4096 fp16 N(0,1) vectors, head_dim 128, seeded rotation.
+    d, n = 128, 4096
+    rng = np.random.default_rng(0)
+    x16 = rng.standard_normal((n, d)).astype(np.float16)
+    x = x16.astype(np.float64)
+    pi = o.operational_rotation(d, 0)
+    c, t = o.operational_codebook(d, bits)
+    idx, norms, _ = o.encode_k(x16, pi, t)
+    xh = o.decode_k(idx, norms, pi, c)
+    rel = np.sum((xh - x) ** 2, axis=1) / np.sum(x * x, axis=1)
+    D = o.sphere_distortion(d, c, t)
+    assert abs(rel.mean() - D) < 4.0 * rel.std() / math.sqrt(n) + 2e-4 * D
+    lo, hi = o.distortion_bounds(bits)
+    assert rel.mean() < hi
+    if bits == 4:
+        # the turbo-attn demo prints relative error 0.10 for 4-bit, d = 128 (a Hadamard rotation
+        # there; the same codebook family): sqrt of our distortion rounds to the printed figure
+        err = math.sqrt(np.sum((xh - x) ** 2) / np.sum(x * x))
+        assert round(err, 2) == GOLDEN["tkv_demo_relative_error"]["value"]
+
+
+# ---------------------------------------------------------------------------------- value codec
+
+def _group(vals, d=32):
+    v = np.zeros((1, d), np.float16)
+    v[0, :len(vals)] = vals
+    v[0, len(vals):] = vals[-1]
+    return v
+
+
+def test_value_constant_group():
+    x = np.full((1, 32), 1.75, np.float16)
+    data, s, z, q = o.encode_v(x, 2)
+    assert np.all(q == 0) and float(s[0, 0]) == 0.0 and float(z[0, 0]) == 1.75
+    assert np.all(o.decode_v(data, s, z, 2, 32) == 1.75)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_value_two_value_group(bits):
+    x = np.zeros((1, 32), np.float16)
+    x[0, ::2] = -1.0
+    x[0, 1::2] = 3.0
+    data, s, z, q = o.encode_v(x, bits)
+    levels = (1 << bits) - 1
+    assert np.array_equal(q[0, ::2], np.zeros(16)) and np.array_equal(q[0, 1::2], np.full(16, levels))
+    out = o.decode_v(data, s, z, bits, 32)
+    # the endpoints come back up to the fp16 rounding of the scale
+    assert np.all(out[0, ::2] == -1.0)
+    assert np.all(np.abs(out[0, 1::2] - 3.0) <= levels * abs(float(s[0, 0]) - 4.0 / levels) + 1e-6)
+
+
+def test_value_round_half_even():
+    # min 0, max 3 at 2 bits: scale = 1, so x = 0.5, 1.5, 2.5 sit exactly on half-integers
+    x = _group([0.0, 3.0, 0.5, 1.5, 2.5, 1.0, 2.0])
+    _, s, z, q = o.encode_v(x, 2)
+    assert float(s[0, 0]) == 1.0 and float(z[0, 0]) == 0.0
+    assert list(q[0, :7]) == [0, 3, 0, 2, 2, 1, 2]
+
+
+def test_value_pack_order_matches_store_py():
+    g2, g4 = GOLDEN["value_pack_order_2bit"], GOLDEN["value_pack_order_4bit"]
+    assert int(o.pack_lsb(np.array([g2["q"]]), 2)[0, 0]) == g2["byte"]
+    assert int(o.pack_lsb(np.array([g4["q"]]), 4)[0, 0]) == g4["byte"]
+
+
+@pytest.mark.parametrize("row", GOLDEN["value_bytes_d128"]["rows"])
+def test_value_bytes_formula_and_arrays(row):
+    f = o.v_formula_nbytes((5, 128), row["bits"], row["group"], row["layout"])
+    assert f["compressed_v_bytes"] == 5 * row["payload"]
+    assert f["scales_bytes"] == 5 * row["scales"] and f["zeros_bytes"] == 5 * row["zeros"]
+    x = np.random.default_rng(0).standard_normal((5, 128)).astype(np.float16)
+    data, s, z, _ = o.encode_v(x, row["bits"], row["group"], row["layout"])
+    assert data.nbytes == f["compressed_v_bytes"] and s.nbytes == f["scales_bytes"] and z.nbytes == f["zeros_bytes"]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("layout", ["group", "token"])
+def test_value_error_bound(bits, layout):
+    rng = np.random.default_rng(bits)
+    x16 = (rng.standard_normal((500, 128)) * np.exp(rng.standard_normal(128))).astype(np.float16)
+    data, s, z, q = o.encode_v(x16, bits, 32, layout)
+    out = o.decode_v(data, s, z, bits, 128, 32, layout)
+    g = 128 if layout == "token" else 32
+    x = x16.astype(np.float64)
+    vmin = x.reshape(500, -1, g).min(-1)
+    vmax = x.reshape(500, -1, g).max(-1)
+    s_exact = (vmax - vmin) / ((1 << bits) - 1)
+    # |x_hat - x| <= s/2 + (2^b - 1) |s16 - s| + |z16 - z| + fp32 slop
+    bound = (0.5 * s_exact + ((1 << bits) - 1) * np.abs(s.astype(np.float64) - s_exact)
+             + np.abs(z.astype(np.float64) - vmin) + 1e-5 * np.maximum(np.abs(vmax), np.abs(vmin)))
+    err = np.abs(out.astype(np.float64) - x).reshape(500, -1, g).max(-1)
+    assert np.all(err <= bound)
+
+
+# ------------------------------------------------------------------------------ byte arithmetic
+
+def test_ratios_the_pages_print():
+    # 4-bit codes + a 2-byte norm at head_dim 128 (turbo-attn demo: 3.88x vs bf16)
+    r = o.k_compression_ratio(128, 4, norm_bytes=2)
+    assert round(r, 2) == GOLDEN["tkv_demo_ratio_vs_bf16"]["value"]
+    # 4.125 bits per number prints as 4.13; 16 / 4.13 prints as 3.87 (turbo-attn 'Why')
+    bpn = 8.0 * (o.k_row_bytes(128, 4) + 2) / 128
+    assert abs(bpn - GOLDEN["tkv_slot_ratio"]["bits_per_number"]) <= 0.005      # printed half-up
+    assert round(16.0 / GOLDEN["tkv_slot_ratio"]["bits_per_number"], 2) == GOLDEN["tkv_slot_ratio"]["value"]
+    # f32 norm (the aitherkvcache signature): 4 bits -> 3.8x, 2 bits -> 7.1x vs FP16
+    g = GOLDEN["aither_range_vs_fp16"]
+    assert round(o.k_compression_ratio(128, g["bits_low"], 4), 1) == g["low"]
+    assert round(o.k_compression_ratio(128, g["bits_high"], 4), 1) == g["high"]
+    assert o.k_row_bytes(128, 4) == 64
+
+
+def test_tqai_average_bits():
+    for row in GOLDEN["tqai_average_bits"]["rows"]:
+        avg = (row["k_bits"] + row["v_bits"]) / 2.0
+        assert avg == row["avg_bits"]
+        if "saved_pct" in row:
+            assert abs(100.0 * (1.0 - avg / 16.0) - row["saved_pct"]) < 1.5
