@@ -1,0 +1,237 @@
+/*
+ * tq.h -- C ABI of libtq: TurboQuant-style KV-cache compression on NVIDIA B200 (sm_100a).
+ *
+ * The hot path, and the page that defines each step:
+ *   - key encode:   norm separation, seeded Haar rotation, nearest Lloyd-Max level, bit packing
+ *                   ("KV Cache API", compressors.py MSECompressor.compress; "aitherkvcache",
+ *                   TurboQuant.encode returning uint8 codes plus f32 norms);
+ *   - value encode: grouped affine min/max quantization with fp16 scale and zero
+ *                   ("KV Cache API", values.py quantize_values);
+ *   - decode:       unpack, codebook gather, inverse rotation, norm rescale; affine dequant for values
+ *                   (compressors.py MSECompressor.decompress; values.py dequantize_values);
+ *   - decode-step attention scored directly against the packed keys
+ *                   ("KV Cache API", store.py TurboQuantKVCache.attention_scores / attend;
+ *                   "turbo-attn", the split-K paged decode kernel with a fused query rotation).
+ *
+ * Conventions shared by every entry point
+ *   - Every call returns a tq_status.  On anything but TQ_OK, tq_last_error() returns a message (owned by
+ *     the library, valid until the next call on the same thread) that names the offending argument.
+ *   - Device pointers are caller-owned (allocate them with any allocator, e.g. PyTorch).  No entry point
+ *     allocates or frees device memory except tq_codec_create / tq_codec_destroy.
+ *   - Kernels are enqueued on the caller's stream (a cudaStream_t passed as void*; NULL = the legacy
+ *     default stream) and return without synchronising.  Outputs are fully overwritten.
+ *   - Argument errors are detected on the host before anything is enqueued; nothing is launched then.
+ *   - Preconditions that are NOT checked on the device: inputs are finite (no NaN/Inf), pointers
+ *     reference allocations of the stated sizes, and outputs do not overlap inputs.
+ *   - Half-precision data are IEEE binary16 passed as void* / uint16_t*.
+ *   - Supported head dims for the device kernels: 64, 128, 256.  Key bits 1..4.  Value bits 2, 3, 4, 8
+ *     with group 32 or group == head_dim (the page's "token" scale layout).
+ *   - Packed rows are LSB-first bitstreams: index j of a row occupies bits [j*b, (j+1)*b) of the row read
+ *     as little-endian bytes; a row has (d*b + 7) / 8 bytes and rows are contiguous.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tq_status {
+    TQ_OK = 0,
+    TQ_ERR_INVALID_ARG = 1,   /* null pointer, negative count, misaligned pointer or stride, bad layout */
+    TQ_ERR_UNSUPPORTED = 2,   /* a head_dim / bits / group / GQA combination the kernels do not implement */
+    TQ_ERR_CUDA = 3,          /* a CUDA runtime call failed; the message carries cudaGetErrorString */
+    TQ_ERR_DEVICE_FLAG = 4    /* a kernel's bounded wait expired and it raised the device error flag */
+} tq_status;
+
+typedef enum tq_dtype {
+    TQ_F16 = 0,               /* IEEE binary16 */
+    TQ_F32 = 1                /* IEEE binary32 */
+} tq_dtype;
+
+/* Message for the last non-TQ_OK status returned on this thread ("" if none). */
+const char* tq_last_error(void);
+
+/* ABI version of this header (major * 100 + minor). */
+int tq_version(void);
+
+/* --------------------------------------------------------------------------------------------------
+ * Host parameter builders (CPU only; no device needed).
+ * ------------------------------------------------------------------------------------------------ */
+
+/*
+ * tq_make_rotation -- the seeded Haar rotation Pi ("KV Cache API", compressors.py MSECompressor.__init__:
+ * G = randn(d, d); Q, R = qr(G); Pi = Q * sign(diag R), zero signs taken as +1; "TurboQuant: A KV Cache
+ * Compression Technique", step 1, Haar-distributed orthogonal matrix).
+ *   d        head dimension, 2..1024.
+ *   seed     G[i][j] is standard normal draw i*d + j of SplitMix64(seed) through Box-Muller (pairs of
+ *            consecutive outputs u1, u2: r = sqrt(-2 ln u1'), draws r cos(2 pi u2'), r sin(2 pi u2'), with
+ *            u1' = (u1 >> 11 + 0.5) 2^-53 and u2' = (u2 >> 11) 2^-53).
+ *   pi       out, nullable: d*d doubles, row-major; the rotated vector is y = Pi x.
+ *   pi_f16   out, nullable: d*d binary16, the nearest fp16 of each entry (Pi_op, what the kernels use).
+ * Errors: TQ_ERR_INVALID_ARG for d out of range or both outputs NULL.
+ */
+tq_status tq_make_rotation(int d, uint64_t seed, double* pi, uint16_t* pi_f16);
+
+/*
+ * tq_build_codebook -- data-independent Lloyd-Max levels for one rotated coordinate ("KV Cache API",
+ * compressors.py calls _solve_codebook(head_dim, bits), body not shown; "TurboQuant: A KV Cache
+ * Compression Technique", step 2, optimal codebooks from a mathematical derivation).  The coordinate
+ * density is the exact marginal of a uniform point on the unit sphere S^(d-1):
+ * f(x) proportional to (1 - x^2)^((d-3)/2) on [-1, 1].
+ *   d, bits       2 <= d <= 65536, 1 <= bits <= 8.
+ *   centroids     out, nullable: 2^bits doubles, ascending (c*).
+ *   centroids_f16 out, nullable: 2^bits binary16, the nearest fp16 of each level (c_op).
+ *   boundaries    out, nullable: 2^bits - 1 floats, midpoints of adjacent c_op levels (exact in fp32).
+ *   distortion    out, nullable: D = E ||y - Q(y)||^2 for a uniform unit vector y quantized coordinate-wise
+ *                 with c_op and these boundaries.
+ * Errors: TQ_ERR_INVALID_ARG for d or bits out of range.
+ */
+tq_status tq_build_codebook(int d, int bits, double* centroids, uint16_t* centroids_f16,
+                            float* boundaries, double* distortion);
+
+/* --------------------------------------------------------------------------------------------------
+ * Key codec handle: Pi_op, Pi_op^T, c_op, boundaries and search tables resident on the current device.
+ * ------------------------------------------------------------------------------------------------ */
+
+typedef struct tq_codec tq_codec;
+
+/*
+ * tq_codec_create -- build the rotation and codebook for (d, k_bits, seed) on the host and upload them to
+ * the current CUDA device (synchronously, with cudaMalloc/cudaMemcpy; not a hot-path call).
+ *   d      64, 128 or 256.       k_bits 1..4.
+ *   out    receives the handle; the handle belongs to the device that was current at creation.
+ * Errors: TQ_ERR_UNSUPPORTED for other d / bits, TQ_ERR_CUDA if the device allocation fails.
+ */
+tq_status tq_codec_create(int d, int k_bits, uint64_t seed, tq_codec** out);
+
+/* Free a codec (NULL is accepted).  The caller must ensure no enqueued work still uses it. */
+tq_status tq_codec_destroy(tq_codec* codec);
+
+/* Read back a codec's parameters (any out pointer may be NULL). */
+tq_status tq_codec_info(const tq_codec* codec, int* d, int* k_bits, uint64_t* seed);
+
+/*
+ * tq_encode_k -- key encode ("KV Cache API", compressors.py MSECompressor.compress: norms, normalise,
+ * rotate, nearest centroid, pack; "aitherkvcache": fp16 [..., 128] -> uint8 [..., 64] at 4 bits + f32 norms).
+ *   x             in, device, binary16 rows: row r starts at x + r * x_row_stride (elements).  x must be
+ *                 16-byte aligned and x_row_stride a multiple of 8 with x_row_stride >= d.
+ *   n             number of rows (0 is a no-op).
+ *   slot_mapping  in, device, nullable, int64[n]: destination row of each input row in the output arrays
+ *                 (a paged pool); a negative entry skips the row.  NULL: row r goes to row r.
+ *   packed        out, device: rows of d*k_bits/8 bytes.      norms  out, device: float per row.
+ * Per row: n = ||x||_2 (fp32); y = Pi_op x / (n + 1e-8); index j = #{i : t_i < y_j}; LSB-first packing.
+ * Indices agree with the fp64 definition except where y_j lies within ~1e-6 of a boundary t_i.
+ */
+tq_status tq_encode_k(const tq_codec* codec, const void* x, int64_t n, int64_t x_row_stride,
+                      const int64_t* slot_mapping, uint8_t* packed, float* norms, void* stream);
+
+/*
+ * tq_decode_k -- key decode ("KV Cache API", compressors.py MSECompressor.decompress: centroids[idx] @ Pi,
+ * times the norm).
+ *   packed, norms in, device: n rows as written by tq_encode_k (contiguous).
+ *   out           out, device: n rows of d elements of out_dtype (TQ_F16 or TQ_F32), 16-byte aligned.
+ * x_hat = n * Pi_op^T c_op[idx], accumulated in fp32 on the tensor cores.
+ */
+tq_status tq_decode_k(const tq_codec* codec, const uint8_t* packed, const float* norms, int64_t n,
+                      void* out, int out_dtype, void* stream);
+
+/* --------------------------------------------------------------------------------------------------
+ * Value codec (no handle: the format is fully described by d, bits and group).
+ * ------------------------------------------------------------------------------------------------ */
+
+/*
+ * tq_encode_v -- grouped affine value quantizer ("KV Cache API", values.py quantize_values).
+ *   d, bits, group  d in {64,128,256}; bits in {2,3,4,8}; group 32 or d (the page's "token" layout).
+ *   x               in, device, binary16 rows with stride x_row_stride (elements; 16-byte aligned rows).
+ *   slot_mapping    as for tq_encode_k.
+ *   data            out, device: rows of (d*bits+7)/8 bytes.
+ *   scales, zeros   out, device: binary16 [rows][d/group].
+ * Per group, in IEEE fp32 with one rounding per operation and in this order:
+ *   scale = max((max - min) / (2^bits - 1), 1e-12); zero = min;
+ *   q = clamp(round_half_even((x - zero) / scale), 0, 2^bits - 1);
+ * scale and zero are then stored as fp16 (round to nearest even).  The result is bit-exact with that
+ * definition.
+ */
+tq_status tq_encode_v(int d, int bits, int group, const void* x, int64_t n, int64_t x_row_stride,
+                      const int64_t* slot_mapping, uint8_t* data, void* scales, void* zeros, void* stream);
+
+/*
+ * tq_decode_v -- value dequantization ("KV Cache API", values.py dequantize_values):
+ * x_hat = float(q) * float(scale16) + float(zero16), two fp32 operations, then stored as out_dtype
+ * (TQ_F32 exact; TQ_F16 round to nearest even).  Inputs are contiguous rows as tq_encode_v writes them.
+ */
+tq_status tq_decode_v(int d, int bits, int group, const uint8_t* data, const void* scales,
+                      const void* zeros, int64_t n, void* out, int out_dtype, void* stream);
+
+/* --------------------------------------------------------------------------------------------------
+ * Decode-step attention over the compressed cache.
+ * ------------------------------------------------------------------------------------------------ */
+
+/*
+ * Cache layouts.  Every pool array (K payload, K norms, V data, V scales, V zeros) is indexed by a row:
+ *   contiguous: row = (b * num_kv_heads + h) * max_seq_len + t;
+ *   paged:      row = (block_table[b * max_blocks + t / block_size] * num_kv_heads + h) * block_size
+ *                     + t % block_size.
+ * Sequence b attends to tokens 0 .. seq_lens[b]-1 (all max_seq_len tokens if seq_lens is NULL in the
+ * contiguous layout; seq_lens is required for the paged layout).  Query head hq reads kv head
+ * hq / (num_q_heads / num_kv_heads).
+ */
+typedef struct tq_attend_args {
+    int batch;                 /* B >= 1 */
+    int num_q_heads;           /* H_q, a multiple of num_kv_heads; H_q / H_kv <= 8 */
+    int num_kv_heads;          /* H_kv >= 1 */
+    int head_dim;              /* must equal the codec's d */
+    int v_bits;                /* 2, 3, 4 or 8 */
+    int v_group;               /* 32 or head_dim */
+    float scale;               /* softmax scale; 0 means 1/sqrt(head_dim) ("KV Cache API", attention_scores) */
+    int64_t max_seq_len;       /* contiguous layout: T per (b, h); paged: ignored */
+    const int32_t* block_table;/* NULL: contiguous layout.  Else device int32 [batch][max_blocks] */
+    int max_blocks;            /* paged: columns of block_table */
+    int block_size;            /* paged: tokens per block (16) */
+    const int32_t* seq_lens;   /* device int32 [batch], nullable in the contiguous layout */
+    const void* q;             /* device binary16 [batch][num_q_heads][head_dim] */
+    const uint8_t* k_packed;   /* device pool of key rows (tq_encode_k format) */
+    const float* k_norms;      /* device pool of key norms */
+    const uint8_t* v_data;     /* device pool of value rows (tq_encode_v format) */
+    const void* v_scales;      /* device binary16 pool [rows][head_dim / v_group] */
+    const void* v_zeros;       /* device binary16 pool [rows][head_dim / v_group] */
+    float* out;                /* device float [batch][num_q_heads][head_dim] */
+    void* workspace;           /* device scratch for split-K partials, tq_attend_workspace_bytes(args) bytes,
+                                  16-byte aligned; it must be zero-filled once before first use and is left
+                                  zero-filled (in its counter area) by every completed call */
+    size_t workspace_bytes;
+} tq_attend_args;
+
+/* Bytes of workspace tq_attend_decode needs for these arguments on the current device (0 on error). */
+size_t tq_attend_workspace_bytes(const tq_attend_args* args);
+
+/*
+ * tq_attend_decode -- one decode step of attention against the compressed cache ("KV Cache API",
+ * store.py attention_scores + softmax + attend; "turbo-attn", split-K paged decode with the query
+ * rotated once).  For each (b, hq) with h = hq / G:
+ *   q_rot = Pi_op q;  s_t = scale * n_t * <q_rot, c_op[idx_t]>;  p = softmax(s);
+ *   out = sum_t p_t * (q_t * scale16_t + zero16_t)   (the value dequantized inside the kernel).
+ * No fp16 key or value is written to memory.  A sequence of length 0 yields zeros.
+ * Concurrent calls must use distinct workspaces.
+ */
+tq_status tq_attend_decode(const tq_codec* codec, const tq_attend_args* args, void* stream);
+
+/* --------------------------------------------------------------------------------------------------
+ * Diagnostics.
+ * ------------------------------------------------------------------------------------------------ */
+
+/*
+ * Read (and optionally clear) the current device's error flag, which a kernel sets when one of its bounded
+ * waits expires.  Synchronises the device.  flag_out receives 0 when nothing was raised.
+ */
+tq_status tq_read_device_flag(int* flag_out, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

@@ -1,0 +1,543 @@
+// libtq: the C ABI of include/tq.h over the sm_100a kernels.  Host-side validation, codec lifecycle,
+// TMA descriptor creation and template dispatch live here; the kernels are in the included headers.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "tq_attend_kernel.cuh"
+#include "tq_codec_kernels.cuh"
+#include "tq_internal.h"
+
+using namespace tq;
+using namespace tq::dev;
+
+// ------------------------------------------------------------------------------------------ helpers
+
+namespace {
+
+#define TQ_CUDA(call, what)                                                                        \
+    do {                                                                                           \
+        cudaError_t e_ = (call);                                                                   \
+        if (e_ != cudaSuccess) return fail(TQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e_));    \
+    } while (0)
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int sm_count() {
+    static std::mutex mu;
+    static std::vector<int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    std::lock_guard<std::mutex> lk(mu);
+    if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1, 0);
+    if (cache[dev] == 0) {
+        int v = 0;
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = v > 0 ? v : 148;
+    }
+    return cache[dev];
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D fp16 tensor map over rows x cols (row stride in elements), 128B swizzle, box of 64 cols x box_rows.
+tq_status make_tmap_f16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t row_stride,
+                        uint32_t box_rows) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return fail(TQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {row_stride * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+    return TQ_OK;
+}
+
+// Raise the dynamic shared-memory limit of a kernel once per device.
+template <typename K>
+cudaError_t allow_smem(K kernel, uint32_t bytes, std::atomic<uint64_t>& done_mask) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done_mask.load() & bit) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (e == cudaSuccess) done_mask.fetch_or(bit);
+    return e;
+}
+
+bool supported_d(int d) { return d == 64 || d == 128 || d == 256; }
+
+}  // namespace
+
+// ------------------------------------------------------------------------------------------- codec
+
+struct tq_codec {
+    int d = 0, bits = 0, device = 0;
+    uint64_t seed = 0;
+    __half* pi_op = nullptr;        // d x d, rotated = Pi_op x
+    __half* pi_op_t = nullptr;      // Pi_op^T, the decode-side B operand
+    uint2* enc_lut = nullptr;       // 2048 grid cells {boundary bits, count below}
+    uint32_t* pair_lut = nullptr;   // 2^(2 bits) half2 pairs
+    CUtensorMap tmap_pi, tmap_pit;
+};
+
+namespace {
+
+// Grid table of the encode search (see encode_k_kernel): cell c holds the y with rint(512 y + 640) = c.
+tq_status build_grid_lut(int bits, const float* t, std::vector<uint2>& lut) {
+    const int nb = (1 << bits) - 1;
+    lut.assign(2048, make_uint2(0x7F800000u, static_cast<uint32_t>(nb)));
+    for (int c = 0; c <= 1280; ++c) {
+        const double lo = (c - 640.5) / 512.0, hi = (c - 639.5) / 512.0;
+        uint32_t below = 0;
+        int inside = 0;
+        float b = INFINITY;
+        for (int i = 0; i < nb; ++i) {
+            const double ti = t[i];
+            if (ti < lo) ++below;
+            else if (ti <= hi) { ++inside; b = t[i]; }
+        }
+        if (inside > 1) return fail(TQ_ERR_UNSUPPORTED, "codebook boundaries closer than the search grid (bits=%d)", bits);
+        uint32_t bb;
+        std::memcpy(&bb, &b, 4);
+        lut[c] = make_uint2(bb, below);
+    }
+    return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" tq_status tq_codec_create(int d, int k_bits, uint64_t seed, tq_codec** out) {
+    clear_error();
+    if (!out) return fail(TQ_ERR_INVALID_ARG, "tq_codec_create: out is NULL");
+    *out = nullptr;
+    if (!supported_d(d)) return fail(TQ_ERR_UNSUPPORTED, "tq_codec_create: d=%d (supported: 64, 128, 256)", d);
+    if (k_bits < 1 || k_bits > 4) return fail(TQ_ERR_UNSUPPORTED, "tq_codec_create: k_bits=%d (supported: 1..4)", k_bits);
+    const size_t dd = static_cast<size_t>(d) * d;
+    std::vector<uint16_t> pi16(dd), pit16(dd);
+    std::vector<double> pi(dd);
+    host_rotation(d, seed, pi.data());
+    for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j) {
+            pi16[static_cast<size_t>(i) * d + j] = f64_to_f16(pi[static_cast<size_t>(i) * d + j]);
+            pit16[static_cast<size_t>(j) * d + i] = pi16[static_cast<size_t>(i) * d + j];
+        }
+    const int k = 1 << k_bits;
+    std::vector<uint16_t> c16(k);
+    std::vector<float> t(k - 1);
+    tq_status st = tq_build_codebook(d, k_bits, nullptr, c16.data(), t.data(), nullptr);
+    if (st != TQ_OK) return st;
+    std::vector<uint2> lut;
+    if ((st = build_grid_lut(k_bits, t.data(), lut)) != TQ_OK) return st;
+    std::vector<uint32_t> pairs(1u << (2 * k_bits));
+    for (uint32_t key = 0; key < pairs.size(); ++key)
+        pairs[key] = static_cast<uint32_t>(c16[key & (k - 1)]) | (static_cast<uint32_t>(c16[key >> k_bits]) << 16);
+
+    tq_codec* c = new tq_codec();
+    c->d = d;
+    c->bits = k_bits;
+    c->seed = seed;
+    cudaGetDevice(&c->device);
+    auto cleanup = [&](tq_status s) {
+        tq_codec_destroy(c);
+        return s;
+    };
+    if (cudaMalloc(&c->pi_op, dd * 2) != cudaSuccess || cudaMalloc(&c->pi_op_t, dd * 2) != cudaSuccess ||
+        cudaMalloc(&c->enc_lut, 2048 * sizeof(uint2)) != cudaSuccess ||
+        cudaMalloc(&c->pair_lut, pairs.size() * 4) != cudaSuccess)
+        return cleanup(fail(TQ_ERR_CUDA, "tq_codec_create: cudaMalloc failed"));
+    if (cudaMemcpy(c->pi_op, pi16.data(), dd * 2, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->pi_op_t, pit16.data(), dd * 2, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->enc_lut, lut.data(), 2048 * sizeof(uint2), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->pair_lut, pairs.data(), pairs.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
+        return cleanup(fail(TQ_ERR_CUDA, "tq_codec_create: cudaMemcpy failed"));
+    if ((st = make_tmap_f16(&c->tmap_pi, c->pi_op, d, d, d, d)) != TQ_OK) return cleanup(st);
+    if ((st = make_tmap_f16(&c->tmap_pit, c->pi_op_t, d, d, d, d)) != TQ_OK) return cleanup(st);
+    *out = c;
+    return TQ_OK;
+}
+
+extern "C" tq_status tq_codec_destroy(tq_codec* c) {
+    if (!c) return TQ_OK;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(c->device);
+    cudaFree(c->pi_op);
+    cudaFree(c->pi_op_t);
+    cudaFree(c->enc_lut);
+    cudaFree(c->pair_lut);
+    cudaSetDevice(prev);
+    delete c;
+    return TQ_OK;
+}
+
+extern "C" tq_status tq_codec_info(const tq_codec* c, int* d, int* k_bits, uint64_t* seed) {
+    clear_error();
+    if (!c) return fail(TQ_ERR_INVALID_ARG, "tq_codec_info: codec is NULL");
+    if (d) *d = c->d;
+    if (k_bits) *k_bits = c->bits;
+    if (seed) *seed = c->seed;
+    return TQ_OK;
+}
+
+// ---------------------------------------------------------------------------------------- key codec
+
+namespace {
+
+template <int D, int BITS>
+tq_status launch_encode_k(const tq_codec* c, const void* x, int64_t n, int64_t stride, const int64_t* slots,
+                          uint8_t* packed, float* norms, cudaStream_t st) {
+    static std::atomic<uint64_t> mask{0};
+    constexpr uint32_t smem = enc_smem_bytes<D>();
+    auto kern = encode_k_kernel<D, BITS>;
+    TQ_CUDA(allow_smem(kern, smem, mask), "tq_encode_k: cudaFuncSetAttribute");
+    CUtensorMap tx;
+    tq_status s = make_tmap_f16(&tx, x, static_cast<uint64_t>(n), D, static_cast<uint64_t>(stride), 128);
+    if (s != TQ_OK) return s;
+    const int64_t tiles = (n + 127) / 128;
+    const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+    kern<<<grid, KeyCfg<D>::kThreads, smem, st>>>(tx, c->tmap_pi, c->enc_lut, n, slots, packed, norms);
+    TQ_CUDA(cudaGetLastError(), "tq_encode_k: launch");
+    return TQ_OK;
+}
+
+template <int D, int BITS>
+tq_status launch_decode_k(const tq_codec* c, const uint8_t* packed, const float* norms, int64_t n, void* out,
+                          int dtype, cudaStream_t st) {
+    static std::atomic<uint64_t> mask16{0}, mask32{0};
+    constexpr uint32_t smem = dec_smem_bytes<D>();
+    const int64_t tiles = (n + 127) / 128;
+    const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+    if (dtype == TQ_F32) {
+        auto kern = decode_k_kernel<D, BITS, true>;
+        TQ_CUDA(allow_smem(kern, smem, mask32), "tq_decode_k: cudaFuncSetAttribute");
+        kern<<<grid, KeyCfg<D>::kThreads, smem, st>>>(c->tmap_pit, c->pair_lut, packed, norms, n, out);
+    } else {
+        auto kern = decode_k_kernel<D, BITS, false>;
+        TQ_CUDA(allow_smem(kern, smem, mask16), "tq_decode_k: cudaFuncSetAttribute");
+        kern<<<grid, KeyCfg<D>::kThreads, smem, st>>>(c->tmap_pit, c->pair_lut, packed, norms, n, out);
+    }
+    TQ_CUDA(cudaGetLastError(), "tq_decode_k: launch");
+    return TQ_OK;
+}
+
+#define TQ_DISPATCH_DB(d, bits, FN, ...)                                                              \
+    switch ((d) * 10 + (bits)) {                                                                      \
+        case 641: return FN<64, 1>(__VA_ARGS__);                                                      \
+        case 642: return FN<64, 2>(__VA_ARGS__);                                                      \
+        case 643: return FN<64, 3>(__VA_ARGS__);                                                      \
+        case 644: return FN<64, 4>(__VA_ARGS__);                                                      \
+        case 1281: return FN<128, 1>(__VA_ARGS__);                                                    \
+        case 1282: return FN<128, 2>(__VA_ARGS__);                                                    \
+        case 1283: return FN<128, 3>(__VA_ARGS__);                                                    \
+        case 1284: return FN<128, 4>(__VA_ARGS__);                                                    \
+        case 2561: return FN<256, 1>(__VA_ARGS__);                                                    \
+        case 2562: return FN<256, 2>(__VA_ARGS__);                                                    \
+        case 2563: return FN<256, 3>(__VA_ARGS__);                                                    \
+        case 2564: return FN<256, 4>(__VA_ARGS__);                                                    \
+        default: return fail(TQ_ERR_UNSUPPORTED, "unsupported d=%d bits=%d", (d), (bits));            \
+    }
+
+}  // namespace
+
+extern "C" tq_status tq_encode_k(const tq_codec* c, const void* x, int64_t n, int64_t x_row_stride,
+                                 const int64_t* slot_mapping, uint8_t* packed, float* norms, void* stream) {
+    clear_error();
+    if (!c) return fail(TQ_ERR_INVALID_ARG, "tq_encode_k: codec is NULL");
+    if (n < 0) return fail(TQ_ERR_INVALID_ARG, "tq_encode_k: n=%lld is negative", static_cast<long long>(n));
+    if (n == 0) return TQ_OK;
+    if (n > (1ll << 31) - 256) return fail(TQ_ERR_INVALID_ARG, "tq_encode_k: n=%lld exceeds 2^31-256 rows", static_cast<long long>(n));
+    if (!x || !packed || !norms) return fail(TQ_ERR_INVALID_ARG, "tq_encode_k: x, packed and norms must be non-NULL");
+    if (!aligned(x, 16)) return fail(TQ_ERR_INVALID_ARG, "tq_encode_k: x must be 16-byte aligned");
+    if (x_row_stride < c->d || x_row_stride % 8)
+        return fail(TQ_ERR_INVALID_ARG, "tq_encode_k: x_row_stride=%lld must be >= d and a multiple of 8",
+                    static_cast<long long>(x_row_stride));
+    if (!aligned(packed, 16) || !aligned(norms, 4))
+        return fail(TQ_ERR_INVALID_ARG, "tq_encode_k: packed must be 16-byte and norms 4-byte aligned");
+    if (slot_mapping && !aligned(slot_mapping, 8)) return fail(TQ_ERR_INVALID_ARG, "tq_encode_k: slot_mapping misaligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TQ_DISPATCH_DB(c->d, c->bits, launch_encode_k, c, x, n, x_row_stride, slot_mapping, packed, norms, st);
+}
+
+extern "C" tq_status tq_decode_k(const tq_codec* c, const uint8_t* packed, const float* norms, int64_t n, void* out,
+                                 int out_dtype, void* stream) {
+    clear_error();
+    if (!c) return fail(TQ_ERR_INVALID_ARG, "tq_decode_k: codec is NULL");
+    if (n < 0) return fail(TQ_ERR_INVALID_ARG, "tq_decode_k: n=%lld is negative", static_cast<long long>(n));
+    if (out_dtype != TQ_F16 && out_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "tq_decode_k: out_dtype=%d", out_dtype);
+    if (n == 0) return TQ_OK;
+    if (!packed || !norms || !out) return fail(TQ_ERR_INVALID_ARG, "tq_decode_k: packed, norms and out must be non-NULL");
+    if (!aligned(packed, 16) || !aligned(norms, 4) || !aligned(out, 16))
+        return fail(TQ_ERR_INVALID_ARG, "tq_decode_k: packed and out must be 16-byte, norms 4-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TQ_DISPATCH_DB(c->d, c->bits, launch_decode_k, c, packed, norms, n, out, out_dtype, st);
+}
+
+// -------------------------------------------------------------------------------------- value codec
+
+namespace {
+
+int grid_for(int64_t units) {
+    const int64_t blocks = (units + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+    return static_cast<int>(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
+}
+
+template <int D, int BITS, int GROUP>
+tq_status launch_encode_v(const void* x, int64_t n, int64_t stride, const int64_t* slots, uint8_t* data, void* scales,
+                          void* zeros, cudaStream_t st) {
+    encode_v_kernel<D, BITS, GROUP><<<grid_for(n * (D / 32)), 256, 0, st>>>(
+        static_cast<const __half*>(x), n, stride, slots, data, static_cast<__half*>(scales), static_cast<__half*>(zeros));
+    TQ_CUDA(cudaGetLastError(), "tq_encode_v: launch");
+    return TQ_OK;
+}
+
+template <int D, int BITS, int GROUP>
+tq_status launch_decode_v(const uint8_t* data, const void* scales, const void* zeros, int64_t n, void* out, int dtype,
+                          cudaStream_t st) {
+    const int grid = grid_for(n * (D / 32));
+    if (dtype == TQ_F32)
+        decode_v_kernel<D, BITS, GROUP, true><<<grid, 256, 0, st>>>(data, static_cast<const __half*>(scales),
+                                                                    static_cast<const __half*>(zeros), n, out);
+    else
+        decode_v_kernel<D, BITS, GROUP, false><<<grid, 256, 0, st>>>(data, static_cast<const __half*>(scales),
+                                                                     static_cast<const __half*>(zeros), n, out);
+    TQ_CUDA(cudaGetLastError(), "tq_decode_v: launch");
+    return TQ_OK;
+}
+
+// dispatch over d in {64,128,256}, bits in {2,3,4,8}, group in {32, d}
+#define TQ_V_CASE(D_, B_, FN, ...)                                                                    \
+    case D_ * 100 + B_ * 10 + 0: return FN<D_, B_, 32>(__VA_ARGS__);                                  \
+    case D_ * 100 + B_ * 10 + 1: return FN<D_, B_, D_>(__VA_ARGS__);
+#define TQ_V_D(D_, FN, ...)                                                                           \
+    TQ_V_CASE(D_, 2, FN, __VA_ARGS__) TQ_V_CASE(D_, 3, FN, __VA_ARGS__) TQ_V_CASE(D_, 4, FN, __VA_ARGS__) \
+    TQ_V_CASE(D_, 8, FN, __VA_ARGS__)
+#define TQ_DISPATCH_V(d, bits, group, FN, ...)                                                        \
+    switch ((d) * 100 + (bits) * 10 + ((group) == (d) ? 1 : 0)) {                                     \
+        TQ_V_D(64, FN, __VA_ARGS__)                                                                   \
+        TQ_V_D(128, FN, __VA_ARGS__)                                                                  \
+        TQ_V_D(256, FN, __VA_ARGS__)                                                                  \
+        default: return fail(TQ_ERR_UNSUPPORTED, "unsupported value format d=%d bits=%d group=%d", (d), (bits), (group)); \
+    }
+
+tq_status check_v_format(const char* fn, int d, int bits, int group) {
+    if (!supported_d(d)) return fail(TQ_ERR_UNSUPPORTED, "%s: d=%d (supported: 64, 128, 256)", fn, d);
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 8)
+        return fail(TQ_ERR_UNSUPPORTED, "%s: bits=%d (value bits must be one of 2, 3, 4, 8)", fn, bits);
+    if (group != 32 && group != d) return fail(TQ_ERR_UNSUPPORTED, "%s: group=%d (32 or d)", fn, group);
+    return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" tq_status tq_encode_v(int d, int bits, int group, const void* x, int64_t n, int64_t x_row_stride,
+                                 const int64_t* slot_mapping, uint8_t* data, void* scales, void* zeros, void* stream) {
+    clear_error();
+    tq_status s = check_v_format("tq_encode_v", d, bits, group);
+    if (s != TQ_OK) return s;
+    if (n < 0) return fail(TQ_ERR_INVALID_ARG, "tq_encode_v: n=%lld is negative", static_cast<long long>(n));
+    if (n == 0) return TQ_OK;
+    if (!x || !data || !scales || !zeros) return fail(TQ_ERR_INVALID_ARG, "tq_encode_v: NULL pointer argument");
+    if (!aligned(x, 16) || x_row_stride < d || x_row_stride % 8)
+        return fail(TQ_ERR_INVALID_ARG, "tq_encode_v: x must be 16-byte aligned with x_row_stride >= d, a multiple of 8");
+    if (!aligned(data, 16) || !aligned(scales, 2) || !aligned(zeros, 2))
+        return fail(TQ_ERR_INVALID_ARG, "tq_encode_v: data must be 16-byte aligned");
+    if (slot_mapping && !aligned(slot_mapping, 8)) return fail(TQ_ERR_INVALID_ARG, "tq_encode_v: slot_mapping misaligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TQ_DISPATCH_V(d, bits, group, launch_encode_v, x, n, x_row_stride, slot_mapping, data, scales, zeros, st);
+}
+
+extern "C" tq_status tq_decode_v(int d, int bits, int group, const uint8_t* data, const void* scales, const void* zeros,
+                                 int64_t n, void* out, int out_dtype, void* stream) {
+    clear_error();
+    tq_status s = check_v_format("tq_decode_v", d, bits, group);
+    if (s != TQ_OK) return s;
+    if (n < 0) return fail(TQ_ERR_INVALID_ARG, "tq_decode_v: n=%lld is negative", static_cast<long long>(n));
+    if (out_dtype != TQ_F16 && out_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "tq_decode_v: out_dtype=%d", out_dtype);
+    if (n == 0) return TQ_OK;
+    if (!data || !scales || !zeros || !out) return fail(TQ_ERR_INVALID_ARG, "tq_decode_v: NULL pointer argument");
+    if (!aligned(data, 16) || !aligned(out, 16) || !aligned(scales, 2) || !aligned(zeros, 2))
+        return fail(TQ_ERR_INVALID_ARG, "tq_decode_v: data and out must be 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TQ_DISPATCH_V(d, bits, group, launch_decode_v, data, scales, zeros, n, out, out_dtype, st);
+}
+
+// ---------------------------------------------------------------------------------------- attention
+
+namespace {
+
+constexpr int kAttendCtasPerSm = 3;
+
+struct AttendPlan {
+    int num_splits;
+    size_t counter_bytes, partial_bytes;
+};
+
+tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan) {
+    if (!a) return fail(TQ_ERR_INVALID_ARG, "tq_attend: args is NULL");
+    if (a->batch < 1 || a->num_kv_heads < 1 || a->num_q_heads < 1)
+        return fail(TQ_ERR_INVALID_ARG, "tq_attend: batch, num_q_heads, num_kv_heads must be >= 1");
+    if (a->num_q_heads % a->num_kv_heads)
+        return fail(TQ_ERR_INVALID_ARG, "tq_attend: num_q_heads=%d is not a multiple of num_kv_heads=%d", a->num_q_heads,
+                    a->num_kv_heads);
+    if (a->num_q_heads / a->num_kv_heads > 8)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_attend: GQA group %d > 8", a->num_q_heads / a->num_kv_heads);
+    if (!supported_d(a->head_dim)) return fail(TQ_ERR_UNSUPPORTED, "tq_attend: head_dim=%d", a->head_dim);
+    tq_status s = check_v_format("tq_attend", a->head_dim, a->v_bits, a->v_group);
+    if (s != TQ_OK) return s;
+    int64_t max_chunks;
+    if (a->block_table) {
+        if (a->block_size != 16) return fail(TQ_ERR_UNSUPPORTED, "tq_attend: block_size=%d (supported: 16)", a->block_size);
+        if (a->max_blocks < 1) return fail(TQ_ERR_INVALID_ARG, "tq_attend: max_blocks=%d", a->max_blocks);
+        if (!a->seq_lens) return fail(TQ_ERR_INVALID_ARG, "tq_attend: the paged layout needs seq_lens");
+        max_chunks = a->max_blocks;
+    } else {
+        if (a->max_seq_len < 0 || a->max_seq_len % 16)
+            return fail(TQ_ERR_INVALID_ARG, "tq_attend: max_seq_len=%lld must be a non-negative multiple of 16",
+                        static_cast<long long>(a->max_seq_len));
+        max_chunks = a->max_seq_len / 16;
+    }
+    const int64_t bh = static_cast<int64_t>(a->batch) * a->num_kv_heads;
+    int64_t splits = (static_cast<int64_t>(sm_count()) * kAttendCtasPerSm + bh - 1) / bh;
+    const int64_t by_len = (max_chunks + 7) / 8;            // at least ~8 chunks (128 tokens) per split
+    if (splits > by_len) splits = by_len;
+    if (splits > 1024) splits = 1024;
+    if (splits < 1) splits = 1;
+    plan->num_splits = static_cast<int>(splits);
+    plan->counter_bytes = ((static_cast<size_t>(bh) * 4 + 255) / 256) * 256;
+    plan->partial_bytes = (splits > 1) ? static_cast<size_t>(bh) * splits * (16 + 8 * a->head_dim) * 4 : 0;
+    return TQ_OK;
+}
+
+template <int D, int KB, int VB, int VG>
+tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const AttendPlan& plan, cudaStream_t st) {
+    using Cfg = AttCfg<D, KB, VB, VG>;
+    static std::atomic<uint64_t> mask{0};
+    auto kern = attend_kernel<D, KB, VB, VG>;
+    TQ_CUDA(allow_smem(kern, Cfg::kSmem, mask), "tq_attend_decode: cudaFuncSetAttribute");
+    AttendParams p;
+    p.batch = a->batch;
+    p.num_q_heads = a->num_q_heads;
+    p.num_kv_heads = a->num_kv_heads;
+    p.group = a->num_q_heads / a->num_kv_heads;
+    const float scale = (a->scale == 0.f) ? 1.0f / std::sqrt(static_cast<float>(D)) : a->scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.max_seq_len = a->max_seq_len;
+    p.block_table = a->block_table;
+    p.max_blocks = a->max_blocks;
+    p.seq_lens = a->seq_lens;
+    p.q = static_cast<const __half*>(a->q);
+    p.pi_op = c->pi_op;
+    p.pair_lut = c->pair_lut;
+    p.k_packed = a->k_packed;
+    p.k_norms = a->k_norms;
+    p.v_data = a->v_data;
+    p.v_scales = static_cast<const __half*>(a->v_scales);
+    p.v_zeros = static_cast<const __half*>(a->v_zeros);
+    p.out = a->out;
+    p.counters = static_cast<int*>(a->workspace);
+    p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(a->workspace) + plan.counter_bytes);
+    p.num_splits = plan.num_splits;
+    dim3 grid(plan.num_splits, a->num_kv_heads, a->batch);
+    kern<<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(p);
+    TQ_CUDA(cudaGetLastError(), "tq_attend_decode: launch");
+    return TQ_OK;
+}
+
+template <int D, int KB>
+tq_status attend_v(const tq_codec* c, const tq_attend_args* a, const AttendPlan& plan, cudaStream_t st) {
+    const bool tok = a->v_group == D;
+    switch (a->v_bits * 2 + (tok ? 1 : 0)) {
+        case 4: return launch_attend<D, KB, 2, 32>(c, a, plan, st);
+        case 5: return launch_attend<D, KB, 2, D>(c, a, plan, st);
+        case 6: return launch_attend<D, KB, 3, 32>(c, a, plan, st);
+        case 7: return launch_attend<D, KB, 3, D>(c, a, plan, st);
+        case 8: return launch_attend<D, KB, 4, 32>(c, a, plan, st);
+        case 9: return launch_attend<D, KB, 4, D>(c, a, plan, st);
+        case 16: return launch_attend<D, KB, 8, 32>(c, a, plan, st);
+        case 17: return launch_attend<D, KB, 8, D>(c, a, plan, st);
+        default: return fail(TQ_ERR_UNSUPPORTED, "tq_attend_decode: v_bits=%d", a->v_bits);
+    }
+}
+
+}  // namespace
+
+extern "C" size_t tq_attend_workspace_bytes(const tq_attend_args* a) {
+    clear_error();
+    AttendPlan plan;
+    if (plan_attend(a, &plan) != TQ_OK) return 0;
+    return plan.counter_bytes + plan.partial_bytes;
+}
+
+extern "C" tq_status tq_attend_decode(const tq_codec* c, const tq_attend_args* a, void* stream) {
+    clear_error();
+    if (!c) return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: codec is NULL");
+    AttendPlan plan;
+    tq_status s = plan_attend(a, &plan);
+    if (s != TQ_OK) return s;
+    if (a->head_dim != c->d) return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: head_dim=%d but the codec has d=%d", a->head_dim, c->d);
+    if (!a->q || !a->k_packed || !a->k_norms || !a->v_data || !a->v_scales || !a->v_zeros || !a->out || !a->workspace)
+        return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: NULL pointer in args");
+    if (a->workspace_bytes < plan.counter_bytes + plan.partial_bytes)
+        return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: workspace_bytes=%zu < %zu required", a->workspace_bytes,
+                    plan.counter_bytes + plan.partial_bytes);
+    if (!aligned(a->q, 16) || !aligned(a->k_packed, 16) || !aligned(a->k_norms, 16) || !aligned(a->v_data, 16) ||
+        !aligned(a->v_scales, 16) || !aligned(a->v_zeros, 16) || !aligned(a->out, 16) || !aligned(a->workspace, 16))
+        return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: every pointer must be 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (c->d * 10 + c->bits) {
+        case 641: return attend_v<64, 1>(c, a, plan, st);
+        case 642: return attend_v<64, 2>(c, a, plan, st);
+        case 643: return attend_v<64, 3>(c, a, plan, st);
+        case 644: return attend_v<64, 4>(c, a, plan, st);
+        case 1281: return attend_v<128, 1>(c, a, plan, st);
+        case 1282: return attend_v<128, 2>(c, a, plan, st);
+        case 1283: return attend_v<128, 3>(c, a, plan, st);
+        case 1284: return attend_v<128, 4>(c, a, plan, st);
+        case 2561: return attend_v<256, 1>(c, a, plan, st);
+        case 2562: return attend_v<256, 2>(c, a, plan, st);
+        case 2563: return attend_v<256, 3>(c, a, plan, st);
+        case 2564: return attend_v<256, 4>(c, a, plan, st);
+        default: return fail(TQ_ERR_UNSUPPORTED, "tq_attend_decode: d=%d bits=%d", c->d, c->bits);
+    }
+}
+
+// --------------------------------------------------------------------------------------- diagnostics
+
+extern "C" tq_status tq_read_device_flag(int* flag_out, int clear) {
+    clear_error();
+    if (!flag_out) return fail(TQ_ERR_INVALID_ARG, "tq_read_device_flag: flag_out is NULL");
+    TQ_CUDA(cudaDeviceSynchronize(), "tq_read_device_flag: cudaDeviceSynchronize");
+    unsigned v = 0;
+    TQ_CUDA(cudaMemcpyFromSymbol(&v, g_error_flag, sizeof(v)), "tq_read_device_flag: read");
+    *flag_out = static_cast<int>(v);
+    if (clear) {
+        unsigned z = 0;
+        TQ_CUDA(cudaMemcpyToSymbol(g_error_flag, &z, sizeof(z)), "tq_read_device_flag: clear");
+    }
+    return TQ_OK;
+}

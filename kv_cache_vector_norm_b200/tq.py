@@ -1,0 +1,291 @@
+"""Python binding of libtq (include/tq.h): argument marshalling only.
+
+Every computation runs in the library's CUDA kernels (or, for tq_make_rotation / tq_build_codebook, in
+its host C++).  PyTorch provides device memory and the current stream.  If libtq.so is missing this
+module raises at import time -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtq.so")
+
+TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_DEVICE_FLAG = range(5)
+TQ_F16, TQ_F32 = 0, 1
+
+_c_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+class AttendArgs(ctypes.Structure):
+    """Mirror of tq_attend_args."""
+    _fields_ = [
+        ("batch", ctypes.c_int), ("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int), ("v_bits", ctypes.c_int), ("v_group", ctypes.c_int),
+        ("scale", ctypes.c_float), ("max_seq_len", ctypes.c_int64),
+        ("block_table", ctypes.c_void_p), ("max_blocks", ctypes.c_int), ("block_size", ctypes.c_int),
+        ("seq_lens", ctypes.c_void_p), ("q", ctypes.c_void_p), ("k_packed", ctypes.c_void_p),
+        ("k_norms", ctypes.c_void_p), ("v_data", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+        ("v_zeros", ctypes.c_void_p), ("out", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+# name -> (restype, argtypes)
+SIGNATURES = {
+    "tq_last_error": (ctypes.c_char_p, []),
+    "tq_version": (ctypes.c_int, []),
+    "tq_make_rotation": (ctypes.c_int, [ctypes.c_int, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]),
+    "tq_build_codebook": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p]),
+    "tq_codec_create": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_uint64, ctypes.POINTER(ctypes.c_void_p)]),
+    "tq_codec_destroy": (ctypes.c_int, [ctypes.c_void_p]),
+    "tq_codec_info": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "tq_encode_k": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "tq_decode_k": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                   ctypes.c_int, ctypes.c_void_p]),
+    "tq_encode_v": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64,
+                                   ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_void_p]),
+    "tq_decode_v": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
+    "tq_attend_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(AttendArgs)]),
+    "tq_attend_decode": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs), ctypes.c_void_p]),
+    "tq_read_device_flag": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), ctypes.c_int]),
+}
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libtq.so not found at {LIB_PATH}; build it with "
+                          "`python -m kv_cache_vector_norm_b200._build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+
+class TQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = LIB.tq_last_error().decode(errors="replace")
+        super().__init__(f"{fn} failed with status {status}: {msg}")
+
+
+def _check(fn: str, status: int):
+    if status != TQ_OK:
+        raise TQError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device=None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+
+
+# ------------------------------------------------------------------------------- host parameters
+
+def make_rotation(d: int, seed: int):
+    """(Pi fp64 [d, d], Pi_op fp16 [d, d]) from tq_make_rotation."""
+    pi = np.empty((d, d), np.float64)
+    pi16 = np.empty((d, d), np.uint16)
+    _check("tq_make_rotation", LIB.tq_make_rotation(d, seed, pi.ctypes.data, pi16.ctypes.data))
+    return pi, pi16.view(np.float16)
+
+
+def build_codebook(d: int, bits: int):
+    """dict(centroids fp64, centroids_f16, boundaries f32, distortion) from tq_build_codebook."""
+    k = 1 << bits
+    c = np.empty(k, np.float64)
+    c16 = np.empty(k, np.uint16)
+    t = np.empty(max(k - 1, 1), np.float32)
+    dist = ctypes.c_double()
+    _check("tq_build_codebook", LIB.tq_build_codebook(d, bits, c.ctypes.data, c16.ctypes.data, t.ctypes.data,
+                                                      ctypes.byref(dist)))
+    return {"centroids": c, "centroids_f16": c16.view(np.float16), "boundaries": t[:k - 1], "distortion": dist.value}
+
+
+# ------------------------------------------------------------------------------------ key codec
+
+class Codec:
+    """A key codec (rotation + codebook resident on the current CUDA device)."""
+
+    def __init__(self, d: int, bits: int, seed: int = 0):
+        h = ctypes.c_void_p()
+        _check("tq_codec_create", LIB.tq_codec_create(d, bits, seed, ctypes.byref(h)))
+        self._h = h
+        self.d, self.bits, self.seed = d, bits, seed
+        self.row_bytes = d * bits // 8
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            LIB.tq_codec_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def encode_k(self, x: torch.Tensor, slot_mapping: torch.Tensor | None = None,
+                 packed: torch.Tensor | None = None, norms: torch.Tensor | None = None):
+        """x: [N, d] fp16 (row stride a multiple of 8).  Returns (packed u8 [rows, d*b/8], norms f32 [rows])."""
+        _need_cuda(x, "x", torch.float16)
+        if x.dim() != 2 or x.shape[1] != self.d or x.stride(1) != 1:
+            raise ValueError(f"x must be [N, {self.d}] with unit column stride")
+        n = x.shape[0]
+        if packed is None:
+            packed = torch.empty((n, self.row_bytes), dtype=torch.uint8, device=x.device)
+        if norms is None:
+            norms = torch.empty((packed.shape[0],), dtype=torch.float32, device=x.device)
+        if slot_mapping is not None:
+            _need_cuda(slot_mapping, "slot_mapping", torch.int64)
+        _check("tq_encode_k", LIB.tq_encode_k(self._h, _ptr(x), n, x.stride(0), _ptr(slot_mapping), _ptr(packed),
+                                              _ptr(norms), _stream(x.device)))
+        return packed, norms
+
+    def decode_k(self, packed: torch.Tensor, norms: torch.Tensor, out_dtype=torch.float16,
+                 out: torch.Tensor | None = None):
+        _need_cuda(packed, "packed", torch.uint8)
+        _need_cuda(norms, "norms", torch.float32)
+        n = packed.shape[0]
+        if out is None:
+            out = torch.empty((n, self.d), dtype=out_dtype, device=packed.device)
+        dt = TQ_F32 if out.dtype == torch.float32 else TQ_F16
+        _check("tq_decode_k", LIB.tq_decode_k(self._h, _ptr(packed), _ptr(norms), n, _ptr(out), dt,
+                                              _stream(packed.device)))
+        return out
+
+
+# ---------------------------------------------------------------------------------- value codec
+
+def v_row_bytes(d: int, bits: int) -> int:
+    return (d * bits + 7) // 8
+
+
+def encode_v(x: torch.Tensor, bits: int, group: int = 32, slot_mapping: torch.Tensor | None = None,
+             data: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+             zeros: torch.Tensor | None = None):
+    """x: [N, d] fp16.  Returns (data u8 [rows, (d*b+7)/8], scales f16 [rows, d/group], zeros f16)."""
+    _need_cuda(x, "x", torch.float16)
+    n, d = x.shape
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit column stride")
+    g = d // group
+    if data is None:
+        data = torch.empty((n, v_row_bytes(d, bits)), dtype=torch.uint8, device=x.device)
+    rows = data.shape[0]
+    if scales is None:
+        scales = torch.empty((rows, g), dtype=torch.float16, device=x.device)
+    if zeros is None:
+        zeros = torch.empty((rows, g), dtype=torch.float16, device=x.device)
+    if slot_mapping is not None:
+        _need_cuda(slot_mapping, "slot_mapping", torch.int64)
+    _check("tq_encode_v", LIB.tq_encode_v(d, bits, group, _ptr(x), n, x.stride(0), _ptr(slot_mapping), _ptr(data),
+                                          _ptr(scales), _ptr(zeros), _stream(x.device)))
+    return data, scales, zeros
+
+
+def decode_v(data: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, d: int, bits: int, group: int = 32,
+             out_dtype=torch.float16, out: torch.Tensor | None = None):
+    _need_cuda(data, "data", torch.uint8)
+    n = data.shape[0]
+    if out is None:
+        out = torch.empty((n, d), dtype=out_dtype, device=data.device)
+    dt = TQ_F32 if out.dtype == torch.float32 else TQ_F16
+    _check("tq_decode_v", LIB.tq_decode_v(d, bits, group, _ptr(data), _ptr(scales), _ptr(zeros), n, _ptr(out), dt,
+                                          _stream(data.device)))
+    return out
+
+
+# ------------------------------------------------------------------------------------ attention
+
+@dataclass
+class Cache:
+    """Device pools of one layer's compressed cache (rows in the layouts of tq.h)."""
+    k_packed: torch.Tensor
+    k_norms: torch.Tensor
+    v_data: torch.Tensor
+    v_scales: torch.Tensor
+    v_zeros: torch.Tensor
+
+
+def _attend_args(codec: Codec, q, cache: Cache, *, num_kv_heads, v_bits, v_group, max_seq_len, block_table,
+                 seq_lens, scale, out, workspace):
+    b, hq, d = q.shape
+    a = AttendArgs()
+    a.batch, a.num_q_heads, a.num_kv_heads, a.head_dim = b, hq, num_kv_heads, d
+    a.v_bits, a.v_group, a.scale = v_bits, v_group, float(scale)
+    a.max_seq_len = int(max_seq_len or 0)
+    a.block_table = block_table.data_ptr() if block_table is not None else None
+    a.max_blocks = block_table.shape[1] if block_table is not None else 0
+    a.block_size = 16 if block_table is not None else 0
+    a.seq_lens = seq_lens.data_ptr() if seq_lens is not None else None
+    a.q = q.data_ptr()
+    a.k_packed, a.k_norms = cache.k_packed.data_ptr(), cache.k_norms.data_ptr()
+    a.v_data, a.v_scales, a.v_zeros = cache.v_data.data_ptr(), cache.v_scales.data_ptr(), cache.v_zeros.data_ptr()
+    a.out = out.data_ptr() if out is not None else None
+    a.workspace = workspace.data_ptr() if workspace is not None else None
+    a.workspace_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return a
+
+
+def attend_workspace_bytes(codec: Codec, q, cache: Cache, **kw) -> int:
+    a = _attend_args(codec, q, cache, out=None, workspace=None, **kw)
+    nb = LIB.tq_attend_workspace_bytes(ctypes.byref(a))
+    if nb == 0:
+        raise TQError("tq_attend_workspace_bytes", TQ_ERR_INVALID_ARG)
+    return nb
+
+
+def attend_workspace(codec: Codec, q, cache: Cache, **kw) -> torch.Tensor:
+    """A zero-filled workspace of the size tq_attend_workspace_bytes asks for."""
+    return torch.zeros(attend_workspace_bytes(codec, q, cache, **kw), dtype=torch.uint8, device=q.device)
+
+
+def attend_decode(codec: Codec, q: torch.Tensor, cache: Cache, *, num_kv_heads: int, v_bits: int, v_group: int = 32,
+                  max_seq_len: int | None = None, block_table: torch.Tensor | None = None,
+                  seq_lens: torch.Tensor | None = None, scale: float = 0.0, out: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """One decode step: q [B, H_q, d] fp16 against the compressed cache.  Returns out [B, H_q, d] f32."""
+    _need_cuda(q, "q", torch.float16)
+    kw = dict(num_kv_heads=num_kv_heads, v_bits=v_bits, v_group=v_group, max_seq_len=max_seq_len,
+              block_table=block_table, seq_lens=seq_lens, scale=scale)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = attend_workspace(codec, q, cache, **kw)
+    a = _attend_args(codec, q, cache, out=out, workspace=workspace, **kw)
+    _check("tq_attend_decode", LIB.tq_attend_decode(codec.handle, ctypes.byref(a), _stream(q.device)))
+    return out
+
+
+def read_device_flag(clear: bool = True) -> int:
+    v = ctypes.c_int()
+    _check("tq_read_device_flag", LIB.tq_read_device_flag(ctypes.byref(v), 1 if clear else 0))
+    return v.value

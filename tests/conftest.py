@@ -1,4 +1,5 @@
-"""Shared pytest setup: the ``gpu`` marker and the repository root on sys.path."""
+"""Shared pytest setup: the ``gpu`` marker, the repository root on sys.path, and an in-tree build of
+libtq.so when it is missing or older than its sources (nvcc cross-compiles without a GPU)."""
 import os
 import sys
 
@@ -9,4 +10,6 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (sm_100a) and the built libtq")
-    config.addinivalue_line("markers", "slow: long CPU-side case")
+    from kv_cache_vector_norm_b200 import _build
+    if _build.needs_build():
+        _build.build()
