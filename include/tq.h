@@ -200,14 +200,18 @@ typedef struct tq_attend_args {
     const void* v_scales;      /* device binary16 pool [rows][head_dim / v_group] */
     const void* v_zeros;       /* device binary16 pool [rows][head_dim / v_group] */
     float* out;                /* device float [batch][num_q_heads][head_dim] */
-    void* workspace;           /* device scratch for split-K partials, tq_attend_workspace_bytes(args) bytes,
-                                  16-byte aligned; it must be zero-filled once before first use and is left
-                                  zero-filled (in its counter area) by every completed call */
+    void* workspace;           /* device scratch for split-K partials (16-byte aligned) of at least the size
+                                  tq_attend_workspace_bytes reports; may be NULL when that size is 0.  Its
+                                  contents need no initialisation and are overwritten by every call. */
     size_t workspace_bytes;
 } tq_attend_args;
 
-/* Bytes of workspace tq_attend_decode needs for these arguments on the current device (0 on error). */
-size_t tq_attend_workspace_bytes(const tq_attend_args* args);
+/*
+ * tq_attend_workspace_bytes -- bytes of workspace tq_attend_decode needs for these arguments on the current
+ * device (0 when the launch needs no split-K partials).  Only the shape fields of args are read.
+ * Errors: the same argument checks as tq_attend_decode (TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED).
+ */
+tq_status tq_attend_workspace_bytes(const tq_attend_args* args, size_t* bytes);
 
 /*
  * tq_attend_decode -- one decode step of attention against the compressed cache ("KV Cache API",
@@ -215,8 +219,10 @@ size_t tq_attend_workspace_bytes(const tq_attend_args* args);
  * rotated once).  For each (b, hq) with h = hq / G:
  *   q_rot = Pi_op q;  s_t = scale * n_t * <q_rot, c_op[idx_t]>;  p = softmax(s);
  *   out = sum_t p_t * (q_t * scale16_t + zero16_t)   (the value dequantized inside the kernel).
- * No fp16 key or value is written to memory.  A sequence of length 0 yields zeros.
- * Concurrent calls must use distinct workspaces.
+ * No fp16 key or value is written to memory.  A sequence of length 0 yields zeros.  When the sequence axis
+ * is split over several CTAs, a second kernel (a programmatic dependent launch on the same stream) merges
+ * the per-split partials with a log-sum-exp rescale.  Calls that overlap on the GPU must use distinct
+ * workspaces.
  */
 tq_status tq_attend_decode(const tq_codec* codec, const tq_attend_args* args, void* stream);
 

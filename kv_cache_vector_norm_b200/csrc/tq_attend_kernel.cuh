@@ -36,7 +36,6 @@ struct AttendParams {
     const __half* v_zeros;
     float* out;
     float* partials;                                 // [B][H_kv][splits][16 + 8 d]
-    int* counters;                                   // [B][H_kv]
     int num_splits;
 };
 
@@ -45,33 +44,38 @@ struct AttCfg {
     static constexpr int kWarps = 4;                 // consumer warps
     static constexpr int kThreads = 32 * (kWarps + 1);
     static constexpr int kChunkTok = 16;             // tokens per chunk (= one paged block)
+    static constexpr int kTileTok = kWarps * kChunkTok;
     static constexpr int kStages = 4;
     static constexpr int kKRow = D * KB / 8;
     static constexpr int kVRow = D * VB / 8;
     static constexpr int kVGroups = D / VG;
+    // one stage holds the tile's 64 tokens array by array; chunk c of an array starts at c * 16 rows
     static constexpr int kKOff = 0;
-    static constexpr int kNOff = kKOff + kChunkTok * kKRow;
-    static constexpr int kVOff = kNOff + kChunkTok * 4;
-    static constexpr int kSOff = kVOff + kChunkTok * kVRow;
-    static constexpr int kZOff = kSOff + kChunkTok * kVGroups * 2;
-    static constexpr int kChunkBytes = kZOff + kChunkTok * kVGroups * 2;
-    static constexpr int kStageBytes = kWarps * kChunkBytes;
+    static constexpr int kNOff = kKOff + kTileTok * kKRow;
+    static constexpr int kVOff = kNOff + kTileTok * 4;
+    static constexpr int kSOff = kVOff + kTileTok * kVRow;
+    static constexpr int kZOff = kSOff + kTileTok * kVGroups * 2;
+    static constexpr int kStageBytes = kZOff + kTileTok * kVGroups * 2;
     static constexpr int kQuarterBits = D * KB / 4;  // one lane's quarter of a key row (16-bit multiple)
     static constexpr int kQuarterHalves = kQuarterBits / 16;
     static constexpr int kQuarterWords = (kQuarterHalves + 1) / 2 + 1;
     static constexpr int kMinBlocks = (D == 256) ? 1 : 3;
     static constexpr int kPartFloats = 16 + 8 * D;
-    // shared memory: stages | q fragments | rotated q | pair lut | reduction | barriers
+    // key lookups: 4 codes -> two half2 (KB <= 3), else 2 codes -> one half2
+    static constexpr bool kQuad = (KB <= 3);
+    static constexpr int kLutBytes = kQuad ? (1 << (4 * KB)) * 8 : (1 << (2 * KB)) * 4;
+    // shared memory: stages | q fragments | rotated q | key table | pair table | reduction | barriers
     static constexpr int kCombineFloats = kWarps * kPartFloats;
     static constexpr int kRingBytes =
         (kStages * kStageBytes > kCombineFloats * 4) ? kStages * kStageBytes : kCombineFloats * 4;
     static constexpr int kQfOff = kRingBytes;
     static constexpr int kQrOff = kQfOff + (D / 16) * 32 * 16;
     static constexpr int kLutOff = kQrOff + 8 * D * 4;
-    static constexpr int kRedOff = kLutOff + (1 << (2 * KB)) * 4;
+    static constexpr int kPairOff = kLutOff + kLutBytes;
+    static constexpr int kRedOff = kPairOff + (1 << (2 * KB)) * 4;
     static constexpr int kBarOff = (kRedOff + 8 * 4 + 15) & ~15;
     static constexpr int kSmem = kBarOff + 8 * (2 * kStages) + 16;
-    static_assert(kChunkBytes % 16 == 0 && kNOff % 16 == 0 && kVOff % 16 == 0 && kSOff % 16 == 0 && kZOff % 16 == 0,
+    static_assert(kNOff % 16 == 0 && kVOff % 16 == 0 && kSOff % 16 == 0 && kZOff % 16 == 0 && kStageBytes % 16 == 0,
                   "bulk copies need 16-byte multiples");
 };
 
@@ -108,32 +112,77 @@ __device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t& hi, uin
     lo = pack_bf16(x0 - h0, x1 - h1);
 }
 
-// bf16x2 {code[token a][col], code[token b][col]} of the value codes (exact small integers).
+// Value codes of one 32-column slice of a row: 32 * VB bits as words.
 template <int VB>
-__device__ __forceinline__ uint32_t vcode_pair(const uint8_t* row_a, const uint8_t* row_b, int col) {
+struct VSlice {
+    static constexpr int kWords = VB;            // 32 columns x VB bits = VB words
+};
+
+template <int VB>
+__device__ __forceinline__ void load_vslice(const uint8_t* row, int slice, uint32_t (&w)[VB]) {
+    const uint8_t* p = row + slice * 4 * VB;     // 32 * VB bits = 4 * VB bytes, 4-byte aligned
+    if constexpr (VB == 2) {
+        const uint2 t = *reinterpret_cast<const uint2*>(p);
+        w[0] = t.x; w[1] = t.y;
+    } else if constexpr (VB == 4) {
+        const uint4 t = *reinterpret_cast<const uint4*>(p);
+        w[0] = t.x; w[1] = t.y; w[2] = t.z; w[3] = t.w;
+    } else if constexpr (VB == 8) {
+        const uint4 t0 = reinterpret_cast<const uint4*>(p)[0], t1 = reinterpret_cast<const uint4*>(p)[1];
+        w[0] = t0.x; w[1] = t0.y; w[2] = t0.z; w[3] = t0.w; w[4] = t1.x; w[5] = t1.y; w[6] = t1.z; w[7] = t1.w;
+    } else {
+#pragma unroll
+        for (int i = 0; i < VB; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
+    }
+}
+
+// bf16x2 {code_a[c], code_b[c]} for column c (0..31) of a slice held in registers (exact small integers).
+template <int VB>
+__device__ __forceinline__ uint32_t vcode_pair(const uint32_t (&wa)[VB], const uint32_t (&wb)[VB], int c) {
+    const int bit = c * VB;
     if constexpr (VB == 2 || VB == 4) {
-        const int bit = col * VB;
-        const uint32_t wa = *reinterpret_cast<const uint32_t*>(row_a + (bit >> 5) * 4);
-        const uint32_t wb = *reinterpret_cast<const uint32_t*>(row_b + (bit >> 5) * 4);
+        const uint32_t a = wa[bit >> 5], b = wb[bit >> 5];
         const int sh = bit & 31;
         // put the 16-bit halves holding the field side by side, then mask into a bf16 magic of 128
-        const uint32_t z = (sh < 16) ? __byte_perm(wa, wb, 0x5410) : __byte_perm(wa, wb, 0x7632);
+        const uint32_t z = (sh < 16) ? __byte_perm(a, b, 0x5410) : __byte_perm(a, b, 0x7632);
         const uint32_t m = (VB == 2) ? 0x00030003u : 0x000F000Fu;
         const uint32_t v = ((z >> (sh & 15)) & m) | 0x43004300u;
         __nv_bfloat162 r = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&v), __floats2bfloat162_rn(128.f, 128.f));
         return *reinterpret_cast<uint32_t*>(&r);
-    } else if constexpr (VB == 8) {
-        return pack_bf16(static_cast<float>(row_a[col]), static_cast<float>(row_b[col]));
     } else {
-        const int bit = col * VB, byte = bit >> 3, sh = bit & 7;
-        uint32_t qa = row_a[byte], qb = row_b[byte];
-        if (sh + VB > 8) {
-            qa |= static_cast<uint32_t>(row_a[byte + 1]) << 8;
-            qb |= static_cast<uint32_t>(row_b[byte + 1]) << 8;
+        const int wi = bit >> 5, sh = bit & 31;
+        uint32_t qa = wa[wi] >> sh, qb = wb[wi] >> sh;
+        if (sh + VB > 32) {
+            qa |= wa[wi + 1] << (32 - sh);
+            qb |= wb[wi + 1] << (32 - sh);
         }
-        qa = (qa >> sh) & ((1u << VB) - 1u);
-        qb = (qb >> sh) & ((1u << VB) - 1u);
+        qa &= (1u << VB) - 1u;
+        qb &= (1u << VB) - 1u;
         return pack_bf16(static_cast<float>(qa), static_cast<float>(qb));
+    }
+}
+
+// n fp16 values at p (n in {1, 2, 4, 8}, naturally aligned) as floats
+template <int N>
+__device__ __forceinline__ void load_halves(const __half* p, float (&o)[N]) {
+    if constexpr (N == 1) {
+        o[0] = __half2float(p[0]);
+    } else if constexpr (N == 2) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(p));
+        o[0] = f.x; o[1] = f.y;
+    } else if constexpr (N == 4) {
+        const uint2 t = *reinterpret_cast<const uint2*>(p);
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&t.x));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&t.y));
+        o[0] = f0.x; o[1] = f0.y; o[2] = f1.x; o[3] = f1.y;
+    } else {
+        const uint4 t = *reinterpret_cast<const uint4*>(p);
+        const uint32_t u[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u[k]));
+            o[2 * k] = f.x; o[2 * k + 1] = f.y;
+        }
     }
 }
 
@@ -148,7 +197,7 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
     extern __shared__ __align__(16) uint8_t smem[];
     uint4* s_qf = reinterpret_cast<uint4*>(smem + C::kQfOff);
     float* s_qr = reinterpret_cast<float*>(smem + C::kQrOff);
-    uint32_t* s_lut = reinterpret_cast<uint32_t*>(smem + C::kLutOff);
+    uint32_t* s_pair = reinterpret_cast<uint32_t*>(smem + C::kPairOff);
     float* s_red = reinterpret_cast<float*>(smem + C::kRedOff);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     const uint32_t b_full = smem_u32(bars), b_empty = b_full + 8 * S;
@@ -173,7 +222,17 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         *abort_flag = 0;
         fence_mbar_init();
     }
-    for (int i = threadIdx.x; i < (1 << (2 * KB)); i += blockDim.x) s_lut[i] = p.pair_lut[i];
+    for (int i = threadIdx.x; i < (1 << (2 * KB)); i += blockDim.x) s_pair[i] = p.pair_lut[i];
+    __syncthreads();
+    if constexpr (C::kQuad) {
+        // quad table: key = 4 codes (4 KB bits, LSB first) -> {half2(c0, c1), half2(c2, c3)}
+        uint2* q4 = reinterpret_cast<uint2*>(smem + C::kLutOff);
+        for (int i = threadIdx.x; i < (1 << (4 * KB)); i += blockDim.x)
+            q4[i] = make_uint2(s_pair[i & ((1 << (2 * KB)) - 1)], s_pair[i >> (2 * KB)]);
+    } else {
+        uint32_t* q2 = reinterpret_cast<uint32_t*>(smem + C::kLutOff);
+        for (int i = threadIdx.x; i < (1 << (2 * KB)); i += blockDim.x) q2[i] = s_pair[i];
+    }
     __syncthreads();
 
     if (warp == C::kWarps) {
@@ -184,22 +243,30 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                 if (!mbar_wait(b_empty + 8 * s, static_cast<uint32_t>((ti / S) & 1) ^ 1u, abort_flag)) break;
                 const int64_t c0 = c_begin + ti * C::kWarps;
                 const int nc = static_cast<int>((c_end - c0 < C::kWarps) ? c_end - c0 : C::kWarps);
-                mbar_arrive_expect_tx(b_full + 8 * s, nc * C::kChunkBytes);
+                mbar_arrive_expect_tx(b_full + 8 * s, nc * (C::kStageBytes / C::kWarps));
                 uint8_t* st = smem + s * C::kStageBytes;
-                for (int c = 0; c < nc; ++c) {
-                    int64_t row0;
-                    if (p.block_table)
-                        row0 = (static_cast<int64_t>(p.block_table[static_cast<int64_t>(b) * p.max_blocks + c0 + c]) *
-                                    p.num_kv_heads + h) * 16;
-                    else
-                        row0 = (static_cast<int64_t>(b) * p.num_kv_heads + h) * p.max_seq_len + (c0 + c) * 16;
-                    uint8_t* dst = st + c * C::kChunkBytes;
-                    const uint32_t bar = b_full + 8 * s;
-                    bulk_load(smem_u32(dst + C::kKOff), p.k_packed + row0 * C::kKRow, 16 * C::kKRow, bar);
-                    bulk_load(smem_u32(dst + C::kNOff), p.k_norms + row0, 64, bar);
-                    bulk_load(smem_u32(dst + C::kVOff), p.v_data + row0 * C::kVRow, 16 * C::kVRow, bar);
-                    bulk_load(smem_u32(dst + C::kSOff), p.v_scales + row0 * G8, 32 * G8, bar);
-                    bulk_load(smem_u32(dst + C::kZOff), p.v_zeros + row0 * G8, 32 * G8, bar);
+                const uint32_t bar = b_full + 8 * s;
+                if (!p.block_table) {
+                    // the tile's chunks are consecutive rows of the pool: one copy per array
+                    const int64_t row0 = (static_cast<int64_t>(b) * p.num_kv_heads + h) * p.max_seq_len + c0 * 16;
+                    const int rows = nc * 16;
+                    bulk_load(smem_u32(st + C::kKOff), p.k_packed + row0 * C::kKRow, rows * C::kKRow, bar);
+                    bulk_load(smem_u32(st + C::kNOff), p.k_norms + row0, rows * 4, bar);
+                    bulk_load(smem_u32(st + C::kVOff), p.v_data + row0 * C::kVRow, rows * C::kVRow, bar);
+                    bulk_load(smem_u32(st + C::kSOff), p.v_scales + row0 * G8, rows * G8 * 2, bar);
+                    bulk_load(smem_u32(st + C::kZOff), p.v_zeros + row0 * G8, rows * G8 * 2, bar);
+                } else {
+                    for (int c = 0; c < nc; ++c) {
+                        const int64_t blk = p.block_table[static_cast<int64_t>(b) * p.max_blocks + c0 + c];
+                        const int64_t row0 = (blk * p.num_kv_heads + h) * 16;
+                        bulk_load(smem_u32(st + C::kKOff + c * 16 * C::kKRow), p.k_packed + row0 * C::kKRow,
+                                  16 * C::kKRow, bar);
+                        bulk_load(smem_u32(st + C::kNOff + c * 64), p.k_norms + row0, 64, bar);
+                        bulk_load(smem_u32(st + C::kVOff + c * 16 * C::kVRow), p.v_data + row0 * C::kVRow,
+                                  16 * C::kVRow, bar);
+                        bulk_load(smem_u32(st + C::kSOff + c * 32 * G8), p.v_scales + row0 * G8, 32 * G8, bar);
+                        bulk_load(smem_u32(st + C::kZOff + c * 32 * G8), p.v_zeros + row0 * G8, 32 * G8, bar);
+                    }
                 }
             }
             // drain: the last issued stages have landed before the CTA may reuse or leave them
@@ -211,17 +278,19 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         // q_rot[g][n] = sum_k q[g][k] Pi_op[n][k] on the tensor cores (fp16 inputs are exact products)
         const __half* qg = p.q + (static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * G) * D;
         for (int nt = warp; nt < NT; nt += C::kWarps) {
-            float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+            // every fragment of this n-tile is loaded before the first MMA, so the loads overlap
+            uint32_t bf[KS][2], af[KS][2];
+            const __half* prow = p.pi_op + (8 * nt + gid) * D + 2 * tig;
+#pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
-                uint4 a = make_uint4(0u, 0u, 0u, 0u);
-                if (gid < G) {
-                    a.x = *reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig);
-                    a.z = *reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig + 8);
-                }
-                const __half* prow = p.pi_op + (8 * nt + gid) * D + 16 * ks + 2 * tig;
-                mma_f16(c, a, *reinterpret_cast<const uint32_t*>(prow), *reinterpret_cast<const uint32_t*>(prow + 8));
+                bf[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(prow + 16 * ks));
+                bf[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(prow + 16 * ks + 8));
+                af[ks][0] = (gid < G) ? __ldg(reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig)) : 0u;
+                af[ks][1] = (gid < G) ? __ldg(reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig + 8)) : 0u;
             }
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) mma_f16(c, make_uint4(af[ks][0], 0u, af[ks][1], 0u), bf[ks][0], bf[ks][1]);
             s_qr[gid * D + 8 * nt + 2 * tig] = c[0];
             s_qr[gid * D + 8 * nt + 2 * tig + 1] = c[1];
         }
@@ -242,13 +311,13 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         // k-slots (2tig, 2tig+1, 2tig+8, 2tig+9) of k-step ks <- coords tig*D/4 + 4ks + (0, 1, 2, 3)
         for (int i = threadIdx.x; i < KS * 32; i += 32 * C::kWarps) {
             const int ks = i >> 5, ln = i & 31, g = ln >> 2, tg = ln & 3;
-            const int c0 = tg * (D / 4) + 4 * ks;
+            const int cc = tg * (D / 4) + 4 * ks;
             uint4 f = make_uint4(0u, 0u, 0u, 0u);
             if (g < G) {
                 float x[4], hi[4], lo[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    x[e] = s_qr[g * D + c0 + e] * p.scale_log2 * pre;
+                    x[e] = s_qr[g * D + cc + e] * p.scale_log2 * pre;
                     hi[e] = __half2float(__float2half_rn(x[e]));
                     lo[e] = x[e] - hi[e];
                 }
@@ -262,6 +331,8 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         named_bar_sync(1, 32 * C::kWarps);
 
         // ------------------------------------------------------------------ token loop
+        const uint2* lut4 = reinterpret_cast<const uint2*>(smem + C::kLutOff);
+        const uint32_t* lut2 = reinterpret_cast<const uint32_t*>(smem + C::kLutOff);
         float o[NT][4];
 #pragma unroll
         for (int m = 0; m < NT; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
@@ -269,54 +340,54 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
 #pragma unroll
         for (int g = 0; g < G8; ++g) zacc[g] = 0.f;
         float m_run = -INFINITY, l_run = 0.f;
+        const int tok[4] = {2 * tig, 2 * tig + 1, 8 + 2 * tig, 9 + 2 * tig};
 
         for (int64_t ti = 0; ti < ntiles; ++ti) {
             const int s = static_cast<int>(ti % S);
             if (!mbar_wait(b_full + 8 * s, static_cast<uint32_t>((ti / S) & 1), abort_flag)) break;
             const int64_t chunk = c_begin + ti * C::kWarps + warp;
             if (chunk < c_end) {
-                const uint8_t* ch = smem + s * C::kStageBytes + warp * C::kChunkBytes;
+                const uint8_t* st = smem + s * C::kStageBytes;
+                const uint8_t* kch = st + C::kKOff + warp * 16 * C::kKRow;
                 // ---- scores: S'[16 x 8 tokens] per n-tile, rows gid (hi part) and gid+8 (lo part)
-                float sc[2][4];
+                uint32_t w[2][C::kQuarterWords];
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
                     // this lane's quarter of the key row of token 8nt + gid
-                    const uint8_t* krow = ch + C::kKOff + (8 * nt + gid) * C::kKRow;
-                    uint32_t w[C::kQuarterWords];
+                    const uint8_t* krow = kch + (8 * nt + gid) * C::kKRow;
                     if constexpr (C::kQuarterHalves % 2 == 0) {
                         const uint32_t* k32 = reinterpret_cast<const uint32_t*>(krow) + tig * (C::kQuarterHalves / 2);
 #pragma unroll
-                        for (int i = 0; i < C::kQuarterWords; ++i) w[i] = (2 * i < C::kQuarterHalves) ? k32[i] : 0u;
+                        for (int i = 0; i < C::kQuarterWords; ++i) w[nt][i] = (2 * i < C::kQuarterHalves) ? k32[i] : 0u;
                     } else {
                         const uint16_t* k16 = reinterpret_cast<const uint16_t*>(krow) + tig * C::kQuarterHalves;
 #pragma unroll
                         for (int i = 0; i < C::kQuarterWords; ++i) {
                             const uint32_t lo16 = (2 * i < C::kQuarterHalves) ? k16[2 * i] : 0u;
                             const uint32_t hi16 = (2 * i + 1 < C::kQuarterHalves) ? k16[2 * i + 1] : 0u;
-                            w[i] = lo16 | (hi16 << 16);
+                            w[nt][i] = lo16 | (hi16 << 16);
                         }
                     }
+                }
+                float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-                    for (int ks = 0; ks < KS; ++ks) {
-                        const uint4 a = s_qf[ks * 32 + lane];
-                        const int bp = 4 * ks * KB;
-                        uint32_t keys[2];
+                for (int ks = 0; ks < KS; ++ks) {
+                    const uint4 a = s_qf[ks * 32 + lane];
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int bb = bp + 2 * e * KB;
-                            const int wi = bb >> 5, sh = bb & 31;
-                            uint32_t v = w[wi] >> sh;
-                            if (sh + 2 * KB > 32) v |= w[wi + 1] << (32 - sh);
-                            keys[e] = v & ((1u << (2 * KB)) - 1u);
+                    for (int nt = 0; nt < 2; ++nt) {
+                        if constexpr (C::kQuad) {
+                            const uint2 bb = lut4[get_bits<4 * KB>(w[nt], 4 * ks * KB)];
+                            mma_f16(sc[nt], a, bb.x, bb.y);
+                        } else {
+                            const uint32_t k0 = get_bits<2 * KB>(w[nt], 4 * ks * KB);
+                            const uint32_t k1 = get_bits<2 * KB>(w[nt], 4 * ks * KB + 2 * KB);
+                            mma_f16(sc[nt], a, lut2[k0], lut2[k1]);
                         }
-                        mma_f16(sc[nt], a, s_lut[keys[0]], s_lut[keys[1]]);
                     }
                 }
                 // ---- logits (log2 domain) of head gid for tokens 2tig, 2tig+1, 8+2tig, 9+2tig
-                const float* nrm = reinterpret_cast<const float*>(ch + C::kNOff);
+                const float* nrm = reinterpret_cast<const float*>(st + C::kNOff) + warp * 16;
                 float lg[4];
-                int tok[4] = {2 * tig, 2 * tig + 1, 8 + 2 * tig, 9 + 2 * tig};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int nt = e >> 1, k = e & 1;
@@ -334,40 +405,62 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                 for (int e = 0; e < 4; ++e) pr[e] = exp2f(lg[e] - m_use);
                 l_run = l_run * corr + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
                 m_run = m_new;
+                if (__any_sync(0xffffffffu, corr != 1.0f)) {     // some head's running max moved
 #pragma unroll
-                for (int m = 0; m < NT; ++m) {
-                    o[m][0] *= corr; o[m][1] *= corr; o[m][2] *= corr; o[m][3] *= corr;
-                }
-                // ---- values: per scale group, A = hi/lo of p * scale, B = integer codes
-                const __half* vs = reinterpret_cast<const __half*>(ch + C::kSOff);
-                const __half* vz = reinterpret_cast<const __half*>(ch + C::kZOff);
-                const uint8_t* vrow[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) vrow[e] = ch + C::kVOff + tok[e] * C::kVRow;
-#pragma unroll
-                for (int g8 = 0; g8 < G8; ++g8) {
-                    float wv[4];
-                    float zs = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        wv[e] = pr[e] * __half2float(vs[tok[e] * G8 + g8]);
-                        zs = fmaf(pr[e], __half2float(vz[tok[e] * G8 + g8]), zs);
+                    for (int m = 0; m < NT; ++m) {
+                        o[m][0] *= corr; o[m][1] *= corr; o[m][2] *= corr; o[m][3] *= corr;
                     }
-                    zacc[g8] = zacc[g8] * corr + zs;
-                    uint4 a;
-                    split_bf16(wv[0], wv[1], a.x, a.y);
-                    split_bf16(wv[2], wv[3], a.z, a.w);
 #pragma unroll
-                    for (int mm = 0; mm < VG / 8; ++mm) {
-                        const int m = g8 * (VG / 8) + mm;
-                        const int col = 8 * m + gid;
-                        const uint32_t b0 = vcode_pair<VB>(vrow[0], vrow[1], col);
-                        const uint32_t b1 = vcode_pair<VB>(vrow[2], vrow[3], col);
-                        mma_bf16(o[m], a, b0, b1);
+                    for (int g8 = 0; g8 < G8; ++g8) zacc[g8] *= corr;
+                }
+                // ---- zero term on FMAs
+                const __half* zch = reinterpret_cast<const __half*>(st + C::kZOff) + warp * 16 * G8;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float zr[G8];
+                    load_halves<G8>(zch + tok[e] * G8, zr);
+#pragma unroll
+                    for (int g8 = 0; g8 < G8; ++g8) zacc[g8] = fmaf(pr[e], zr[g8], zacc[g8]);
+                }
+                // ---- values: A = hi/lo of p * scale (per scale group), B = integer codes, per 32-column slice
+                const __half* sch = reinterpret_cast<const __half*>(st + C::kSOff) + warp * 16 * G8;
+                float sc4[4][G8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) load_halves<G8>(sch + tok[e] * G8, sc4[e]);
+                const uint8_t* vch = st + C::kVOff + warp * 16 * C::kVRow;
+                const uint8_t* vrow0 = vch + tok[0] * C::kVRow;
+                const uint8_t* vrow1 = vch + tok[1] * C::kVRow;
+                const uint8_t* vrow2 = vch + tok[2] * C::kVRow;
+                const uint8_t* vrow3 = vch + tok[3] * C::kVRow;
+                uint4 a;
+#pragma unroll
+                for (int sl = 0; sl < D / 32; ++sl) {
+                    const int g8 = (sl * 32) / VG;
+                    if (sl == 0 || (sl * 32) % VG == 0) {
+                        split_bf16(pr[0] * sc4[0][g8], pr[1] * sc4[1][g8], a.x, a.y);
+                        split_bf16(pr[2] * sc4[2][g8], pr[3] * sc4[3][g8], a.z, a.w);
+                    }
+                    if constexpr (VB == 8) {
+                        // 8-bit codes: one byte per column, read per n-tile to keep registers low
+#pragma unroll
+                        for (int mm = 0; mm < 4; ++mm) {
+                            const int c = sl * 32 + 8 * mm + gid;
+                            mma_bf16(o[4 * sl + mm], a, pack_bf16(static_cast<float>(vrow0[c]), static_cast<float>(vrow1[c])),
+                                     pack_bf16(static_cast<float>(vrow2[c]), static_cast<float>(vrow3[c])));
+                        }
+                    } else {
+                        uint32_t w0[VB], w1[VB], w2[VB], w3[VB];
+                        load_vslice<VB>(vrow0, sl, w0);
+                        load_vslice<VB>(vrow1, sl, w1);
+                        load_vslice<VB>(vrow2, sl, w2);
+                        load_vslice<VB>(vrow3, sl, w3);
+#pragma unroll
+                        for (int mm = 0; mm < 4; ++mm) {
+                            const int c = 8 * mm + gid;
+                            mma_bf16(o[4 * sl + mm], a, vcode_pair<VB>(w0, w1, c), vcode_pair<VB>(w2, w3, c));
+                        }
                     }
                 }
-            } else {
-                // no chunk for this warp in this stage: keep running statistics unchanged
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(b_empty + 8 * s);
@@ -425,35 +518,64 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                 }
             }
         }
-        if (p.num_splits > 1) {
-            // ---------------------------------------------------------------- split-K merge, last CTA
-            __threadfence();
-            named_bar_sync(1, 32 * C::kWarps);
-            int* ctr = p.counters + static_cast<int64_t>(b) * p.num_kv_heads + h;
-            if (tid == 0) s_red[4] = __int_as_float(atomicAdd(ctr, 1));
-            named_bar_sync(1, 32 * C::kWarps);
-            if (__float_as_int(s_red[4]) == p.num_splits - 1) {
-                __threadfence();
-                const float* base =
-                    p.partials + (static_cast<int64_t>(b) * p.num_kv_heads + h) * p.num_splits * C::kPartFloats;
-                for (int i = tid; i < G * D; i += 32 * C::kWarps) {
-                    const int g = i / D, col = i % D;
-                    float M = -INFINITY;
-                    for (int sp = 0; sp < p.num_splits; ++sp) M = fmaxf(M, __ldcg(base + sp * C::kPartFloats + g));
-                    const float Mu = (M == -INFINITY) ? 0.f : M;
-                    float L = 0.f, O = 0.f;
-                    for (int sp = 0; sp < p.num_splits; ++sp) {
-                        const float* ps = base + sp * C::kPartFloats;
-                        const float f = exp2f(__ldcg(ps + g) - Mu);
-                        L += __ldcg(ps + 8 + g) * f;
-                        O += __ldcg(ps + 16 + g * D + col) * f;
-                    }
-                    p.out[(static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * G + g) * D + col] =
-                        (L > 0.f) ? O / L : 0.f;
-                }
-                if (tid == 0) *ctr = 0;      // leave the counter zeroed for the next call
-            }
-        }
+        // the merge grid (launched as a programmatic dependent) may start; it waits for this grid to finish
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    }
+}
+
+// Split-K merge: out[b][h*G+g][:] = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M), M = max_s m_s.
+// One CTA per (g, h, b); pass 1 gives every split's weight, pass 2 spreads the splits over
+// kMergeThreads / D slices so the partial loads are issued in parallel.
+constexpr int kMergeThreads = 512;
+constexpr int kMaxSplits = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kMergeThreads) attend_merge_kernel(const AttendParams p) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    constexpr int kPart = 16 + 8 * D;
+    constexpr int kSlices = kMergeThreads / D;
+    __shared__ float s_f[kMaxSplits];
+    __shared__ float s_red[kMergeThreads / 32];
+    __shared__ float s_part[kSlices][D];
+    const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    const int S = p.num_splits;
+    const float* base = p.partials + (static_cast<int64_t>(b) * p.num_kv_heads + h) * S * kPart;
+    const float m = (tid < S) ? __ldcg(base + static_cast<int64_t>(tid) * kPart + g) : -INFINITY;
+    float M = m;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if ((tid & 31) == 0) s_red[tid >> 5] = M;
+    __syncthreads();
+    M = s_red[0];
+#pragma unroll
+    for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, s_red[w]);
+    const float Mu = (M == -INFINITY) ? 0.f : M;
+    float lw = 0.f;
+    if (tid < S) {
+        const float f = exp2f(m - Mu);
+        s_f[tid] = f;
+        lw = __ldcg(base + static_cast<int64_t>(tid) * kPart + 8 + g) * f;
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
+    __syncthreads();
+    if ((tid & 31) == 0) s_red[tid >> 5] = lw;
+    __syncthreads();
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeThreads / 32; ++w) L += s_red[w];
+    const int col = tid % D, slice = tid / D;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int sp = slice; sp < S; sp += kSlices)
+        acc += __ldcg(base + static_cast<int64_t>(sp) * kPart + 16 + g * D + col) * s_f[sp];
+    s_part[slice][col] = acc;
+    __syncthreads();
+    if (slice == 0) {
+#pragma unroll
+        for (int k = 1; k < kSlices; ++k) acc += s_part[k][col];
+        p.out[(static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * p.group + g) * D + col] =
+            (L > 0.f) ? acc / L : 0.f;
     }
 }
 

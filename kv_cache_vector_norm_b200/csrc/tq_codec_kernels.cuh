@@ -6,175 +6,202 @@
 namespace tq {
 namespace dev {
 
-// --------------------------------------------------------------------------------- bit-field helpers
-
-// OR value v (< 2^BITS) into the little-endian bitstream `w` at field j (compile-time after unrolling).
-template <int BITS, int NW>
-__device__ __forceinline__ void put_field(uint32_t (&w)[NW], int j, uint32_t v) {
-    const int bit = j * BITS, wi = bit >> 5, sh = bit & 31;
-    w[wi] |= v << sh;
-    if (sh + BITS > 32) w[wi + 1] |= v >> (32 - sh);
-}
-
-// Field of width W starting at bit `bit` of the little-endian bitstream `w`.
-template <int W, int NW>
-__device__ __forceinline__ uint32_t get_bits(const uint32_t (&w)[NW], int bit) {
-    const int wi = bit >> 5, sh = bit & 31;
-    uint32_t v = w[wi] >> sh;
-    if (sh + W > 32) v |= w[wi + 1] << (32 - sh);
-    return (W == 32) ? v : (v & ((1u << W) - 1u));
-}
-
-// Store NW words (4-byte aligned destination; wider vectors where NW allows and `dst` is aligned to them).
-template <int NW>
-__device__ __forceinline__ void store_words(uint8_t* dst, const uint32_t (&w)[NW]) {
-    if constexpr (NW % 4 == 0) {
-#pragma unroll
-        for (int i = 0; i < NW; i += 4)
-            *reinterpret_cast<uint4*>(dst + 4 * i) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
-    } else if constexpr (NW == 2) {
-        *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
-    } else {
-#pragma unroll
-        for (int i = 0; i < NW; ++i) reinterpret_cast<uint32_t*>(dst)[i] = w[i];
-    }
-}
-
-template <int NW>
-__device__ __forceinline__ void load_words(const uint8_t* src, uint32_t (&w)[NW]) {
-    if constexpr (NW % 4 == 0) {
-#pragma unroll
-        for (int i = 0; i < NW; i += 4) {
-            uint4 v = *reinterpret_cast<const uint4*>(src + 4 * i);
-            w[i] = v.x; w[i + 1] = v.y; w[i + 2] = v.z; w[i + 3] = v.w;
-        }
-    } else if constexpr (NW == 2) {
-        uint2 v = *reinterpret_cast<const uint2*>(src);
-        w[0] = v.x; w[1] = v.y;
-    } else {
-#pragma unroll
-        for (int i = 0; i < NW; ++i) w[i] = reinterpret_cast<const uint32_t*>(src)[i];
-    }
-}
-
 // ------------------------------------------------------------------------------------ value codec
-// "KV Cache API", values.py quantize_values / dequantize_values.  One thread owns one 32-element unit of
-// a row (a whole group when GROUP == 32); with GROUP == D the D/32 units of a row sit in consecutive
-// lanes and reduce min/max with shuffles.  Every step is the page's fp32 operation, rounded once.
+// "KV Cache API", values.py quantize_values / dequantize_values.  One lane owns 8 consecutive elements of
+// a row (16 bytes of fp16), so every warp-wide load and store is contiguous; the lanes of one scale group
+// (4 for group 32, d/8 for the per-token layout) reduce min/max with shuffles.  Every arithmetic step is
+// the page's fp32 operation with one rounding.
+
+// Code of one element: round_half_even(a / s) with the page's IEEE fp32 division, for 0 <= a <= (2^b - 1) s.
+// Fast path: with r = RN(1/s) the product qa = RN(a r) is within 2^-22 (relative) of RN(a / s); adding
+// 1.5 * 2^23 rounds qa to the nearest integer (ties to even) in the low mantissa bits, and when qa lies
+// farther than 2^-21 qa from the half-integers both qa and RN(a / s) round to that same integer.
+// Otherwise (rare) the exact quotient is rounded.  Returns the integer code.
+__device__ __forceinline__ uint32_t quant_code(float a, float s, float r) {
+    constexpr float kMagic = 12582912.0f;                  // 1.5 * 2^23
+    const float qa = __fmul_rn(a, r);
+    const float t = __fadd_rn(qa, kMagic);
+    const float k = __fsub_rn(t, kMagic);
+    const float dev = fabsf(__fsub_rn(qa, k));
+    uint32_t code = __float_as_uint(t) - 0x4B400000u;
+    if (!(__fmaf_rn(qa, 4.76837158203125e-7f, dev) < 0.5f))
+        code = __float_as_uint(__fadd_rn(rintf(__fdiv_rn(a, s)), kMagic)) - 0x4B400000u;
+    return code;
+}
+
+template <int D, int GROUP>
+struct VLanes {
+    static constexpr int kRowLanes = D / 8;                       // lanes per row (8 elements each)
+    static constexpr int kRowsPerWarp = 32 / kRowLanes;           // 1, 2 or 4
+    static constexpr int kGroupLanes = GROUP / 8;                 // lanes per scale group (4 or D/8)
+};
+
+// Encode: one lane owns 16 consecutive elements (two 16-byte loads), so a group of 32 spans 2 lanes
+// (or d/16 lanes in the per-token layout) and the per-group division and reciprocal are shared by 16
+// elements.
+template <int D, int GROUP>
+struct VEncLanes {
+    static constexpr int kRowLanes = D / 16;
+    static constexpr int kRowsPerWarp = 32 / kRowLanes;           // 2, 4 or 8
+    static constexpr int kGroupLanes = GROUP / 16;                // 2 or d/16
+};
 
 template <int D, int BITS, int GROUP>
 __global__ void __launch_bounds__(256) encode_v_kernel(const __half* __restrict__ x, int64_t n, int64_t stride,
                                                        const int64_t* __restrict__ slots, uint8_t* __restrict__ data,
                                                        __half* __restrict__ scales, __half* __restrict__ zeros) {
-    constexpr int kUnits = D / 32;
+    using L = VEncLanes<D, GROUP>;
     constexpr int kRowBytes = D * BITS / 8;
     constexpr int kGroups = D / GROUP;
-    constexpr float kLevels = static_cast<float>((1 << BITS) - 1);
-    const int64_t total = n * kUnits;
-    const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    // warp-uniform trip count so every lane takes part in the shuffles
-    for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31); base < total; base += step) {
-        const int64_t u = base + (threadIdx.x & 31);
-        const bool valid = u < total;
-        const int64_t row = valid ? u / kUnits : 0;
-        const int part = static_cast<int>(u % kUnits);
-        float v[32];
+    constexpr uint32_t kLevels = (1u << BITS) - 1u;
+    constexpr int kW = (16 * BITS + 31) / 32;                     // words holding this lane's 16 codes
+    const int lane = threadIdx.x & 31;
+    const int j = lane % L::kRowLanes;                            // 16-element chunk index within the row
+    const int gl = j % L::kGroupLanes;                            // lane index within the scale group
+    const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
+    for (int64_t wrow = (static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5)) * L::kRowsPerWarp;
+         wrow < n; wrow += warps_total * L::kRowsPerWarp) {
+        const int64_t row = wrow + lane / L::kRowLanes;
+        const bool valid = row < n;
+        float v[16];
         if (valid) {
-            const uint4* p = reinterpret_cast<const uint4*>(x + row * stride + part * 32);
+            const uint4* src = reinterpret_cast<const uint4*>(x + row * stride) + 2 * j;
+            const uint4 w0 = __ldg(src), w1 = __ldg(src + 1);
+            const __half2* h0 = reinterpret_cast<const __half2*>(&w0);
+            const __half2* h1 = reinterpret_cast<const __half2*>(&w1);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint4 w = __ldg(p + i);
-                const __half2* h = reinterpret_cast<const __half2*>(&w);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    float2 f = __half22float2(h[k]);
-                    v[8 * i + 2 * k] = f.x;
-                    v[8 * i + 2 * k + 1] = f.y;
-                }
+            for (int k = 0; k < 4; ++k) {
+                const float2 f0 = __half22float2(h0[k]), f1 = __half22float2(h1[k]);
+                v[2 * k] = f0.x;
+                v[2 * k + 1] = f0.y;
+                v[8 + 2 * k] = f1.x;
+                v[8 + 2 * k + 1] = f1.y;
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            for (int k = 0; k < 16; ++k) v[k] = 0.f;
         }
-        float vmin = v[0], vmax = v[0];
+        float vmin = fminf(v[0], v[1]), vmax = fmaxf(v[0], v[1]);
 #pragma unroll
-        for (int i = 1; i < 32; ++i) {
-            vmin = fminf(vmin, v[i]);
-            vmax = fmaxf(vmax, v[i]);
+        for (int k = 2; k < 16; ++k) {
+            vmin = fminf(vmin, v[k]);
+            vmax = fmaxf(vmax, v[k]);
         }
-        if constexpr (GROUP == D) {
 #pragma unroll
-            for (int off = 1; off < kUnits; off <<= 1) {
-                vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, off));
-                vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
-            }
+        for (int off = 1; off < L::kGroupLanes; off <<= 1) {
+            vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, off));
+            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
         }
-        float scale = __fdiv_rn(__fsub_rn(vmax, vmin), kLevels);
+        float scale = __fdiv_rn(__fsub_rn(vmax, vmin), static_cast<float>(kLevels));
         scale = fmaxf(scale, 1e-12f);
         const float zero = vmin;
-        uint32_t w[BITS];
+        const float rcp = __frcp_rn(scale);
+        uint32_t chunk[kW];
 #pragma unroll
-        for (int i = 0; i < BITS; ++i) w[i] = 0u;
+        for (int k = 0; k < kW; ++k) chunk[k] = 0u;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            float q = rintf(__fdiv_rn(__fsub_rn(v[i], zero), scale));
-            q = fminf(fmaxf(q, 0.f), kLevels);
-            put_field<BITS>(w, i, static_cast<uint32_t>(q));
+        for (int k = 0; k < 16; ++k) {
+            // the page clamps to [0, 2^b - 1]; with a in [0, max - min] the code can only exceed the top
+            // level through rounding, so one min() keeps the clamp
+            const uint32_t q = min(quant_code(__fsub_rn(v[k], zero), scale, rcp), kLevels);
+            put_field<BITS>(chunk, k, q);
         }
-        if (valid) {
-            const int64_t orow = slots ? slots[row] : row;
+        const int64_t orow = valid ? (slots ? slots[row] : row) : -1;
+        uint8_t* dst = data + orow * kRowBytes;
+        if constexpr (BITS == 2) {
+            if (orow >= 0) reinterpret_cast<uint32_t*>(dst)[j] = chunk[0];
+        } else if constexpr (BITS == 4) {
+            if (orow >= 0) reinterpret_cast<uint2*>(dst)[j] = make_uint2(chunk[0], chunk[1]);
+        } else if constexpr (BITS == 8) {
+            if (orow >= 0) reinterpret_cast<uint4*>(dst)[j] = make_uint4(chunk[0], chunk[1], chunk[2], chunk[3]);
+        } else {
+            // 3 bits: 16 codes = 48 bits = 3 half-words at byte 6j (2-byte aligned)
             if (orow >= 0) {
-                store_words<BITS>(data + orow * kRowBytes + part * 4 * BITS, w);
-                if (GROUP == 32 || part == 0) {
-                    const int gi = (GROUP == 32) ? part : 0;
-                    scales[orow * kGroups + gi] = __float2half_rn(scale);
-                    zeros[orow * kGroups + gi] = __float2half_rn(zero);
-                }
+                uint16_t* h = reinterpret_cast<uint16_t*>(dst + 6 * j);
+                h[0] = static_cast<uint16_t>(chunk[0]);
+                h[1] = static_cast<uint16_t>(chunk[0] >> 16);
+                h[2] = static_cast<uint16_t>(chunk[1]);
             }
+        }
+        if (orow >= 0 && gl == 0) {
+            const int gi = j / L::kGroupLanes;
+            scales[orow * kGroups + gi] = __float2half_rn(scale);
+            zeros[orow * kGroups + gi] = __float2half_rn(zero);
         }
     }
 }
 
+template <int D, int BITS>
+__device__ __forceinline__ void load_vchunk(const uint8_t* src, int j, uint32_t (&c)[2]) {
+    if constexpr (BITS == 4) {
+        c[0] = reinterpret_cast<const uint32_t*>(src)[j];
+        c[1] = 0u;
+    } else if constexpr (BITS == 8) {
+        const uint2 t = reinterpret_cast<const uint2*>(src)[j];
+        c[0] = t.x;
+        c[1] = t.y;
+    } else if constexpr (BITS == 2) {
+        c[0] = reinterpret_cast<const uint16_t*>(src)[j];
+        c[1] = 0u;
+    } else {
+        // 24 bits at byte 3j: the aligned 32-bit word holding its start, plus the next one when needed
+        const int byte = 3 * j, wi = byte >> 2, sh = 8 * (byte & 3);
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(src);
+        const uint64_t both = static_cast<uint64_t>(w[wi]) | (sh > 8 ? static_cast<uint64_t>(w[wi + 1]) << 32 : 0ull);
+        c[0] = static_cast<uint32_t>(both >> sh) & 0xFFFFFFu;
+        c[1] = 0u;
+    }
+}
+
+// Decode: one lane owns 8 consecutive elements of a row (kU rows per lane per iteration, loads first).
 template <int D, int BITS, int GROUP, bool OUT_F32>
 __global__ void __launch_bounds__(256) decode_v_kernel(const uint8_t* __restrict__ data, const __half* __restrict__ scales,
                                                        const __half* __restrict__ zeros, int64_t n, void* __restrict__ out) {
-    constexpr int kUnits = D / 32;
+    using L = VLanes<D, GROUP>;
+    constexpr int kU = 1;                                         // rows per lane per iteration
     constexpr int kRowBytes = D * BITS / 8;
     constexpr int kGroups = D / GROUP;
-    const int64_t total = n * kUnits;
-    const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < total; u += step) {
-        const int64_t row = u / kUnits;
-        const int part = static_cast<int>(u % kUnits);
-        uint32_t w[BITS];
-        load_words<BITS>(data + row * kRowBytes + part * 4 * BITS, w);
-        const int gi = (GROUP == 32) ? part : 0;
-        const float s = __half2float(scales[row * kGroups + gi]);
-        const float z = __half2float(zeros[row * kGroups + gi]);
-        float y[32];
+    const int lane = threadIdx.x & 31;
+    const int j = lane % L::kRowLanes;
+    const int gi = j / L::kGroupLanes;
+    const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
+    const int64_t step = warps_total * L::kRowsPerWarp;
+    for (int64_t wrow = (static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5)) * L::kRowsPerWarp;
+         wrow < n; wrow += step * kU) {
+        uint32_t c[kU][2];
+        float s[kU], z[kU];
+        int64_t rows[kU];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const uint32_t q = get_bits<BITS>(w, i * BITS);
-            y[i] = __fadd_rn(__fmul_rn(static_cast<float>(q), s), z);
+        for (int u = 0; u < kU; ++u) {
+            rows[u] = wrow + u * step + lane / L::kRowLanes;
+            if (rows[u] < n) {
+                load_vchunk<D, BITS>(data + rows[u] * kRowBytes, j, c[u]);
+                s[u] = __half2float(scales[rows[u] * kGroups + gi]);
+                z[u] = __half2float(zeros[rows[u] * kGroups + gi]);
+            }
         }
-        if constexpr (OUT_F32) {
-            float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + row * D + part * 32);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
-        } else {
-            uint4* o = reinterpret_cast<uint4*>(static_cast<__half*>(out) + row * D + part * 32);
+        for (int u = 0; u < kU; ++u) {
+            if (rows[u] >= n) continue;
+            float y[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t q = get_bits<BITS>(c[u], k * BITS);
+                y[k] = __fadd_rn(__fmul_rn(static_cast<float>(q), s[u]), z[u]);
+            }
+            if constexpr (OUT_F32) {
+                float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + rows[u] * D) + 2 * j;
+                o[0] = make_float4(y[0], y[1], y[2], y[3]);
+                o[1] = make_float4(y[4], y[5], y[6], y[7]);
+            } else {
                 uint4 pk;
-                __half2 h0 = __floats2half2_rn(y[8 * i], y[8 * i + 1]);
-                __half2 h1 = __floats2half2_rn(y[8 * i + 2], y[8 * i + 3]);
-                __half2 h2 = __floats2half2_rn(y[8 * i + 4], y[8 * i + 5]);
-                __half2 h3 = __floats2half2_rn(y[8 * i + 6], y[8 * i + 7]);
+                __half2 h0 = __floats2half2_rn(y[0], y[1]), h1 = __floats2half2_rn(y[2], y[3]);
+                __half2 h2 = __floats2half2_rn(y[4], y[5]), h3 = __floats2half2_rn(y[6], y[7]);
                 pk.x = *reinterpret_cast<uint32_t*>(&h0);
                 pk.y = *reinterpret_cast<uint32_t*>(&h1);
                 pk.z = *reinterpret_cast<uint32_t*>(&h2);
                 pk.w = *reinterpret_cast<uint32_t*>(&h3);
-                o[i] = pk;
+                reinterpret_cast<uint4*>(static_cast<__half*>(out) + rows[u] * D)[j] = pk;
             }
         }
     }
@@ -196,12 +223,14 @@ struct KeyCfg {
     static constexpr int kPiBlockBytes = D * 128;            // one 64-column block of the d x d matrix
     static constexpr int kEncStages = (D == 256) ? 1 : (D == 128 ? 4 : 6);
     static constexpr int kDecBufs = (D == 256) ? 1 : 2;
+    static constexpr int kDecInBufs = (D == 256) ? 1 : 2;    // packed-row staging buffers (decode)
     static constexpr int kEpiWarps = 8;
     static constexpr int kThreads = 32 * (2 + kEpiWarps);
     static constexpr int kTmemCols = 2 * D;                  // two accumulator buffers
     static constexpr int kHalfCols = D / 2;
     static constexpr int kChunks = kHalfCols / 32;           // 32-column TMEM loads per thread per tile
     static constexpr int kLutEntries = 2048;                 // encode grid table
+    static constexpr bool kEncStaged = (D <= 128);           // packed output staged for a bulk store
     static constexpr uint32_t kIdesc = idesc_f16_f32(128, D);
 };
 
@@ -211,51 +240,91 @@ struct KeyCfg {
 constexpr float kGridScale = 512.0f;
 constexpr float kGridMagic = 12583552.0f;   // 1.5 * 2^23 + 640
 
-struct EncSmem {
-    uint32_t pi, x, lut, norm, bar;
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Encode CTA: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-3 compute the row norms of
+// each X stage ahead of the epilogue, warps 4.. are the epilogue (kEncEpiWarps: warp w reads TMEM lanes
+// 32*(w%4).. and owns kEncCols columns of them).
+template <int D>
+struct EncCfg {
+    static constexpr int kNormWarps = 2;
+    static constexpr int kEpiWarps = (D == 64) ? 8 : 16;
+    static constexpr int kFirstEpi = 2 + kNormWarps;
+    static constexpr int kThreads = 32 * (kFirstEpi + kEpiWarps);
+    static constexpr int kCols = D * 4 / kEpiWarps;          // columns per epilogue warp: 32, 32, 64
+    static constexpr int kChunks = kCols / 32;
 };
 
-template <int D>
-__host__ __device__ constexpr uint32_t enc_smem_bytes() {
+template <int D, int BITS>
+struct EncLayout {
     using C = KeyCfg<D>;
-    return C::kPiBytes + C::kEncStages * C::kTileBytes + C::kLutEntries * 8 + 2 * 2 * 128 * 4 +
-           8 * (2 * C::kEncStages + 8) + 16 + 1024;
+    static constexpr int kRowBytes = D * BITS / 8;
+    static constexpr int kPkBytes = C::kEncStaged ? 128 * kRowBytes : 0;   // one staged packed tile
+    static constexpr uint32_t kPi = 0;
+    static constexpr uint32_t kX = kPi + C::kPiBytes;
+    static constexpr uint32_t kLut = kX + C::kEncStages * C::kTileBytes;
+    static constexpr uint32_t kPk = kLut + C::kLutEntries * 4;
+    static constexpr uint32_t kNorm = kPk + 2 * kPkBytes;                   // [stage][128] {norm, 1/(norm+1e-8)}
+    static constexpr uint32_t kBar = kNorm + C::kEncStages * 128 * 8;
+    static constexpr int kBars = 4 * C::kEncStages + 10;
+    static constexpr uint32_t kMisc = kBar + 8 * kBars;
+    static constexpr uint32_t kBytes = kMisc + 16 + 1024;                  // + alignment slack
+};
+
+template <int D, int BITS>
+__host__ __device__ constexpr uint32_t enc_smem_bytes() {
+    return EncLayout<D, BITS>::kBytes;
 }
 
 template <int D, int BITS>
-__global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
+__global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
     encode_k_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_pi,
-                    const uint2* __restrict__ lut_g, int64_t n, const int64_t* __restrict__ slots,
+                    const uint32_t* __restrict__ lut_g, int64_t n, const int64_t* __restrict__ slots,
                     uint8_t* __restrict__ packed, float* __restrict__ norms) {
     using C = KeyCfg<D>;
+    using E = EncCfg<D>;
+    using Lo = EncLayout<D, BITS>;
     constexpr int S = C::kEncStages;
-    constexpr int kRowBytes = D * BITS / 8;
+    constexpr int kRowBytes = Lo::kRowBytes;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* s_pi = smem;
-    uint8_t* s_x = s_pi + C::kPiBytes;
-    uint2* s_lut = reinterpret_cast<uint2*>(s_x + S * C::kTileBytes);
-    float* s_norm = reinterpret_cast<float*>(s_lut + C::kLutEntries);          // [2 bufs][2 halves][128]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(s_norm + 2 * 2 * 128);
-    // barrier slots
-    const uint32_t b_xfull = smem_u32(bars), b_xempty = b_xfull + 8 * S, b_accfull = b_xempty + 8 * S,
-                   b_accempty = b_accfull + 16, b_pifull = b_accempty + 16, b_normrdy = b_pifull + 8,
-                   b_final = b_normrdy + 16;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 8);
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);   // stays a shared-space pointer
+    uint8_t* s_pi = smem + Lo::kPi;
+    uint8_t* s_x = smem + Lo::kX;
+    const uint32_t* s_lut = reinterpret_cast<const uint32_t*>(smem + Lo::kLut);
+    uint8_t* s_pk = smem + Lo::kPk;
+    float2* s_norm = reinterpret_cast<float2*>(smem + Lo::kNorm);
+    const uint32_t bar0 = smem_u32(smem + Lo::kBar);
+    const uint32_t b_xfull = bar0, b_xempty = b_xfull + 8 * S, b_nrdy = b_xempty + 8 * S, b_nfree = b_nrdy + 8 * S,
+                   b_accfull = b_nfree + 8 * S, b_accempty = b_accfull + 16, b_pifull = b_accempty + 16,
+                   b_final = b_pifull + 8, b_pkfull = b_final + 8, b_pkempty = b_pkfull + 16;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lo::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t num_tiles = (n + 127) / 128;
+    const bool staged = C::kEncStaged && (slots == nullptr);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(b_xfull + 8 * s, 1);
-            mbar_init(b_xempty + 8 * s, 1 + C::kEpiWarps);
+            mbar_init(b_xempty + 8 * s, 1 + E::kNormWarps);
+            mbar_init(b_nrdy + 8 * s, E::kNormWarps);
+            mbar_init(b_nfree + 8 * s, E::kEpiWarps);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(b_accfull + 8 * a, 1);
-            mbar_init(b_accempty + 8 * a, C::kEpiWarps);
-            mbar_init(b_normrdy + 8 * a, C::kEpiWarps);
+            mbar_init(b_accempty + 8 * a, E::kEpiWarps);
+            mbar_init(b_pkfull + 8 * a, E::kEpiWarps);
+            mbar_init(b_pkempty + 8 * a, 1);
         }
         mbar_init(b_pifull, 1);
         mbar_init(b_final, 1);
@@ -266,7 +335,8 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
-    for (int i = threadIdx.x; i < C::kLutEntries; i += blockDim.x) s_lut[i] = lut_g[i];
+    for (int i = threadIdx.x; i < C::kLutEntries; i += blockDim.x)
+        reinterpret_cast<uint32_t*>(smem + Lo::kLut)[i] = lut_g[i];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -281,14 +351,12 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
             int li = 0;
             for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
                 const int s = li % S;
-                const uint32_t ph = (li / S) & 1;
-                if (!mbar_wait(b_xempty + 8 * s, ph ^ 1, abort_flag)) break;
+                if (!mbar_wait(b_xempty + 8 * s, ((li / S) & 1) ^ 1, abort_flag)) break;
                 mbar_arrive_expect_tx(b_xfull + 8 * s, C::kTileBytes);
                 for (int kb = 0; kb < C::kKB; ++kb)
                     tma_load_2d(smem_u32(s_x + s * C::kTileBytes + kb * C::kTileBlockBytes), &tmap_x, b_xfull + 8 * s,
                                 kb * 64, static_cast<int>(tile * 128));
             }
-            // drain: every issued load has landed before the CTA may exit
             for (int k = (li > S ? li - S : 0); k < li; ++k) mbar_wait_drain(b_xfull + 8 * (k % S), (k / S) & 1);
             mbar_wait_drain(b_pifull, 0);
         }
@@ -314,60 +382,83 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
                 umma_commit(b_accfull + 8 * a);
                 umma_commit(b_xempty + 8 * s);
             }
-            // every MMA has completed before TMEM is released
             umma_commit(b_final);
             mbar_wait_drain(b_final, 0);
         }
-    } else {
-        // -------------------------------------------------------------------- epilogue
-        const int ew = warp - 2;
-        const int quarter = warp & 3;
-        const int half = ew >> 2;
-        const int r = quarter * 32 + lane;
+    } else if (warp < E::kFirstEpi) {
+        // -------------------------------------------------------------------- row norms, ahead of the epilogue
+        const int t = (warp - 2) * 32 + lane;                 // rows t and t + 64 of each tile
         int li = 0;
         for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
-            const int s = li % S, a = li & 1, nb = li & 1;
+            const int s = li % S;
             if (!mbar_wait(b_xfull + 8 * s, (li / S) & 1, abort_flag)) break;
-            // sum of squares of this half of row r (squares of fp16 values are exact in fp32)
+            if (!mbar_wait(b_nfree + 8 * s, ((li / S) & 1) ^ 1, abort_flag)) break;
             const uint8_t* xs = s_x + s * C::kTileBytes;
-            float acc[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+            for (int hrow = 0; hrow < 2; ++hrow) {
+                const int r = t + 64 * hrow;
+                float acc[8];
 #pragma unroll
-            for (int c = 0; c < C::kHalfCols / 8; ++c) {
-                const int col = half * C::kHalfCols + c * 8;
-                const uint4 v = *reinterpret_cast<const uint4*>(xs + (col >> 6) * C::kTileBlockBytes +
-                                                                sw128_offset(r, (col & 63) >> 3));
-                const __half2* h = reinterpret_cast<const __half2*>(&v);
+                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 8
+                for (int c = 0; c < D / 8; ++c) {
+                    // squares of fp16 values are exact in fp32; eight partial sums keep the rounding small
+                    const uint4 v = *reinterpret_cast<const uint4*>(xs + (c >> 3) * C::kTileBlockBytes + sw128_offset(r, c & 7));
+                    const __half2* h = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float2 f = __half22float2(h[k]);
-                    acc[2 * k] = fmaf(f.x, f.x, acc[2 * k]);
-                    acc[2 * k + 1] = fmaf(f.y, f.y, acc[2 * k + 1]);
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 f = __half22float2(h[k]);
+                        acc[2 * k] = fmaf(f.x, f.x, acc[2 * k]);
+                        acc[2 * k + 1] = fmaf(f.y, f.y, acc[2 * k + 1]);
+                    }
+                }
+                const float nrm = sqrtf(((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
+                s_norm[s * 128 + r] = make_float2(nrm, 1.0f / (nrm + 1e-8f));
+                const int64_t row = tile * 128 + r;
+                if (row < n) {
+                    const int64_t orow = slots ? slots[row] : row;
+                    if (orow >= 0) norms[orow] = nrm;
                 }
             }
-            const float part = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
             __syncwarp();
-            if (lane == 0) mbar_arrive(b_xempty + 8 * s);
-            s_norm[nb * 256 + half * 128 + r] = part;
+            if (lane == 0) {
+                mbar_arrive(b_xempty + 8 * s);
+                mbar_arrive(b_nrdy + 8 * s);
+            }
+        }
+    } else {
+        // -------------------------------------------------------------------- epilogue
+        const int ew = warp - E::kFirstEpi;
+        const int quarter = warp & 3;
+        const int c0 = (ew >> 2) * E::kCols;                  // first column of this warp
+        const int r = quarter * 32 + lane;
+        const bool issuer = (ew == 0 && lane == 0);           // issues the bulk stores of staged tiles
+        int li = 0;
+        for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
+            const int s = li % S, a = li & 1, pb = li & 1;
+            if (!mbar_wait(b_nrdy + 8 * s, (li / S) & 1, abort_flag)) break;
+            const float inv = s_norm[s * 128 + r].y;
             __syncwarp();
-            if (lane == 0) mbar_arrive(b_normrdy + 8 * nb);
-            if (!mbar_wait(b_normrdy + 8 * nb, (li >> 1) & 1, abort_flag)) break;
-            const float nrm = sqrtf(s_norm[nb * 256 + r] + s_norm[nb * 256 + 128 + r]);
-            const float inv = 1.0f / (nrm + 1e-8f);
+            if (lane == 0) mbar_arrive(b_nfree + 8 * s);
             const int64_t row = tile * 128 + r;
             int64_t orow = -1;
-            if (row < n) orow = slots ? slots[row] : row;
-            if (half == 0 && orow >= 0) norms[orow] = nrm;
+            if (!staged && row < n) orow = slots ? slots[row] : row;
 
             if (!mbar_wait(b_accfull + 8 * a, (li >> 1) & 1, abort_flag)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * D + half * C::kHalfCols;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * D + c0;
+            uint8_t* pk = s_pk + pb * Lo::kPkBytes + r * kRowBytes;
+            if (staged && !mbar_wait(b_pkempty + 8 * pb, ((li >> 1) & 1) ^ 1, abort_flag)) break;
 #pragma unroll
-            for (int ch = 0; ch < C::kChunks; ++ch) {
+            for (int k = 0; k < E::kChunks; ++k) {
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(taddr + ch * 32, v);
+                tmem_ld_32x32b_x32(taddr + k * 32, v);
                 tmem_ld_wait();
+                if (k == E::kChunks - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(b_accempty + 8 * a);   // TMEM buffer a is free for tile li + 2
+                }
                 uint32_t w[BITS];
 #pragma unroll
                 for (int i = 0; i < BITS; ++i) w[i] = 0u;
@@ -375,17 +466,41 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
                 for (int j = 0; j < 32; ++j) {
                     const float y = __uint_as_float(v[j]) * inv;
                     const float g = fmaf(y, kGridScale, kGridMagic);
-                    const uint2 e = s_lut[__float_as_uint(g) & (C::kLutEntries - 1)];
-                    const uint32_t idx = e.y + (y > __uint_as_float(e.x) ? 1u : 0u);
+                    const uint32_t e = s_lut[__float_as_uint(g) & (C::kLutEntries - 1)];
+                    const uint32_t idx = (e & 15u) + (y > __uint_as_float(e & ~15u) ? 1u : 0u);
                     put_field<BITS>(w, j, idx);
                 }
-                if (orow >= 0)
-                    store_words<BITS>(packed + orow * kRowBytes + (half * C::kHalfCols + ch * 32) * BITS / 8, w);
+                const int boff = (c0 + k * 32) * BITS / 8;
+                if (staged) {
+#pragma unroll
+                    for (int i = 0; i < BITS; ++i) reinterpret_cast<uint32_t*>(pk + boff)[i] = w[i];
+                } else if (orow >= 0) {
+                    store_words<BITS>(packed + orow * kRowBytes + boff, w);
+                }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b_accempty + 8 * a);
+            if (staged) {
+                // make this warp's rows visible to the bulk copy engine, then hand the tile to the issuer
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_pkfull + 8 * pb);
+                if (issuer) {
+                    if (!mbar_wait(b_pkfull + 8 * pb, (li >> 1) & 1, abort_flag)) break;
+                    const int64_t rows = (n - tile * 128 < 128) ? n - tile * 128 : 128;
+                    const uint32_t bytes = static_cast<uint32_t>(rows * kRowBytes);
+                    const uint32_t bulk = bytes & ~15u;
+                    uint8_t* gdst = packed + tile * 128 * kRowBytes;
+                    const uint32_t ssrc = smem_u32(s_pk + pb * Lo::kPkBytes);
+                    if (bulk) bulk_store(gdst, ssrc, bulk);
+                    for (uint32_t o = bulk; o < bytes; o += 4)       // a ragged tail of whole words
+                        *reinterpret_cast<uint32_t*>(gdst + o) =
+                            *reinterpret_cast<const uint32_t*>(s_pk + pb * Lo::kPkBytes + o);
+                    bulk_commit();
+                    bulk_wait_read<1>();                          // the previous tile's buffer has been read
+                    if (li >= 1) mbar_arrive(b_pkempty + 8 * (pb ^ 1));
+                }
+            }
         }
+        if (staged && issuer) bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -395,10 +510,26 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
     }
 }
 
-template <int D>
-__host__ __device__ constexpr uint32_t dec_smem_bytes() {
+template <int D, int BITS>
+struct DecLayout {
     using C = KeyCfg<D>;
-    return C::kPiBytes + C::kDecBufs * C::kTileBytes + 256 * 4 + 8 * (2 * C::kDecBufs + 8) + 16 + 1024;
+    static constexpr int kRowBytes = D * BITS / 8;
+    static constexpr int kInBytes = 128 * kRowBytes + 128 * 4;            // packed rows + norms
+    static constexpr uint32_t kPit = 0;
+    static constexpr uint32_t kA = kPit + C::kPiBytes;
+    static constexpr uint32_t kIn = kA + C::kDecBufs * C::kTileBytes;
+    static constexpr uint32_t kPair = kIn + C::kDecInBufs * kInBytes;
+    static constexpr uint32_t kPatch = (kPair + 256 * 4 + 127) & ~127u;   // per-warp output transpose
+    static constexpr uint32_t kPatchBytes = 32 * 64;                      // 32 rows x 64 bytes
+    static constexpr uint32_t kBar = kPatch + C::kEpiWarps * kPatchBytes;
+    static constexpr int kBars = 2 * C::kDecBufs + 2 * C::kDecInBufs + 8;
+    static constexpr uint32_t kMisc = kBar + 8 * kBars;
+    static constexpr uint32_t kBytes = kMisc + 16 + 1024;
+};
+
+template <int D, int BITS>
+__host__ __device__ constexpr uint32_t dec_smem_bytes() {
+    return DecLayout<D, BITS>::kBytes;
 }
 
 template <int D, int BITS, bool OUT_F32>
@@ -407,19 +538,25 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
                     const uint8_t* __restrict__ packed, const float* __restrict__ norms, int64_t n,
                     void* __restrict__ out) {
     using C = KeyCfg<D>;
+    using Lo = DecLayout<D, BITS>;
     constexpr int NB = C::kDecBufs;
-    constexpr int kRowBytes = D * BITS / 8;
+    constexpr int NI = C::kDecInBufs;
+    constexpr int kRowBytes = Lo::kRowBytes;
     constexpr int kHalfWords = kRowBytes / 8;      // 32-bit words in half a packed row
     constexpr int kPairs = 1 << (2 * BITS);
+    constexpr int kOutBytes = OUT_F32 ? 4 : 2;
+    constexpr int kPasses = 32 * kOutBytes / 64;   // 64-byte row segments of one 32-column chunk
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* s_pit = smem;
-    uint8_t* s_a = s_pit + C::kPiBytes;
-    uint32_t* s_pair = reinterpret_cast<uint32_t*>(s_a + NB * C::kTileBytes);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(s_pair + 256);
-    const uint32_t b_afull = smem_u32(bars), b_aempty = b_afull + 8 * NB, b_accfull = b_aempty + 8 * NB,
-                   b_accempty = b_accfull + 16, b_pifull = b_accempty + 16, b_final = b_pifull + 8;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NB + 8);
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);   // stays a shared-space pointer
+    uint8_t* s_pit = smem + Lo::kPit;
+    uint8_t* s_a = smem + Lo::kA;
+    uint8_t* s_in = smem + Lo::kIn;
+    uint32_t* s_pair = reinterpret_cast<uint32_t*>(smem + Lo::kPair);
+    const uint32_t bar0 = smem_u32(smem + Lo::kBar);
+    const uint32_t b_afull = bar0, b_aempty = b_afull + 8 * NB, b_infull = b_aempty + 8 * NB,
+                   b_inempty = b_infull + 8 * NI, b_accfull = b_inempty + 8 * NI, b_accempty = b_accfull + 16,
+                   b_pifull = b_accempty + 16, b_final = b_pifull + 8;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lo::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -429,6 +566,10 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
         for (int b = 0; b < NB; ++b) {
             mbar_init(b_afull + 8 * b, C::kEpiWarps);
             mbar_init(b_aempty + 8 * b, 1);
+        }
+        for (int b = 0; b < NI; ++b) {
+            mbar_init(b_infull + 8 * b, 1);
+            mbar_init(b_inempty + 8 * b, C::kEpiWarps);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(b_accfull + 8 * a, 1);
@@ -449,11 +590,32 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
+    // a tile's packed rows and norms go through the staging buffer when both copies are 16-byte multiples
+    auto tile_rows = [&](int64_t tile) -> int64_t { return (n - tile * 128 < 128) ? n - tile * 128 : 128; };
+    auto bulk_ok = [&](int64_t rows) -> bool { return ((rows * kRowBytes) % 16 == 0) && ((rows * 4) % 16 == 0); };
+
     if (warp == 0) {
         if (lane == 0) {
+            // ---------------------------------------------------------------- producer
             mbar_arrive_expect_tx(b_pifull, C::kPiBytes);
             for (int kb = 0; kb < C::kKB; ++kb)
                 tma_load_2d(smem_u32(s_pit + kb * C::kPiBlockBytes), &tmap_pit, b_pifull, kb * 64, 0);
+            int li = 0;
+            for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
+                const int ib = li % NI;
+                if (!mbar_wait(b_inempty + 8 * ib, ((li / NI) & 1) ^ 1, abort_flag)) break;
+                const int64_t rows = tile_rows(tile);
+                if (bulk_ok(rows)) {
+                    const uint32_t pb = static_cast<uint32_t>(rows * kRowBytes), nbytes = static_cast<uint32_t>(rows * 4);
+                    mbar_arrive_expect_tx(b_infull + 8 * ib, pb + nbytes);
+                    uint8_t* dst = s_in + ib * Lo::kInBytes;
+                    bulk_load(smem_u32(dst), packed + tile * 128 * kRowBytes, pb, b_infull + 8 * ib);
+                    bulk_load(smem_u32(dst + 128 * kRowBytes), norms + tile * 128, nbytes, b_infull + 8 * ib);
+                } else {
+                    mbar_arrive(b_infull + 8 * ib);              // ragged tail: read straight from global
+                }
+            }
+            for (int k = (li > NI ? li - NI : 0); k < li; ++k) mbar_wait_drain(b_infull + 8 * (k % NI), (k / NI) & 1);
             mbar_wait_drain(b_pifull, 0);
         }
     } else if (warp == 1) {
@@ -485,19 +647,34 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
         const int quarter = warp & 3;
         const int half = ew >> 2;
         const int r = quarter * 32 + lane;
+        uint8_t* patch = smem + Lo::kPatch + ew * Lo::kPatchBytes;
+        float nrm_next = 0.f;
 
         // build the A tile (c_op[idx] as fp16, 128B-swizzled K-major) for local tile index lt
         auto build = [&](int lt, int64_t tile) -> bool {
-            const int b = lt % NB;
+            const int b = lt % NB, ib = lt % NI;
             if (!mbar_wait(b_aempty + 8 * b, ((lt / NB) & 1) ^ 1, abort_flag)) return false;
+            if (!mbar_wait(b_infull + 8 * ib, (lt / NI) & 1, abort_flag)) return false;
+            const int64_t rows = tile_rows(tile);
             const int64_t row = tile * 128 + r;
             uint32_t w[kHalfWords];
-            if (row < n) {
-                load_words<kHalfWords>(packed + row * kRowBytes + half * (kRowBytes / 2), w);
+            if (r < rows) {
+                if (bulk_ok(rows)) {
+                    const uint8_t* src = s_in + ib * Lo::kInBytes + r * kRowBytes + half * (kRowBytes / 2);
+#pragma unroll
+                    for (int i = 0; i < kHalfWords; ++i) w[i] = reinterpret_cast<const uint32_t*>(src)[i];
+                    nrm_next = reinterpret_cast<const float*>(s_in + ib * Lo::kInBytes + 128 * kRowBytes)[r];
+                } else {
+                    load_words<kHalfWords>(packed + row * kRowBytes + half * (kRowBytes / 2), w);
+                    nrm_next = norms[row];
+                }
             } else {
 #pragma unroll
                 for (int i = 0; i < kHalfWords; ++i) w[i] = 0u;
+                nrm_next = 0.f;
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_inempty + 8 * ib);
             uint8_t* as = s_a + b * C::kTileBytes;
 #pragma unroll
             for (int c = 0; c < C::kHalfCols / 8; ++c) {
@@ -519,11 +696,11 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
         if (tile < num_tiles) ok = build(0, tile);
         int li = 0;
         for (; ok && tile < num_tiles; tile += gridDim.x, ++li) {
+            const float nrm = nrm_next;
             const int64_t next = tile + gridDim.x;
             if (next < num_tiles && !build(li + 1, next)) break;
             const int a = li & 1;
-            const int64_t row = tile * 128 + r;
-            const float nrm = (row < n) ? norms[row] : 0.f;
+            const int64_t rows = tile_rows(tile);
             if (!mbar_wait(b_accfull + 8 * a, (li >> 1) & 1, abort_flag)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * D + half * C::kHalfCols;
@@ -532,33 +709,53 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(taddr + ch * 32, v);
                 tmem_ld_wait();
-                if (row < n) {
-                    const int col = half * C::kHalfCols + ch * 32;
-                    if constexpr (OUT_F32) {
-                        float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + row * D + col);
+                if (ch == C::kChunks - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(b_accempty + 8 * a);
+                }
+                // per 64-byte segment of this row's chunk: scale, convert, write it into the warp's patch as
+                // four 16-byte pieces (swizzled by row), then read the patch back row-contiguously (4 lanes per
+                // row, 8 rows per instruction) so each warp store covers whole 64-byte row segments
+                const int col0 = half * C::kHalfCols + ch * 32;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            o[i] = make_float4(__uint_as_float(v[4 * i]) * nrm, __uint_as_float(v[4 * i + 1]) * nrm,
-                                               __uint_as_float(v[4 * i + 2]) * nrm, __uint_as_float(v[4 * i + 3]) * nrm);
-                    } else {
-                        uint4* o = reinterpret_cast<uint4*>(static_cast<__half*>(out) + row * D + col);
+                for (int ps = 0; ps < kPasses; ++ps) {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            uint32_t pk[4];
+                    for (int pc = 0; pc < 4; ++pc) {
+                        uint4 pk;
+                        if constexpr (OUT_F32) {
+                            const int e0 = (ps * 4 + pc) * 4;
+                            pk = make_uint4(__float_as_uint(__uint_as_float(v[e0]) * nrm),
+                                            __float_as_uint(__uint_as_float(v[e0 + 1]) * nrm),
+                                            __float_as_uint(__uint_as_float(v[e0 + 2]) * nrm),
+                                            __float_as_uint(__uint_as_float(v[e0 + 3]) * nrm));
+                        } else {
+                            uint32_t hw[4];
 #pragma unroll
                             for (int k = 0; k < 4; ++k) {
-                                __half2 h2 = __floats2half2_rn(__uint_as_float(v[8 * i + 2 * k]) * nrm,
-                                                               __uint_as_float(v[8 * i + 2 * k + 1]) * nrm);
-                                pk[k] = *reinterpret_cast<uint32_t*>(&h2);
+                                __half2 h2 = __floats2half2_rn(__uint_as_float(v[8 * pc + 2 * k]) * nrm,
+                                                               __uint_as_float(v[8 * pc + 2 * k + 1]) * nrm);
+                                hw[k] = *reinterpret_cast<uint32_t*>(&h2);
                             }
-                            o[i] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            pk = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                        }
+                        *reinterpret_cast<uint4*>(patch + lane * 64 + ((pc ^ ((lane >> 1) & 3)) * 16)) = pk;
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int it = 0; it < 4; ++it) {
+                        const int rr = it * 8 + (lane >> 2), pc = lane & 3;
+                        const uint4 val = *reinterpret_cast<const uint4*>(patch + rr * 64 + ((pc ^ ((rr >> 1) & 3)) * 16));
+                        const int trow = quarter * 32 + rr;
+                        if (trow < rows) {
+                            uint8_t* gdst = static_cast<uint8_t*>(out) + ((tile * 128 + trow) * D + col0) * kOutBytes +
+                                            ps * 64 + pc * 16;
+                            *reinterpret_cast<uint4*>(gdst) = val;
                         }
                     }
+                    __syncwarp();
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b_accempty + 8 * a);
         }
     }
     tc_fence_before();

@@ -181,6 +181,57 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
+// --------------------------------------------------------------------------------- bit-field helpers
+
+// OR value v (< 2^BITS) into the little-endian bitstream `w` at field j (compile-time after unrolling).
+template <int BITS, int NW>
+__device__ __forceinline__ void put_field(uint32_t (&w)[NW], int j, uint32_t v) {
+    const int bit = j * BITS, wi = bit >> 5, sh = bit & 31;
+    w[wi] |= v << sh;
+    if (sh + BITS > 32) w[wi + 1] |= v >> (32 - sh);
+}
+
+// Field of width W starting at bit `bit` of the little-endian bitstream `w`.
+template <int W, int NW>
+__device__ __forceinline__ uint32_t get_bits(const uint32_t (&w)[NW], int bit) {
+    const int wi = bit >> 5, sh = bit & 31;
+    uint32_t v = w[wi] >> sh;
+    if (sh + W > 32) v |= w[wi + 1] << (32 - sh);
+    return (W == 32) ? v : (v & ((1u << W) - 1u));
+}
+
+// Store NW words (4-byte aligned destination; wider vectors where NW allows and `dst` is aligned to them).
+template <int NW>
+__device__ __forceinline__ void store_words(uint8_t* dst, const uint32_t (&w)[NW]) {
+    if constexpr (NW % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < NW; i += 4)
+            *reinterpret_cast<uint4*>(dst + 4 * i) = make_uint4(w[i], w[i + 1], w[i + 2], w[i + 3]);
+    } else if constexpr (NW == 2) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < NW; ++i) reinterpret_cast<uint32_t*>(dst)[i] = w[i];
+    }
+}
+
+template <int NW>
+__device__ __forceinline__ void load_words(const uint8_t* src, uint32_t (&w)[NW]) {
+    if constexpr (NW % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < NW; i += 4) {
+            uint4 v = *reinterpret_cast<const uint4*>(src + 4 * i);
+            w[i] = v.x; w[i + 1] = v.y; w[i + 2] = v.z; w[i + 3] = v.w;
+        }
+    } else if constexpr (NW == 2) {
+        uint2 v = *reinterpret_cast<const uint2*>(src);
+        w[0] = v.x; w[1] = v.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < NW; ++i) w[i] = reinterpret_cast<const uint32_t*>(src)[i];
+    }
+}
+
 // ------------------------------------------------------------------------------------- small helpers
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

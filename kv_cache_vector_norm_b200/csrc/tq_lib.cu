@@ -99,7 +99,7 @@ struct tq_codec {
     uint64_t seed = 0;
     __half* pi_op = nullptr;        // d x d, rotated = Pi_op x
     __half* pi_op_t = nullptr;      // Pi_op^T, the decode-side B operand
-    uint2* enc_lut = nullptr;       // 2048 grid cells {boundary bits, count below}
+    uint32_t* enc_lut = nullptr;    // 2048 grid cells: boundary bits | count below (low 4 bits)
     uint32_t* pair_lut = nullptr;   // 2^(2 bits) half2 pairs
     CUtensorMap tmap_pi, tmap_pit;
 };
@@ -107,9 +107,11 @@ struct tq_codec {
 namespace {
 
 // Grid table of the encode search (see encode_k_kernel): cell c holds the y with rint(512 y + 640) = c.
-tq_status build_grid_lut(int bits, const float* t, std::vector<uint2>& lut) {
+// Entry = bits of the one boundary inside the cell (+inf if none) OR the count of boundaries below the
+// cell; the boundaries, midpoints of fp16 levels, have at least 4 zero low bits in fp32 (checked).
+tq_status build_grid_lut(int bits, const float* t, std::vector<uint32_t>& lut) {
     const int nb = (1 << bits) - 1;
-    lut.assign(2048, make_uint2(0x7F800000u, static_cast<uint32_t>(nb)));
+    lut.assign(2048, 0x7F800000u | static_cast<uint32_t>(nb));
     for (int c = 0; c <= 1280; ++c) {
         const double lo = (c - 640.5) / 512.0, hi = (c - 639.5) / 512.0;
         uint32_t below = 0;
@@ -123,7 +125,8 @@ tq_status build_grid_lut(int bits, const float* t, std::vector<uint2>& lut) {
         if (inside > 1) return fail(TQ_ERR_UNSUPPORTED, "codebook boundaries closer than the search grid (bits=%d)", bits);
         uint32_t bb;
         std::memcpy(&bb, &b, 4);
-        lut[c] = make_uint2(bb, below);
+        if (bb & 15u) return fail(TQ_ERR_UNSUPPORTED, "a codebook boundary needs more than 28 significant bits");
+        lut[c] = bb | below;
     }
     return TQ_OK;
 }
@@ -150,7 +153,7 @@ extern "C" tq_status tq_codec_create(int d, int k_bits, uint64_t seed, tq_codec*
     std::vector<float> t(k - 1);
     tq_status st = tq_build_codebook(d, k_bits, nullptr, c16.data(), t.data(), nullptr);
     if (st != TQ_OK) return st;
-    std::vector<uint2> lut;
+    std::vector<uint32_t> lut;
     if ((st = build_grid_lut(k_bits, t.data(), lut)) != TQ_OK) return st;
     std::vector<uint32_t> pairs(1u << (2 * k_bits));
     for (uint32_t key = 0; key < pairs.size(); ++key)
@@ -166,12 +169,12 @@ extern "C" tq_status tq_codec_create(int d, int k_bits, uint64_t seed, tq_codec*
         return s;
     };
     if (cudaMalloc(&c->pi_op, dd * 2) != cudaSuccess || cudaMalloc(&c->pi_op_t, dd * 2) != cudaSuccess ||
-        cudaMalloc(&c->enc_lut, 2048 * sizeof(uint2)) != cudaSuccess ||
+        cudaMalloc(&c->enc_lut, 2048 * sizeof(uint32_t)) != cudaSuccess ||
         cudaMalloc(&c->pair_lut, pairs.size() * 4) != cudaSuccess)
         return cleanup(fail(TQ_ERR_CUDA, "tq_codec_create: cudaMalloc failed"));
     if (cudaMemcpy(c->pi_op, pi16.data(), dd * 2, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(c->pi_op_t, pit16.data(), dd * 2, cudaMemcpyHostToDevice) != cudaSuccess ||
-        cudaMemcpy(c->enc_lut, lut.data(), 2048 * sizeof(uint2), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->enc_lut, lut.data(), 2048 * sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(c->pair_lut, pairs.data(), pairs.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
         return cleanup(fail(TQ_ERR_CUDA, "tq_codec_create: cudaMemcpy failed"));
     if ((st = make_tmap_f16(&c->tmap_pi, c->pi_op, d, d, d, d)) != TQ_OK) return cleanup(st);
@@ -211,7 +214,7 @@ template <int D, int BITS>
 tq_status launch_encode_k(const tq_codec* c, const void* x, int64_t n, int64_t stride, const int64_t* slots,
                           uint8_t* packed, float* norms, cudaStream_t st) {
     static std::atomic<uint64_t> mask{0};
-    constexpr uint32_t smem = enc_smem_bytes<D>();
+    constexpr uint32_t smem = enc_smem_bytes<D, BITS>();
     auto kern = encode_k_kernel<D, BITS>;
     TQ_CUDA(allow_smem(kern, smem, mask), "tq_encode_k: cudaFuncSetAttribute");
     CUtensorMap tx;
@@ -219,7 +222,7 @@ tq_status launch_encode_k(const tq_codec* c, const void* x, int64_t n, int64_t s
     if (s != TQ_OK) return s;
     const int64_t tiles = (n + 127) / 128;
     const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-    kern<<<grid, KeyCfg<D>::kThreads, smem, st>>>(tx, c->tmap_pi, c->enc_lut, n, slots, packed, norms);
+    kern<<<grid, EncCfg<D>::kThreads, smem, st>>>(tx, c->tmap_pi, c->enc_lut, n, slots, packed, norms);
     TQ_CUDA(cudaGetLastError(), "tq_encode_k: launch");
     return TQ_OK;
 }
@@ -228,7 +231,7 @@ template <int D, int BITS>
 tq_status launch_decode_k(const tq_codec* c, const uint8_t* packed, const float* norms, int64_t n, void* out,
                           int dtype, cudaStream_t st) {
     static std::atomic<uint64_t> mask16{0}, mask32{0};
-    constexpr uint32_t smem = dec_smem_bytes<D>();
+    constexpr uint32_t smem = dec_smem_bytes<D, BITS>();
     const int64_t tiles = (n + 127) / 128;
     const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
     if (dtype == TQ_F32) {
@@ -290,8 +293,8 @@ extern "C" tq_status tq_decode_k(const tq_codec* c, const uint8_t* packed, const
     if (out_dtype != TQ_F16 && out_dtype != TQ_F32) return fail(TQ_ERR_INVALID_ARG, "tq_decode_k: out_dtype=%d", out_dtype);
     if (n == 0) return TQ_OK;
     if (!packed || !norms || !out) return fail(TQ_ERR_INVALID_ARG, "tq_decode_k: packed, norms and out must be non-NULL");
-    if (!aligned(packed, 16) || !aligned(norms, 4) || !aligned(out, 16))
-        return fail(TQ_ERR_INVALID_ARG, "tq_decode_k: packed and out must be 16-byte, norms 4-byte aligned");
+    if (!aligned(packed, 16) || !aligned(norms, 16) || !aligned(out, 16))
+        return fail(TQ_ERR_INVALID_ARG, "tq_decode_k: packed, norms and out must be 16-byte aligned");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     TQ_DISPATCH_DB(c->d, c->bits, launch_decode_k, c, packed, norms, n, out, out_dtype, st);
 }
@@ -309,7 +312,7 @@ int grid_for(int64_t units) {
 template <int D, int BITS, int GROUP>
 tq_status launch_encode_v(const void* x, int64_t n, int64_t stride, const int64_t* slots, uint8_t* data, void* scales,
                           void* zeros, cudaStream_t st) {
-    encode_v_kernel<D, BITS, GROUP><<<grid_for(n * (D / 32)), 256, 0, st>>>(
+    encode_v_kernel<D, BITS, GROUP><<<grid_for(n * (D / 16)), 256, 0, st>>>(
         static_cast<const __half*>(x), n, stride, slots, data, static_cast<__half*>(scales), static_cast<__half*>(zeros));
     TQ_CUDA(cudaGetLastError(), "tq_encode_v: launch");
     return TQ_OK;
@@ -318,7 +321,7 @@ tq_status launch_encode_v(const void* x, int64_t n, int64_t stride, const int64_
 template <int D, int BITS, int GROUP>
 tq_status launch_decode_v(const uint8_t* data, const void* scales, const void* zeros, int64_t n, void* out, int dtype,
                           cudaStream_t st) {
-    const int grid = grid_for(n * (D / 32));
+    const int grid = grid_for(n * (D / 8));
     if (dtype == TQ_F32)
         decode_v_kernel<D, BITS, GROUP, true><<<grid, 256, 0, st>>>(data, static_cast<const __half*>(scales),
                                                                     static_cast<const __half*>(zeros), n, out);
@@ -394,7 +397,7 @@ constexpr int kAttendCtasPerSm = 3;
 
 struct AttendPlan {
     int num_splits;
-    size_t counter_bytes, partial_bytes;
+    size_t partial_bytes;
 };
 
 tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan) {
@@ -425,10 +428,9 @@ tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan) {
     int64_t splits = (static_cast<int64_t>(sm_count()) * kAttendCtasPerSm + bh - 1) / bh;
     const int64_t by_len = (max_chunks + 7) / 8;            // at least ~8 chunks (128 tokens) per split
     if (splits > by_len) splits = by_len;
-    if (splits > 1024) splits = 1024;
+    if (splits > kMaxSplits) splits = kMaxSplits;
     if (splits < 1) splits = 1;
     plan->num_splits = static_cast<int>(splits);
-    plan->counter_bytes = ((static_cast<size_t>(bh) * 4 + 255) / 256) * 256;
     plan->partial_bytes = (splits > 1) ? static_cast<size_t>(bh) * splits * (16 + 8 * a->head_dim) * 4 : 0;
     return TQ_OK;
 }
@@ -459,12 +461,25 @@ tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const Attend
     p.v_scales = static_cast<const __half*>(a->v_scales);
     p.v_zeros = static_cast<const __half*>(a->v_zeros);
     p.out = a->out;
-    p.counters = static_cast<int*>(a->workspace);
-    p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(a->workspace) + plan.counter_bytes);
+    p.partials = static_cast<float*>(a->workspace);
     p.num_splits = plan.num_splits;
     dim3 grid(plan.num_splits, a->num_kv_heads, a->batch);
     kern<<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(p);
     TQ_CUDA(cudaGetLastError(), "tq_attend_decode: launch");
+    if (plan.num_splits > 1) {
+        // merge the splits in a programmatic dependent launch: it is scheduled while the main grid drains
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(p.group, a->num_kv_heads, a->batch);
+        cfg.blockDim = dim3(kMergeThreads);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        TQ_CUDA(cudaLaunchKernelEx(&cfg, attend_merge_kernel<D>, p), "tq_attend_decode: merge launch");
+    }
     return TQ_OK;
 }
 
@@ -486,11 +501,15 @@ tq_status attend_v(const tq_codec* c, const tq_attend_args* a, const AttendPlan&
 
 }  // namespace
 
-extern "C" size_t tq_attend_workspace_bytes(const tq_attend_args* a) {
+extern "C" tq_status tq_attend_workspace_bytes(const tq_attend_args* a, size_t* bytes) {
     clear_error();
+    if (!bytes) return fail(TQ_ERR_INVALID_ARG, "tq_attend_workspace_bytes: bytes is NULL");
+    *bytes = 0;
     AttendPlan plan;
-    if (plan_attend(a, &plan) != TQ_OK) return 0;
-    return plan.counter_bytes + plan.partial_bytes;
+    tq_status s = plan_attend(a, &plan);
+    if (s != TQ_OK) return s;
+    *bytes = plan.partial_bytes;
+    return TQ_OK;
 }
 
 extern "C" tq_status tq_attend_decode(const tq_codec* c, const tq_attend_args* a, void* stream) {
@@ -500,11 +519,11 @@ extern "C" tq_status tq_attend_decode(const tq_codec* c, const tq_attend_args* a
     tq_status s = plan_attend(a, &plan);
     if (s != TQ_OK) return s;
     if (a->head_dim != c->d) return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: head_dim=%d but the codec has d=%d", a->head_dim, c->d);
-    if (!a->q || !a->k_packed || !a->k_norms || !a->v_data || !a->v_scales || !a->v_zeros || !a->out || !a->workspace)
+    if (!a->q || !a->k_packed || !a->k_norms || !a->v_data || !a->v_scales || !a->v_zeros || !a->out)
         return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: NULL pointer in args");
-    if (a->workspace_bytes < plan.counter_bytes + plan.partial_bytes)
-        return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: workspace_bytes=%zu < %zu required", a->workspace_bytes,
-                    plan.counter_bytes + plan.partial_bytes);
+    if (plan.partial_bytes && (!a->workspace || a->workspace_bytes < plan.partial_bytes))
+        return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: workspace of %zu bytes required (got %zu)",
+                    plan.partial_bytes, a->workspace ? a->workspace_bytes : static_cast<size_t>(0));
     if (!aligned(a->q, 16) || !aligned(a->k_packed, 16) || !aligned(a->k_norms, 16) || !aligned(a->v_data, 16) ||
         !aligned(a->v_scales, 16) || !aligned(a->v_zeros, 16) || !aligned(a->out, 16) || !aligned(a->workspace, 16))
         return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: every pointer must be 16-byte aligned");

@@ -55,7 +55,7 @@ SIGNATURES = {
                                    ctypes.c_void_p]),
     "tq_decode_v": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
-    "tq_attend_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(AttendArgs)]),
+    "tq_attend_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(AttendArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "tq_attend_decode": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs), ctypes.c_void_p]),
     "tq_read_device_flag": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), ctypes.c_int]),
 }
@@ -257,15 +257,14 @@ def _attend_args(codec: Codec, q, cache: Cache, *, num_kv_heads, v_bits, v_group
 
 def attend_workspace_bytes(codec: Codec, q, cache: Cache, **kw) -> int:
     a = _attend_args(codec, q, cache, out=None, workspace=None, **kw)
-    nb = LIB.tq_attend_workspace_bytes(ctypes.byref(a))
-    if nb == 0:
-        raise TQError("tq_attend_workspace_bytes", TQ_ERR_INVALID_ARG)
-    return nb
+    nb = ctypes.c_size_t()
+    _check("tq_attend_workspace_bytes", LIB.tq_attend_workspace_bytes(ctypes.byref(a), ctypes.byref(nb)))
+    return nb.value
 
 
 def attend_workspace(codec: Codec, q, cache: Cache, **kw) -> torch.Tensor:
-    """A zero-filled workspace of the size tq_attend_workspace_bytes asks for."""
-    return torch.zeros(attend_workspace_bytes(codec, q, cache, **kw), dtype=torch.uint8, device=q.device)
+    """A workspace of the size tq_attend_workspace_bytes asks for (at least 16 bytes)."""
+    return torch.empty(max(16, attend_workspace_bytes(codec, q, cache, **kw)), dtype=torch.uint8, device=q.device)
 
 
 def attend_decode(codec: Codec, q: torch.Tensor, cache: Cache, *, num_kv_heads: int, v_bits: int, v_group: int = 32,

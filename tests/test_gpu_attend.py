@@ -100,7 +100,9 @@ def test_attend_repeated_calls_are_identical():
     a = tq.attend_decode(cd, q, cache, num_kv_heads=2, v_bits=2, max_seq_len=2048, workspace=ws).clone()
     b = tq.attend_decode(cd, q, cache, num_kv_heads=2, v_bits=2, max_seq_len=2048, workspace=ws)
     assert torch.equal(a, b)
-    assert int(ws[:8].view(torch.int32).abs().sum()) == 0           # split counters left zeroed
+    ws.fill_(0xFF)                                                   # stale workspace contents do not matter
+    c = tq.attend_decode(cd, q, cache, num_kv_heads=2, v_bits=2, max_seq_len=2048, workspace=ws)
+    assert torch.equal(a, c)
 
 
 def test_attend_paged():

@@ -66,12 +66,15 @@ def test_argument_errors_are_reported():
     a = tq.AttendArgs()
     a.batch, a.num_q_heads, a.num_kv_heads, a.head_dim, a.v_bits, a.v_group = 1, 12, 1, 128, 2, 32
     a.max_seq_len = 64
-    assert tq.LIB.tq_attend_workspace_bytes(ctypes.byref(a)) == 0          # GQA group 12 > 8
+    nb = ctypes.c_size_t(123)
+    assert tq.LIB.tq_attend_workspace_bytes(ctypes.byref(a), ctypes.byref(nb)) == tq.TQ_ERR_UNSUPPORTED  # GQA 12 > 8
+    assert nb.value == 0
     a.num_q_heads = 8
     a.max_seq_len = 40
-    assert tq.LIB.tq_attend_workspace_bytes(ctypes.byref(a)) == 0          # not a multiple of 16
-    a.max_seq_len = 64
-    assert tq.LIB.tq_attend_workspace_bytes(ctypes.byref(a)) > 0
+    assert tq.LIB.tq_attend_workspace_bytes(ctypes.byref(a), ctypes.byref(nb)) == tq.TQ_ERR_INVALID_ARG  # not 16k
+    a.max_seq_len = 4096
+    assert tq.LIB.tq_attend_workspace_bytes(ctypes.byref(a), ctypes.byref(nb)) == tq.TQ_OK
+    assert nb.value > 0                                                     # one sequence: split over the SMs
     assert tq.LIB.tq_attend_decode(None, ctypes.byref(a), None) == tq.TQ_ERR_INVALID_ARG
     assert tq.LIB.tq_codec_create(96, 4, 0, ctypes.byref(ctypes.c_void_p())) == tq.TQ_ERR_UNSUPPORTED
     assert tq.LIB.tq_codec_create(128, 5, 0, ctypes.byref(ctypes.c_void_p())) == tq.TQ_ERR_UNSUPPORTED
