@@ -12,22 +12,13 @@ namespace dev {
 // (4 for group 32, d/8 for the per-token layout) reduce min/max with shuffles.  Every arithmetic step is
 // the page's fp32 operation with one rounding.
 
-// Code of one element: round_half_even(a / s) with the page's IEEE fp32 division, for 0 <= a <= (2^b - 1) s.
-// Fast path: with r = RN(1/s) the product qa = RN(a r) is within 2^-22 (relative) of RN(a / s); adding
-// 1.5 * 2^23 rounds qa to the nearest integer (ties to even) in the low mantissa bits, and when qa lies
-// farther than 2^-21 qa from the half-integers both qa and RN(a / s) round to that same integer.
-// Otherwise (rare) the exact quotient is rounded.  Returns the integer code.
-__device__ __forceinline__ uint32_t quant_code(float a, float s, float r) {
-    constexpr float kMagic = 12582912.0f;                  // 1.5 * 2^23
-    const float qa = __fmul_rn(a, r);
-    const float t = __fadd_rn(qa, kMagic);
-    const float k = __fsub_rn(t, kMagic);
-    const float dev = fabsf(__fsub_rn(qa, k));
-    uint32_t code = __float_as_uint(t) - 0x4B400000u;
-    if (!(__fmaf_rn(qa, 4.76837158203125e-7f, dev) < 0.5f))
-        code = __float_as_uint(__fadd_rn(rintf(__fdiv_rn(a, s)), kMagic)) - 0x4B400000u;
-    return code;
-}
+// Codes of a group: round_half_even(a / s) with the page's IEEE fp32 division, 0 <= a <= (2^b - 1) s.
+// With r = RN(1/s), the products a RN(r (1 -+ 2^-21)) bracket RN(a / s) (each end is off by at most
+// 3 * 2^-23 relative, inside the 2^-21 bracket); an FMA adding 1.5 * 2^23 rounds each end to the nearest
+// integer (ties to even) in its low mantissa bits.  Rounding is monotonic, so when both ends give the same
+// integer, RN(a / s) rounds to it as well; otherwise the caller recomputes with the exact quotient.
+constexpr float kCodeMagic = 12582912.0f;                   // 1.5 * 2^23
+constexpr uint32_t kCodeMagicBits = 0x4B400000u;
 
 template <int D, int GROUP>
 struct VLanes {
@@ -96,15 +87,29 @@ __global__ void __launch_bounds__(256) encode_v_kernel(const __half* __restrict_
         scale = fmaxf(scale, 1e-12f);
         const float zero = vmin;
         const float rcp = __frcp_rn(scale);
+        const float r_lo = __fmul_rn(rcp, 0.99999952316284180f);   // 1 - 2^-21
+        const float r_hi = __fmul_rn(rcp, 1.00000047683715820f);   // 1 + 2^-21
         uint32_t chunk[kW];
 #pragma unroll
         for (int k = 0; k < kW; ++k) chunk[k] = 0u;
+        bool exact = true;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            // the page clamps to [0, 2^b - 1]; with a in [0, max - min] the code can only exceed the top
-            // level through rounding, so one min() keeps the clamp
-            const uint32_t q = min(quant_code(__fsub_rn(v[k], zero), scale, rcp), kLevels);
-            put_field<BITS>(chunk, k, q);
+            const float a = __fsub_rn(v[k], zero);
+            const float tlo = __fmaf_rn(a, r_lo, kCodeMagic);
+            const float thi = __fmaf_rn(a, r_hi, kCodeMagic);
+            exact &= (__float_as_uint(tlo) == __float_as_uint(thi));
+            // the code never exceeds 2^b - 1 (a <= max - min), so masking the low bits is the page's clamp
+            put_field<BITS>(chunk, k, __float_as_uint(tlo) & kLevels);
+        }
+        if (!exact) {
+#pragma unroll
+            for (int k = 0; k < kW; ++k) chunk[k] = 0u;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float q = rintf(__fdiv_rn(__fsub_rn(v[k], zero), scale));
+                put_field<BITS>(chunk, k, static_cast<uint32_t>(fminf(fmaxf(q, 0.f), static_cast<float>(kLevels))));
+            }
         }
         const int64_t orow = valid ? (slots ? slots[row] : row) : -1;
         uint8_t* dst = data + orow * kRowBytes;
