@@ -226,6 +226,36 @@ tq_status tq_attend_workspace_bytes(const tq_attend_args* args, size_t* bytes);
  */
 tq_status tq_attend_decode(const tq_codec* codec, const tq_attend_args* args, void* stream);
 
+/*
+ * TQ_ATTEND_SCRATCH_BYTES -- size of the library-owned scratch used by tq_attend_decode_noalloc (4 MiB).
+ * That array lives in the library's device image, so every GPU that loads libtq holds it until the process
+ * exits, whether or not the entry point is ever called.
+ */
+#define TQ_ATTEND_SCRATCH_BYTES (4u << 20)
+
+/*
+ * tq_attend_decode_noalloc -- the same decode-step attention as tq_attend_decode, for callers that cannot
+ * allocate device memory at all: code running inside a CUDA graph that is being captured or replayed, a
+ * serving loop whose memory pool is fixed once at start-up, or a host process that only receives a
+ * stream and buffers from elsewhere.  The pages have no counterpart; this is a property of this library.
+ *
+ * Instead of a caller workspace it uses a fixed scratch array of TQ_ATTEND_SCRATCH_BYTES that the library
+ * declares at file scope in device memory; args->workspace and args->workspace_bytes are ignored.  The
+ * entry point calls no allocator (no cudaMalloc, no cudaFree, nothing that allocates).
+ *   - Set-up: the first call on each device looks up the scratch array's device address with
+ *     cudaGetSymbolAddress (with that device current) and caches it; make that first call outside any
+ *     stream capture.
+ *   - Limit: a launch whose split-K partials need more than TQ_ATTEND_SCRATCH_BYTES (see
+ *     tq_attend_workspace_bytes) is rejected with TQ_ERR_INVALID_ARG and a message giving both sizes;
+ *     use tq_attend_decode with a caller workspace for such shapes.
+ *   - Sharing: all calls on a device share the one array and it keeps the last call's partials; nothing
+ *     in it needs to start at zero, since every launch overwrites the part it reads.  Calls that can
+ *     overlap on the GPU (different streams without ordering, or different threads) race on it and must
+ *     be serialised by the caller.
+ * Errors: as tq_attend_decode, plus TQ_ERR_CUDA if the address lookup fails.
+ */
+tq_status tq_attend_decode_noalloc(const tq_codec* codec, const tq_attend_args* args, void* stream);
+
 /* --------------------------------------------------------------------------------------------------
  * Diagnostics.
  * ------------------------------------------------------------------------------------------------ */

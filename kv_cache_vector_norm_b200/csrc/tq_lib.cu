@@ -545,6 +545,53 @@ extern "C" tq_status tq_attend_decode(const tq_codec* c, const tq_attend_args* a
     }
 }
 
+// ---------------------------------------------------------------------- attention without allocation
+
+// Scratch for tq_attend_decode_noalloc: part of this library's device image, so it exists on every device
+// that loads the library, without any allocation call by the entry point.
+static __device__ __align__(256) unsigned char g_attend_scratch[TQ_ATTEND_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_attend_scratch on the current device, looked up once per device.  In host code the
+// array's name is only a stand-in, never a device address, so kernels must receive this pointer.
+tq_status attend_scratch(void** out) {
+    static std::mutex mu;
+    static std::vector<void*> addr;
+    int dev = 0;
+    TQ_CUDA(cudaGetDevice(&dev), "tq_attend_decode_noalloc: cudaGetDevice");
+    std::lock_guard<std::mutex> lk(mu);
+    if (static_cast<int>(addr.size()) <= dev) addr.resize(dev + 1, nullptr);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        TQ_CUDA(cudaGetSymbolAddress(&p, g_attend_scratch), "tq_attend_decode_noalloc: cudaGetSymbolAddress");
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" tq_status tq_attend_decode_noalloc(const tq_codec* c, const tq_attend_args* a, void* stream) {
+    clear_error();
+    if (!c) return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode_noalloc: codec is NULL");
+    AttendPlan plan;
+    tq_status s = plan_attend(a, &plan);
+    if (s != TQ_OK) return s;
+    if (plan.partial_bytes > TQ_ATTEND_SCRATCH_BYTES)
+        return fail(TQ_ERR_INVALID_ARG,
+                    "tq_attend_decode_noalloc: this launch needs %zu bytes of split-K scratch but the static scratch "
+                    "holds %u; use tq_attend_decode with a workspace",
+                    plan.partial_bytes, TQ_ATTEND_SCRATCH_BYTES);
+    void* scratch = nullptr;
+    if ((s = attend_scratch(&scratch)) != TQ_OK) return s;
+    tq_attend_args with_scratch = *a;
+    with_scratch.workspace = scratch;
+    with_scratch.workspace_bytes = TQ_ATTEND_SCRATCH_BYTES;
+    return tq_attend_decode(c, &with_scratch, stream);
+}
+
 // --------------------------------------------------------------------------------------- diagnostics
 
 extern "C" tq_status tq_read_device_flag(int* flag_out, int clear) {

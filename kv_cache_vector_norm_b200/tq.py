@@ -57,6 +57,7 @@ SIGNATURES = {
                                    ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]),
     "tq_attend_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(AttendArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "tq_attend_decode": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs), ctypes.c_void_p]),
+    "tq_attend_decode_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs), ctypes.c_void_p]),
     "tq_read_device_flag": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), ctypes.c_int]),
 }
 
@@ -281,6 +282,27 @@ def attend_decode(codec: Codec, q: torch.Tensor, cache: Cache, *, num_kv_heads: 
         workspace = attend_workspace(codec, q, cache, **kw)
     a = _attend_args(codec, q, cache, out=out, workspace=workspace, **kw)
     _check("tq_attend_decode", LIB.tq_attend_decode(codec.handle, ctypes.byref(a), _stream(q.device)))
+    return out
+
+
+ATTEND_SCRATCH_BYTES = 4 << 20
+
+
+def attend_decode_noalloc(codec: Codec, q: torch.Tensor, cache: Cache, *, num_kv_heads: int, v_bits: int,
+                          v_group: int = 32, max_seq_len: int | None = None, block_table: torch.Tensor | None = None,
+                          seq_lens: torch.Tensor | None = None, scale: float = 0.0,
+                          out: torch.Tensor | None = None) -> torch.Tensor:
+    """attend_decode without a workspace: the library's fixed device scratch (ATTEND_SCRATCH_BYTES) holds the
+    split-K partials, so the call itself allocates nothing on the device; for callers that cannot allocate
+    (graph capture or replay, fixed memory pools).  Calls that overlap on the GPU share that scratch and
+    must be serialised.  `out` should be passed in by such callers, since creating it here allocates."""
+    _need_cuda(q, "q", torch.float16)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    a = _attend_args(codec, q, cache, num_kv_heads=num_kv_heads, v_bits=v_bits, v_group=v_group,
+                     max_seq_len=max_seq_len, block_table=block_table, seq_lens=seq_lens, scale=scale, out=out,
+                     workspace=None)
+    _check("tq_attend_decode_noalloc", LIB.tq_attend_decode_noalloc(codec.handle, ctypes.byref(a), _stream(q.device)))
     return out
 
 
