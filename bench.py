@@ -187,6 +187,9 @@ def gpu_arm(args, w, rank, world, local_rank):
         ("attend", lambda: tq.attend_decode(codec, q, cache, out=out, workspace=ws, **akw)),
     ]
 
+    if args.only:
+        kernels = [kv for kv in kernels if kv[0] == args.only]
+
     def one_step(record):
         for name, fn in kernels:
             flush_buf.fill_(1)
@@ -219,6 +222,8 @@ def gpu_arm(args, w, rank, world, local_rank):
     per = {name: 0.0 for name, _ in kernels}
     for name, e0, e1 in events:
         per[name] += e0.elapsed_time(e1)
+    if args.only:
+        return dict(per=per, launch_ms=[e0.elapsed_time(e1) for _, e0, e1 in events], n=n)
     total_ms = sum(per.values())
     if world > 1:
         tt = torch.tensor([total_ms], device=dev)
@@ -334,6 +339,8 @@ def main():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--workload", default="70b_decode_128k", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["encode_k", "encode_v", "decode_k", "decode_v", "attend"],
+                    help="time one kernel of the path alone (profiling aid; prints its per-launch times)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -379,6 +386,13 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     r = gpu_arm(args, w, rank, world, local_rank)
+    if args.only:
+        if rank == 0:
+            bpv_k = algorithmic_bytes(w)[args.only]
+            ms = [round(x, 5) for x in r["launch_ms"]]
+            print(json.dumps({"mode": "single-kernel", "kernel": args.only, "workload": args.workload,
+                              "launch_ms": ms, "GBps_median": bpv_k * r["n"] / (statistics.median(ms) / 1e3) / 1e9}))
+        return
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

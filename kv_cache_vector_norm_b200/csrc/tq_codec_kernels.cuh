@@ -515,9 +515,20 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
     }
 }
 
+// Decode CTA: warp 0 producer, warp 1 TMEM owner + MMA issuer, warps 2.. builders/epilogue (kEpiWarps:
+// warp w works on rows 32*(w%4).. and owns kCols columns of them).
+template <int D>
+struct DecCfg {
+    static constexpr int kEpiWarps = (D == 128) ? 16 : 8;
+    static constexpr int kThreads = 32 * (2 + kEpiWarps);
+    static constexpr int kCols = D * 4 / kEpiWarps;          // 32, 32, 128
+    static constexpr int kChunks = kCols / 32;
+};
+
 template <int D, int BITS>
 struct DecLayout {
     using C = KeyCfg<D>;
+    using E = DecCfg<D>;
     static constexpr int kRowBytes = D * BITS / 8;
     static constexpr int kInBytes = 128 * kRowBytes + 128 * 4;            // packed rows + norms
     static constexpr uint32_t kPit = 0;
@@ -526,7 +537,7 @@ struct DecLayout {
     static constexpr uint32_t kPair = kIn + C::kDecInBufs * kInBytes;
     static constexpr uint32_t kPatch = (kPair + 256 * 4 + 127) & ~127u;   // per-warp output transpose
     static constexpr uint32_t kPatchBytes = 32 * 64;                      // 32 rows x 64 bytes
-    static constexpr uint32_t kBar = kPatch + C::kEpiWarps * kPatchBytes;
+    static constexpr uint32_t kBar = kPatch + E::kEpiWarps * kPatchBytes;
     static constexpr int kBars = 2 * C::kDecBufs + 2 * C::kDecInBufs + 8;
     static constexpr uint32_t kMisc = kBar + 8 * kBars;
     static constexpr uint32_t kBytes = kMisc + 16 + 1024;
@@ -538,16 +549,17 @@ __host__ __device__ constexpr uint32_t dec_smem_bytes() {
 }
 
 template <int D, int BITS, bool OUT_F32>
-__global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
+__global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
     decode_k_kernel(const __grid_constant__ CUtensorMap tmap_pit, const uint32_t* __restrict__ pair_lut_g,
                     const uint8_t* __restrict__ packed, const float* __restrict__ norms, int64_t n,
                     void* __restrict__ out) {
     using C = KeyCfg<D>;
+    using E = DecCfg<D>;
     using Lo = DecLayout<D, BITS>;
     constexpr int NB = C::kDecBufs;
     constexpr int NI = C::kDecInBufs;
     constexpr int kRowBytes = Lo::kRowBytes;
-    constexpr int kHalfWords = kRowBytes / 8;      // 32-bit words in half a packed row
+    constexpr int kPartWords = E::kCols * BITS / 32;   // 32-bit words of this warp's columns of a packed row
     constexpr int kPairs = 1 << (2 * BITS);
     constexpr int kOutBytes = OUT_F32 ? 4 : 2;
     constexpr int kPasses = 32 * kOutBytes / 64;   // 64-byte row segments of one 32-column chunk
@@ -569,16 +581,16 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < NB; ++b) {
-            mbar_init(b_afull + 8 * b, C::kEpiWarps);
+            mbar_init(b_afull + 8 * b, E::kEpiWarps);
             mbar_init(b_aempty + 8 * b, 1);
         }
         for (int b = 0; b < NI; ++b) {
             mbar_init(b_infull + 8 * b, 1);
-            mbar_init(b_inempty + 8 * b, C::kEpiWarps);
+            mbar_init(b_inempty + 8 * b, E::kEpiWarps);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(b_accfull + 8 * a, 1);
-            mbar_init(b_accempty + 8 * a, C::kEpiWarps);
+            mbar_init(b_accempty + 8 * a, E::kEpiWarps);
         }
         mbar_init(b_pifull, 1);
         mbar_init(b_final, 1);
@@ -650,7 +662,7 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
     } else {
         const int ew = warp - 2;
         const int quarter = warp & 3;
-        const int half = ew >> 2;
+        const int c0 = (ew >> 2) * E::kCols;               // first column of this warp
         const int r = quarter * 32 + lane;
         uint8_t* patch = smem + Lo::kPatch + ew * Lo::kPatchBytes;
         float nrm_next = 0.f;
@@ -662,31 +674,31 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
             if (!mbar_wait(b_infull + 8 * ib, (lt / NI) & 1, abort_flag)) return false;
             const int64_t rows = tile_rows(tile);
             const int64_t row = tile * 128 + r;
-            uint32_t w[kHalfWords];
+            uint32_t w[kPartWords];
             if (r < rows) {
                 if (bulk_ok(rows)) {
-                    const uint8_t* src = s_in + ib * Lo::kInBytes + r * kRowBytes + half * (kRowBytes / 2);
+                    const uint8_t* src = s_in + ib * Lo::kInBytes + r * kRowBytes + c0 * BITS / 8;
 #pragma unroll
-                    for (int i = 0; i < kHalfWords; ++i) w[i] = reinterpret_cast<const uint32_t*>(src)[i];
+                    for (int i = 0; i < kPartWords; ++i) w[i] = reinterpret_cast<const uint32_t*>(src)[i];
                     nrm_next = reinterpret_cast<const float*>(s_in + ib * Lo::kInBytes + 128 * kRowBytes)[r];
                 } else {
-                    load_words<kHalfWords>(packed + row * kRowBytes + half * (kRowBytes / 2), w);
+                    load_words<kPartWords>(packed + row * kRowBytes + c0 * BITS / 8, w);
                     nrm_next = norms[row];
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < kHalfWords; ++i) w[i] = 0u;
+                for (int i = 0; i < kPartWords; ++i) w[i] = 0u;
                 nrm_next = 0.f;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(b_inempty + 8 * ib);
             uint8_t* as = s_a + b * C::kTileBytes;
 #pragma unroll
-            for (int c = 0; c < C::kHalfCols / 8; ++c) {
+            for (int c = 0; c < E::kCols / 8; ++c) {
                 uint32_t h[4];
 #pragma unroll
                 for (int p = 0; p < 4; ++p) h[p] = s_pair[get_bits<2 * BITS>(w, (c * 8 + 2 * p) * BITS)];
-                const int col = half * C::kHalfCols + c * 8;
+                const int col = c0 + c * 8;
                 *reinterpret_cast<uint4*>(as + (col >> 6) * C::kTileBlockBytes + sw128_offset(r, (col & 63) >> 3)) =
                     make_uint4(h[0], h[1], h[2], h[3]);
             }
@@ -708,13 +720,13 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
             const int64_t rows = tile_rows(tile);
             if (!mbar_wait(b_accfull + 8 * a, (li >> 1) & 1, abort_flag)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * D + half * C::kHalfCols;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * D + c0;
 #pragma unroll
-            for (int ch = 0; ch < C::kChunks; ++ch) {
+            for (int ch = 0; ch < E::kChunks; ++ch) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(taddr + ch * 32, v);
                 tmem_ld_wait();
-                if (ch == C::kChunks - 1) {
+                if (ch == E::kChunks - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(b_accempty + 8 * a);
@@ -722,7 +734,7 @@ __global__ void __launch_bounds__(KeyCfg<D>::kThreads, 1)
                 // per 64-byte segment of this row's chunk: scale, convert, write it into the warp's patch as
                 // four 16-byte pieces (swizzled by row), then read the patch back row-contiguously (4 lanes per
                 // row, 8 rows per instruction) so each warp store covers whole 64-byte row segments
-                const int col0 = half * C::kHalfCols + ch * 32;
+                const int col0 = c0 + ch * 32;
 #pragma unroll
                 for (int ps = 0; ps < kPasses; ++ps) {
 #pragma unroll

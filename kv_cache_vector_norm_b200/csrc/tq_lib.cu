@@ -237,11 +237,11 @@ tq_status launch_decode_k(const tq_codec* c, const uint8_t* packed, const float*
     if (dtype == TQ_F32) {
         auto kern = decode_k_kernel<D, BITS, true>;
         TQ_CUDA(allow_smem(kern, smem, mask32), "tq_decode_k: cudaFuncSetAttribute");
-        kern<<<grid, KeyCfg<D>::kThreads, smem, st>>>(c->tmap_pit, c->pair_lut, packed, norms, n, out);
+        kern<<<grid, DecCfg<D>::kThreads, smem, st>>>(c->tmap_pit, c->pair_lut, packed, norms, n, out);
     } else {
         auto kern = decode_k_kernel<D, BITS, false>;
         TQ_CUDA(allow_smem(kern, smem, mask16), "tq_decode_k: cudaFuncSetAttribute");
-        kern<<<grid, KeyCfg<D>::kThreads, smem, st>>>(c->tmap_pit, c->pair_lut, packed, norms, n, out);
+        kern<<<grid, DecCfg<D>::kThreads, smem, st>>>(c->tmap_pit, c->pair_lut, packed, norms, n, out);
     }
     TQ_CUDA(cudaGetLastError(), "tq_decode_k: launch");
     return TQ_OK;
