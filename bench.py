@@ -62,10 +62,21 @@ def peaks():
         return 6650.0, "fallback (6.65 TB/s)"
 
 
-def source_hash():
+# sources each kernel's code and launch configuration come from: a recorded DRAM traffic figure stays valid
+# only while these files are unchanged
+KERNEL_SOURCES = {
+    "encode_k": ("tq_device.cuh", "tq_codec_kernels.cuh", "tq_lib.cu"),
+    "decode_k": ("tq_device.cuh", "tq_codec_kernels.cuh", "tq_lib.cu"),
+    "encode_v": ("tq_device.cuh", "tq_codec_kernels.cuh", "tq_lib.cu"),
+    "decode_v": ("tq_device.cuh", "tq_codec_kernels.cuh", "tq_lib.cu"),
+    "attend": ("tq_device.cuh", "tq_attend_kernel.cuh", "tq_lib.cu"),
+}
+
+
+def source_hash(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kv_cache_vector_norm_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -78,7 +89,7 @@ def traffic_record(kernel, workload):
         with open(path) as f:
             rec = json.load(f)
         e = rec.get(workload, {}).get(kernel)
-        if e and e.get("source_hash") == source_hash():
+        if e and e.get("source_hash") == source_hash(kernel):
             return e["dram_bytes_per_launch"]
     except Exception:
         pass
