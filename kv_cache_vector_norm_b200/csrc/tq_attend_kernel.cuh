@@ -7,11 +7,12 @@
 // ever materialised:
 //   score_t = scale * n_t * <Pi_op q, c_op[idx_t]>       (tensor cores: fp16 codebook values x fp16
 //                                                         hi/lo halves of the rotated query)
-//   out     = sum_t p_t (q_t s_t + z_t) / sum_t p_t       (tensor cores: integer codes x bf16 hi/lo
-//                                                         halves of p_t s_t; the zero term on FMAs)
+//   out     = sum_t p_t (q_t s_t + z_t) / sum_t p_t       (tensor cores: integer codes, exact as bf16
+//                                                         subnormals, x bf16 hi/lo halves of p_t s_t;
+//                                                         the zero term on FMAs)
 // One CTA = one (split, kv head, sequence); warp 4 streams 16-token chunks of every pool array into a
 // shared-memory ring with bulk TMA copies; warps 0..3 each consume one chunk of every stage with
-// mma.sync fragments kept in registers; the last CTA of a (sequence, kv head) merges the splits.
+// mma.sync fragments kept in registers; a second kernel merges the splits.
 #pragma once
 
 #include "tq_device.cuh"
@@ -61,22 +62,26 @@ struct AttCfg {
     static constexpr int kQuarterWords = (kQuarterHalves + 1) / 2 + 1;
     static constexpr int kMinBlocks = (D == 256) ? 1 : 3;
     static constexpr int kPartFloats = 16 + 8 * D;
-    // key lookups: 4 codes -> two half2 (KB <= 3), else 2 codes -> one half2
-    static constexpr bool kQuad = (KB <= 3);
-    static constexpr int kLutBytes = kQuad ? (1 << (4 * KB)) * 8 : (1 << (2 * KB)) * 4;
-    // shared memory: stages | q fragments | rotated q | key table | pair table | reduction | barriers
+    static constexpr bool kQInRegs = (D <= 128);     // score A fragments held in registers
+    // key table: a pair of codes (2 KB bits, first code in the low bits) -> half2 of codebook values, with one
+    // copy per shared-memory bank (entry e of lane l at byte 128 e + 4 l), so lookups never conflict
+    static constexpr int kPairs = 1 << (2 * KB);
+    static constexpr int kLutBytes = kPairs * 128;
+    // shared memory: stages | q fragments | rotated q | key table (aligned to its size at run time) |
+    // per-warp zero sums | reduction | barriers
     static constexpr int kCombineFloats = kWarps * kPartFloats;
     static constexpr int kRingBytes =
         (kStages * kStageBytes > kCombineFloats * 4) ? kStages * kStageBytes : kCombineFloats * 4;
     static constexpr int kQfOff = kRingBytes;
     static constexpr int kQrOff = kQfOff + (D / 16) * 32 * 16;
     static constexpr int kLutOff = kQrOff + 8 * D * 4;
-    static constexpr int kPairOff = kLutOff + kLutBytes;
-    static constexpr int kRedOff = kPairOff + (1 << (2 * KB)) * 4;
+    static constexpr int kZsOff = kLutOff + 2 * kLutBytes;
+    static constexpr int kRedOff = kZsOff + kWarps * 8 * kVGroups * 4;
     static constexpr int kBarOff = (kRedOff + 8 * 4 + 15) & ~15;
     static constexpr int kSmem = kBarOff + 8 * (2 * kStages) + 16;
     static_assert(kNOff % 16 == 0 && kVOff % 16 == 0 && kSOff % 16 == 0 && kZOff % 16 == 0 && kStageBytes % 16 == 0,
                   "bulk copies need 16-byte multiples");
+    static_assert(VG % 32 == 0, "a 32-column slice of the value row lies in one scale group");
 };
 
 __device__ __forceinline__ void mma_f16(float (&c)[4], const uint4& a, uint32_t b0, uint32_t b1) {
@@ -105,61 +110,24 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// hi/lo bf16 split of two values: hi = bf16(x), lo = bf16(x - hi)
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// hi/lo bf16 split of two values: hi = x truncated to bf16 (the upper 16 bits), lo = bf16(x - hi);
+// hi + lo is within 2^-16 |x| of x
 __device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-    hi = pack_bf16(x0, x1);
-    const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xFFFF0000u);
-    lo = pack_bf16(x0 - h0, x1 - h1);
-}
-
-// Value codes of one 32-column slice of a row: 32 * VB bits as words.
-template <int VB>
-struct VSlice {
-    static constexpr int kWords = VB;            // 32 columns x VB bits = VB words
-};
-
-template <int VB>
-__device__ __forceinline__ void load_vslice(const uint8_t* row, int slice, uint32_t (&w)[VB]) {
-    const uint8_t* p = row + slice * 4 * VB;     // 32 * VB bits = 4 * VB bytes, 4-byte aligned
-    if constexpr (VB == 2) {
-        const uint2 t = *reinterpret_cast<const uint2*>(p);
-        w[0] = t.x; w[1] = t.y;
-    } else if constexpr (VB == 4) {
-        const uint4 t = *reinterpret_cast<const uint4*>(p);
-        w[0] = t.x; w[1] = t.y; w[2] = t.z; w[3] = t.w;
-    } else if constexpr (VB == 8) {
-        const uint4 t0 = reinterpret_cast<const uint4*>(p)[0], t1 = reinterpret_cast<const uint4*>(p)[1];
-        w[0] = t0.x; w[1] = t0.y; w[2] = t0.z; w[3] = t0.w; w[4] = t1.x; w[5] = t1.y; w[6] = t1.z; w[7] = t1.w;
-    } else {
-#pragma unroll
-        for (int i = 0; i < VB; ++i) w[i] = reinterpret_cast<const uint32_t*>(p)[i];
-    }
-}
-
-// bf16x2 {code_a[c], code_b[c]} for column c (0..31) of a slice held in registers (exact small integers).
-template <int VB>
-__device__ __forceinline__ uint32_t vcode_pair(const uint32_t (&wa)[VB], const uint32_t (&wb)[VB], int c) {
-    const int bit = c * VB;
-    if constexpr (VB == 2 || VB == 4) {
-        const uint32_t a = wa[bit >> 5], b = wb[bit >> 5];
-        const int sh = bit & 31;
-        // put the 16-bit halves holding the field side by side, then mask into a bf16 magic of 128
-        const uint32_t z = (sh < 16) ? __byte_perm(a, b, 0x5410) : __byte_perm(a, b, 0x7632);
-        const uint32_t m = (VB == 2) ? 0x00030003u : 0x000F000Fu;
-        const uint32_t v = ((z >> (sh & 15)) & m) | 0x43004300u;
-        __nv_bfloat162 r = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&v), __floats2bfloat162_rn(128.f, 128.f));
-        return *reinterpret_cast<uint32_t*>(&r);
-    } else {
-        const int wi = bit >> 5, sh = bit & 31;
-        uint32_t qa = wa[wi] >> sh, qb = wb[wi] >> sh;
-        if (sh + VB > 32) {
-            qa |= wa[wi + 1] << (32 - sh);
-            qb |= wb[wi + 1] << (32 - sh);
-        }
-        qa &= (1u << VB) - 1u;
-        qb &= (1u << VB) - 1u;
-        return pack_bf16(static_cast<float>(qa), static_cast<float>(qb));
-    }
+    const uint32_t u0 = __float_as_uint(x0), u1 = __float_as_uint(x1);
+    hi = __byte_perm(u0, u1, 0x7632);
+    lo = pack_bf16(x0 - __uint_as_float(u0 & 0xFFFF0000u), x1 - __uint_as_float(u1 & 0xFFFF0000u));
 }
 
 // n fp16 values at p (n in {1, 2, 4, 8}, naturally aligned) as floats
@@ -186,22 +154,79 @@ __device__ __forceinline__ void load_halves(const __half* p, float (&o)[N]) {
     }
 }
 
+// The little-endian bitstream `w` shifted right by `bit` (which may be as low as -31), low 32 bits.
+template <int NW>
+__device__ __forceinline__ uint32_t window_shr(const uint32_t (&w)[NW], int bit) {
+    if (bit < 0) return w[0] << (-bit);
+    const int wi = bit >> 5, sh = bit & 31;
+    return sh ? __funnelshift_r(w[wi], w[wi + 1], sh) : w[wi];
+}
+
+// Value codes as bf16 operands without arithmetic.  A bf16 whose upper 8 bits are zero is exactly
+// (its bits) * 2^-133 (subnormals, then the first normal binade with the same spacing), and the tensor cores
+// take subnormal operands exactly; so masking the codes of two tokens out of `pr` (token a in bits 0..15,
+// token b in 16..31) gives a register {code_a, code_b} * 2^(VB pos') * 2^-133, where the scale 2^(VB pos')
+// depends only on the code's position and is divided out of the accumulator at the end.
+// The lane field holds four codes, positions 0..3, VB bits apart (VB = 2, 3, 4).
+template <int VB>
+__device__ __forceinline__ uint32_t vcode_sel(uint32_t pr, int pos) {
+    if constexpr (VB == 2) {
+        return pr & (0x00030003u << (2 * pos));
+    } else {
+        constexpr uint32_t m = (1u << VB) - 1u, mm = m | (m << 16);
+        return (pos < 2) ? (pr & (mm << (VB * pos))) : ((pr >> (2 * VB)) & (mm << (VB * (pos - 2))));
+    }
+}
+
+// log2 of the position scale above: the accumulator row holding code position `pos` carries 2^(that)
+template <int VB>
+__host__ __device__ constexpr int vcode_scale_log2(int pos) {
+    return (VB == 2) ? 2 * pos : ((VB == 8) ? 0 : VB * (pos & 1));
+}
+
+// The lane field of one token's value row for 32-column slice `sl`: the codes of columns
+// 32 sl + 4 gid + (0..3), positions 0..3 (VB = 8: the four bytes).
+template <int VB>
+__device__ __forceinline__ uint32_t vfield(const uint8_t* row, int sl, int gid) {
+    if constexpr (VB == 2) {
+        return row[8 * sl + gid];
+    } else if constexpr (VB == 4) {
+        return *reinterpret_cast<const uint16_t*>(row + 16 * sl + 2 * gid);
+    } else if constexpr (VB == 8) {
+        return *reinterpret_cast<const uint32_t*>(row + 32 * sl + 4 * gid);
+    } else {
+        const int bit = 32 * VB * sl + 4 * VB * gid;
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(row) + (bit >> 5);
+        return __funnelshift_r(w[0], w[1], bit & 31);
+    }
+}
+
+// Fused decode attention for one (split, kv head, sequence).  Per 16-token chunk and warp:
+//   scores  S[head][tok]  = (q hi/lo, fp16 A, rows gid / gid + 8) x (codebook pairs, fp16 B) on mma.sync
+//   values  O^T[col][head] += (value codes, bf16 A, exact) x (hi/lo of p * scale, bf16 B)
+// so each lane's probabilities (head gid, tokens 2tig, 2tig+1, 2tig+8, 2tig+9) are already the B fragment
+// of the value product, and the accumulator is D/16 x 4 registers.
 template <int D, int KB, int VB, int VG>
 __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB, VB, VG>::kMinBlocks)
     attend_kernel(const AttendParams p) {
     using C = AttCfg<D, KB, VB, VG>;
     constexpr int S = C::kStages;
     constexpr int KS = D / 16;                        // k-steps of the score contraction
-    constexpr int NT = D / 8;                         // n-tiles of the value contraction
+    constexpr int MT = D / 16;                        // m-tiles (16 value columns) of the value contraction
+    constexpr int NSL = D / 32;                       // 32-column slices (two m-tiles)
     constexpr int G8 = C::kVGroups;
+    // probabilities enter the value product as p * 2^kPExp so that p * scale * code * 2^-133 stays normal
+    constexpr int kPExp = 80;
     extern __shared__ __align__(16) uint8_t smem[];
     uint4* s_qf = reinterpret_cast<uint4*>(smem + C::kQfOff);
     float* s_qr = reinterpret_cast<float*>(smem + C::kQrOff);
-    uint32_t* s_pair = reinterpret_cast<uint32_t*>(smem + C::kPairOff);
     float* s_red = reinterpret_cast<float*>(smem + C::kRedOff);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     const uint32_t b_full = smem_u32(bars), b_empty = b_full + 8 * S;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S);
+    // the key table starts on a multiple of its size, so an entry's address is (entry << 7) | lane bits
+    const uint32_t lut_addr = (smem_u32(smem + C::kLutOff) + C::kLutBytes - 1) & ~static_cast<uint32_t>(C::kLutBytes - 1);
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + (lut_addr - smem_u32(smem)));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;
@@ -222,17 +247,7 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         *abort_flag = 0;
         fence_mbar_init();
     }
-    for (int i = threadIdx.x; i < (1 << (2 * KB)); i += blockDim.x) s_pair[i] = p.pair_lut[i];
-    __syncthreads();
-    if constexpr (C::kQuad) {
-        // quad table: key = 4 codes (4 KB bits, LSB first) -> {half2(c0, c1), half2(c2, c3)}
-        uint2* q4 = reinterpret_cast<uint2*>(smem + C::kLutOff);
-        for (int i = threadIdx.x; i < (1 << (4 * KB)); i += blockDim.x)
-            q4[i] = make_uint2(s_pair[i & ((1 << (2 * KB)) - 1)], s_pair[i >> (2 * KB)]);
-    } else {
-        uint32_t* q2 = reinterpret_cast<uint32_t*>(smem + C::kLutOff);
-        for (int i = threadIdx.x; i < (1 << (2 * KB)); i += blockDim.x) q2[i] = s_pair[i];
-    }
+    for (int i = threadIdx.x; i < C::kPairs * 32; i += blockDim.x) lut[i] = __ldg(p.pair_lut + (i >> 5));
     __syncthreads();
 
     if (warp == C::kWarps) {
@@ -277,7 +292,7 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         // ------------------------------------------------------------------ rotate the query
         // q_rot[g][n] = sum_k q[g][k] Pi_op[n][k] on the tensor cores (fp16 inputs are exact products)
         const __half* qg = p.q + (static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * G) * D;
-        for (int nt = warp; nt < NT; nt += C::kWarps) {
+        for (int nt = warp; nt < D / 8; nt += C::kWarps) {
             // every fragment of this n-tile is loaded before the first MMA, so the loads overlap
             uint32_t bf[KS][2], af[KS][2];
             const __half* prow = p.pi_op + (8 * nt + gid) * D + 2 * tig;
@@ -331,11 +346,16 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         named_bar_sync(1, 32 * C::kWarps);
 
         // ------------------------------------------------------------------ token loop
-        const uint2* lut4 = reinterpret_cast<const uint2*>(smem + C::kLutOff);
-        const uint32_t* lut2 = reinterpret_cast<const uint32_t*>(smem + C::kLutOff);
-        float o[NT][4];
+        uint4 qa[C::kQInRegs ? KS : 1];
+        if constexpr (C::kQInRegs) {
 #pragma unroll
-        for (int m = 0; m < NT; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
+            for (int ks = 0; ks < KS; ++ks) qa[ks] = s_qf[ks * 32 + lane];
+        }
+        const uint32_t lane_addr = lut_addr + 4u * lane;
+        constexpr uint32_t kFieldMask = static_cast<uint32_t>(C::kPairs - 1) << 7;
+        float o[MT][4];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
         float zacc[G8];
 #pragma unroll
         for (int g = 0; g < G8; ++g) zacc[g] = 0.f;
@@ -372,93 +392,96 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                 float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
                 for (int ks = 0; ks < KS; ++ks) {
-                    const uint4 a = s_qf[ks * 32 + lane];
+                    uint4 a;
+                    if constexpr (C::kQInRegs) a = qa[ks]; else a = s_qf[ks * 32 + lane];
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
-                        if constexpr (C::kQuad) {
-                            const uint2 bb = lut4[get_bits<4 * KB>(w[nt], 4 * ks * KB)];
-                            mma_f16(sc[nt], a, bb.x, bb.y);
-                        } else {
-                            const uint32_t k0 = get_bits<2 * KB>(w[nt], 4 * ks * KB);
-                            const uint32_t k1 = get_bits<2 * KB>(w[nt], 4 * ks * KB + 2 * KB);
-                            mma_f16(sc[nt], a, lut2[k0], lut2[k1]);
-                        }
+                        // code pairs (4ks, 4ks+1) and (4ks+2, 4ks+3) of the lane's quarter
+                        const uint32_t e0 = window_shr(w[nt], 4 * ks * KB - 7) & kFieldMask;
+                        const uint32_t e1 = window_shr(w[nt], (4 * ks + 2) * KB - 7) & kFieldMask;
+                        mma_f16(sc[nt], a, lds_u32(lane_addr | e0), lds_u32(lane_addr | e1));
                     }
                 }
                 // ---- logits (log2 domain) of head gid for tokens 2tig, 2tig+1, 8+2tig, 9+2tig
                 const float* nrm = reinterpret_cast<const float*>(st + C::kNOff) + warp * 16;
+                const int64_t valid = T - chunk * 16;
                 float lg[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int nt = e >> 1, k = e & 1;
                     const float raw = (sc[nt][k] + sc[nt][k + 2]) * unpre * nrm[tok[e]];
-                    lg[e] = (chunk * 16 + tok[e] < T) ? raw : -INFINITY;
+                    lg[e] = (tok[e] < valid) ? raw : -INFINITY;
                 }
                 float mt = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
                 mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
                 mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
                 const float m_new = fmaxf(m_run, mt);
                 const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-                const float corr = exp2f(m_run - m_use);
+                // probabilities carry the factor 2^kPExp (so do l_run and zacc; removed at the end)
+                const float m_off = m_use - static_cast<float>(kPExp);
                 float pr[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) pr[e] = exp2f(lg[e] - m_use);
-                l_run = l_run * corr + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
-                m_run = m_new;
-                if (__any_sync(0xffffffffu, corr != 1.0f)) {     // some head's running max moved
+                for (int e = 0; e < 4; ++e) pr[e] = ex2(lg[e] - m_off);
+                if (__any_sync(0xffffffffu, m_new != m_run)) {     // some head's running max moved
+                    const float corr = ex2(m_run - m_use);
+                    // the accumulator columns are heads 2tig and 2tig+1: their factors sit in lanes 8tig, 8tig+4
+                    const float ca = __shfl_sync(0xffffffffu, corr, 8 * tig);
+                    const float cb = __shfl_sync(0xffffffffu, corr, 8 * tig + 4);
 #pragma unroll
-                    for (int m = 0; m < NT; ++m) {
-                        o[m][0] *= corr; o[m][1] *= corr; o[m][2] *= corr; o[m][3] *= corr;
+                    for (int m = 0; m < MT; ++m) {
+                        o[m][0] *= ca; o[m][1] *= cb; o[m][2] *= ca; o[m][3] *= cb;
                     }
 #pragma unroll
-                    for (int g8 = 0; g8 < G8; ++g8) zacc[g8] *= corr;
+                    for (int g = 0; g < G8; ++g) zacc[g] *= corr;
+                    l_run *= corr;
                 }
-                // ---- zero term on FMAs
+                l_run += (pr[0] + pr[1]) + (pr[2] + pr[3]);
+                m_run = m_new;
+                // ---- zero term on FMAs: zacc[g] += p * z
                 const __half* zch = reinterpret_cast<const __half*>(st + C::kZOff) + warp * 16 * G8;
+                const __half* sch = reinterpret_cast<const __half*>(st + C::kSOff) + warp * 16 * G8;
+                const uint8_t* vch = st + C::kVOff + warp * 16 * C::kVRow;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     float zr[G8];
                     load_halves<G8>(zch + tok[e] * G8, zr);
 #pragma unroll
-                    for (int g8 = 0; g8 < G8; ++g8) zacc[g8] = fmaf(pr[e], zr[g8], zacc[g8]);
+                    for (int g = 0; g < G8; ++g) zacc[g] = fmaf(pr[e], zr[g], zacc[g]);
                 }
-                // ---- values: A = hi/lo of p * scale (per scale group), B = integer codes, per 32-column slice
-                const __half* sch = reinterpret_cast<const __half*>(st + C::kSOff) + warp * 16 * G8;
-                float sc4[4][G8];
+                // ---- values: A = codes (exact bf16), B = hi/lo of p * scale; per 32-column slice
+                uint32_t bh0 = 0, bh1 = 0, bl0 = 0, bl1 = 0;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) load_halves<G8>(sch + tok[e] * G8, sc4[e]);
-                const uint8_t* vch = st + C::kVOff + warp * 16 * C::kVRow;
-                const uint8_t* vrow0 = vch + tok[0] * C::kVRow;
-                const uint8_t* vrow1 = vch + tok[1] * C::kVRow;
-                const uint8_t* vrow2 = vch + tok[2] * C::kVRow;
-                const uint8_t* vrow3 = vch + tok[3] * C::kVRow;
-                uint4 a;
+                for (int sl = 0; sl < NSL; ++sl) {
+                    const int g = (32 * sl) / VG;
+                    if (sl == 0 || (32 * sl) % VG == 0) {
+                        float x[4];
 #pragma unroll
-                for (int sl = 0; sl < D / 32; ++sl) {
-                    const int g8 = (sl * 32) / VG;
-                    if (sl == 0 || (sl * 32) % VG == 0) {
-                        split_bf16(pr[0] * sc4[0][g8], pr[1] * sc4[1][g8], a.x, a.y);
-                        split_bf16(pr[2] * sc4[2][g8], pr[3] * sc4[3][g8], a.z, a.w);
+                        for (int e = 0; e < 4; ++e) x[e] = pr[e] * __half2float(sch[tok[e] * G8 + g]);
+                        split_bf16(x[0], x[1], bh0, bl0);
+                        split_bf16(x[2], x[3], bh1, bl1);
                     }
-                    if constexpr (VB == 8) {
-                        // 8-bit codes: one byte per column, read per n-tile to keep registers low
+                    uint32_t f[4];
 #pragma unroll
-                        for (int mm = 0; mm < 4; ++mm) {
-                            const int c = sl * 32 + 8 * mm + gid;
-                            mma_bf16(o[4 * sl + mm], a, pack_bf16(static_cast<float>(vrow0[c]), static_cast<float>(vrow1[c])),
-                                     pack_bf16(static_cast<float>(vrow2[c]), static_cast<float>(vrow3[c])));
-                        }
-                    } else {
-                        uint32_t w0[VB], w1[VB], w2[VB], w3[VB];
-                        load_vslice<VB>(vrow0, sl, w0);
-                        load_vslice<VB>(vrow1, sl, w1);
-                        load_vslice<VB>(vrow2, sl, w2);
-                        load_vslice<VB>(vrow3, sl, w3);
+                    for (int e = 0; e < 4; ++e) f[e] = vfield<VB>(vch + tok[e] * C::kVRow, sl, gid);
 #pragma unroll
-                        for (int mm = 0; mm < 4; ++mm) {
-                            const int c = 8 * mm + gid;
-                            mma_bf16(o[4 * sl + mm], a, vcode_pair<VB>(w0, w1, c), vcode_pair<VB>(w2, w3, c));
+                    for (int hm = 0; hm < 2; ++hm) {
+                        uint4 a;
+                        if constexpr (VB == 8) {
+                            // bytes pos of both tokens into the low bytes of the 16-bit halves, pos = 2 hm (+1)
+                            const uint32_t s0 = 0x4400u + 0x1111u * (2 * hm), s1 = s0 + 0x1111u;
+                            a.x = __byte_perm(f[0], f[1], s0) & 0x00FF00FFu;
+                            a.y = __byte_perm(f[0], f[1], s1) & 0x00FF00FFu;
+                            a.z = __byte_perm(f[2], f[3], s0) & 0x00FF00FFu;
+                            a.w = __byte_perm(f[2], f[3], s1) & 0x00FF00FFu;
+                        } else {
+                            const uint32_t p01 = __byte_perm(f[0], f[1], 0x5410), p23 = __byte_perm(f[2], f[3], 0x5410);
+                            a.x = vcode_sel<VB>(p01, 2 * hm);
+                            a.y = vcode_sel<VB>(p01, 2 * hm + 1);
+                            a.z = vcode_sel<VB>(p23, 2 * hm);
+                            a.w = vcode_sel<VB>(p23, 2 * hm + 1);
                         }
+                        mma_bf16(o[2 * sl + hm], a, bh0, bh1);
+                        mma_bf16(o[2 * sl + hm], a, bl0, bl1);
                     }
                 }
             }
@@ -470,9 +493,15 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
         l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
 #pragma unroll
-        for (int g8 = 0; g8 < G8; ++g8) {
-            zacc[g8] += __shfl_xor_sync(0xffffffffu, zacc[g8], 1);
-            zacc[g8] += __shfl_xor_sync(0xffffffffu, zacc[g8], 2);
+        for (int g = 0; g < G8; ++g) {
+            zacc[g] += __shfl_xor_sync(0xffffffffu, zacc[g], 1);
+            zacc[g] += __shfl_xor_sync(0xffffffffu, zacc[g], 2);
+        }
+        constexpr float kUnP = 1.0f / static_cast<float>(1ull << 40) / static_cast<float>(1ull << 40);  // 2^-kPExp
+        float* zs = reinterpret_cast<float*>(smem + C::kZsOff) + warp * 8 * G8;
+        if (tig == 0) {
+#pragma unroll
+            for (int g = 0; g < G8; ++g) zs[gid * G8 + g] = zacc[g] * kUnP;
         }
         // the stage ring is free once every consumer is past its last stage
         named_bar_sync(1, 32 * C::kWarps);
@@ -480,14 +509,21 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         float* mine = comb + warp * C::kPartFloats;
         if (tig == 0) {
             mine[gid] = m_run;
-            mine[8 + gid] = l_run;
+            mine[8 + gid] = l_run * kUnP;
         }
 #pragma unroll
-        for (int m = 0; m < NT; ++m) {
-            const int col = 8 * m + 2 * tig;
-            const float z = zacc[(8 * m) / VG];
-            mine[16 + gid * D + col] = o[m][0] + o[m][2] + z;
-            mine[16 + gid * D + col + 1] = o[m][1] + o[m][3] + z;
+        for (int m = 0; m < MT; ++m) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                // row r = gid + 8 (e / 2) of m-tile m is value column 32 (m / 2) + 4 gid + pos, code position
+                // pos = 2 (m % 2) + e / 2; column n = 2 tig + e % 2 is the head
+                const int pos = 2 * (m & 1) + (e >> 1);
+                const int col = 32 * (m >> 1) + 4 * gid + pos;
+                const int hd = 2 * tig + (e & 1);
+                // codes entered as code * 2^(scale + -133), probabilities as p * 2^kPExp
+                const float unit = __int_as_float((127 + 133 - kPExp - vcode_scale_log2<VB>(pos)) << 23);
+                mine[16 + hd * D + col] = o[m][e] * unit + zs[hd * G8 + col / VG];
+            }
         }
         named_bar_sync(1, 32 * C::kWarps);
         // ------------------------------------------------------------------ merge the four warps
