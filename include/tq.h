@@ -200,15 +200,17 @@ typedef struct tq_attend_args {
     const void* v_scales;      /* device binary16 pool [rows][head_dim / v_group] */
     const void* v_zeros;       /* device binary16 pool [rows][head_dim / v_group] */
     float* out;                /* device float [batch][num_q_heads][head_dim] */
-    void* workspace;           /* device scratch for split-K partials (16-byte aligned) of at least the size
-                                  tq_attend_workspace_bytes reports; may be NULL when that size is 0.  Its
-                                  contents need no initialisation and are overwritten by every call. */
+    void* workspace;           /* device scratch (16-byte aligned) of at least the size
+                                  tq_attend_workspace_bytes reports: the prepared query fragments of each
+                                  (sequence, kv head), then the split-K partials.  Its contents need no
+                                  initialisation and are overwritten by every call. */
     size_t workspace_bytes;
 } tq_attend_args;
 
 /*
  * tq_attend_workspace_bytes -- bytes of workspace tq_attend_decode needs for these arguments on the current
- * device (0 when the launch needs no split-K partials).  Only the shape fields of args are read.
+ * device: (head_dim / 16 * 32 + 1) * 16 bytes per (sequence, kv head) for the prepared query, plus the split-K
+ * partials when the sequence axis is split.  Only the shape fields of args are read.
  * Errors: the same argument checks as tq_attend_decode (TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED).
  */
 tq_status tq_attend_workspace_bytes(const tq_attend_args* args, size_t* bytes);
@@ -219,10 +221,11 @@ tq_status tq_attend_workspace_bytes(const tq_attend_args* args, size_t* bytes);
  * rotated once).  For each (b, hq) with h = hq / G:
  *   q_rot = Pi_op q;  s_t = scale * n_t * <q_rot, c_op[idx_t]>;  p = softmax(s);
  *   out = sum_t p_t * (q_t * scale16_t + zero16_t)   (the value dequantized inside the kernel).
- * No fp16 key or value is written to memory.  A sequence of length 0 yields zeros.  When the sequence axis
- * is split over several CTAs, a second kernel (a programmatic dependent launch on the same stream) merges
- * the per-split partials with a log-sum-exp rescale.  Calls that overlap on the GPU must use distinct
- * workspaces.
+ * No fp16 key or value is written to memory.  A sequence of length 0 yields zeros.  A small first kernel
+ * rotates and splits the query once per (sequence, kv head); the attention kernel is its programmatic
+ * dependent on the same stream.  When the sequence axis is split over several CTAs, a third kernel (again a
+ * programmatic dependent) merges the per-split partials with a log-sum-exp rescale.  Calls that overlap on
+ * the GPU must use distinct workspaces.
  */
 tq_status tq_attend_decode(const tq_codec* codec, const tq_attend_args* args, void* stream);
 
@@ -245,10 +248,10 @@ tq_status tq_attend_decode(const tq_codec* codec, const tq_attend_args* args, vo
  *   - Set-up: the first call on each device looks up the scratch array's device address with
  *     cudaGetSymbolAddress (with that device current) and caches it; make that first call outside any
  *     stream capture.
- *   - Limit: a launch whose split-K partials need more than TQ_ATTEND_SCRATCH_BYTES (see
- *     tq_attend_workspace_bytes) is rejected with TQ_ERR_INVALID_ARG and a message giving both sizes;
+ *   - Limit: a launch whose workspace (query fragments and split-K partials) needs more than
+ *     TQ_ATTEND_SCRATCH_BYTES (see tq_attend_workspace_bytes) is rejected with TQ_ERR_INVALID_ARG and a message giving both sizes;
  *     use tq_attend_decode with a caller workspace for such shapes.
- *   - Sharing: all calls on a device share the one array and it keeps the last call's partials; nothing
+ *   - Sharing: all calls on a device share the one array and it keeps the last call's contents; nothing
  *     in it needs to start at zero, since every launch overwrites the part it reads.  Calls that can
  *     overlap on the GPU (different streams without ordering, or different threads) race on it and must
  *     be serialised by the caller.

@@ -37,8 +37,13 @@ struct AttendParams {
     const __half* v_zeros;
     float* out;
     float* partials;                                 // [B][H_kv][splits][16 + 8 d]
+    uint4* qfrag;                                    // [B][H_kv][d/16 * 32 + 1]: score A fragments, 1 / prescale
     int num_splits;
 };
+
+// uint4 slots per (sequence, kv head) of the query-fragment array
+template <int D>
+__host__ __device__ constexpr int qfrag_slots() { return (D / 16) * 32 + 1; }
 
 template <int D, int KB, int VB, int VG>
 struct AttCfg {
@@ -67,17 +72,15 @@ struct AttCfg {
     // copy per shared-memory bank (entry e of lane l at byte 128 e + 4 l), so lookups never conflict
     static constexpr int kPairs = 1 << (2 * KB);
     static constexpr int kLutBytes = kPairs * 128;
-    // shared memory: stages | q fragments | rotated q | key table (aligned to its size at run time) |
-    // per-warp zero sums | reduction | barriers
+    // shared memory: stages | q fragments (d = 256) | key table (aligned to its size at run time) |
+    // per-warp zero sums | barriers
     static constexpr int kCombineFloats = kWarps * kPartFloats;
     static constexpr int kRingBytes =
         (kStages * kStageBytes > kCombineFloats * 4) ? kStages * kStageBytes : kCombineFloats * 4;
     static constexpr int kQfOff = kRingBytes;
-    static constexpr int kQrOff = kQfOff + (D / 16) * 32 * 16;
-    static constexpr int kLutOff = kQrOff + 8 * D * 4;
+    static constexpr int kLutOff = kQfOff + (kQInRegs ? 0 : (D / 16) * 32 * 16);
     static constexpr int kZsOff = kLutOff + 2 * kLutBytes;
-    static constexpr int kRedOff = kZsOff + kWarps * 8 * kVGroups * 4;
-    static constexpr int kBarOff = (kRedOff + 8 * 4 + 15) & ~15;
+    static constexpr int kBarOff = (kZsOff + kWarps * 8 * kVGroups * 4 + 15) & ~15;
     static constexpr int kSmem = kBarOff + 8 * (2 * kStages) + 16;
     static_assert(kNOff % 16 == 0 && kVOff % 16 == 0 && kSOff % 16 == 0 && kZOff % 16 == 0 && kStageBytes % 16 == 0,
                   "bulk copies need 16-byte multiples");
@@ -201,6 +204,82 @@ __device__ __forceinline__ uint32_t vfield(const uint8_t* row, int sl, int gid) 
     }
 }
 
+// Query preparation for one (kv head, sequence): the rotated query q_rot[g] = Pi_op q[g] of each of the
+// group's heads, scaled by softmax scale * log2(e) and a power-of-two prescale, split into fp16 hi/lo halves and
+// laid out as the score A fragments (rows gid = hi, gid + 8 = lo); slot d/16 * 32 holds 1 / prescale.
+// Done once per (kv head, sequence) instead of once per split; the attention grid is its programmatic dependent.
+constexpr int kPrepThreads = 512;
+
+template <int D>
+__global__ void __launch_bounds__(kPrepThreads) attend_prep_kernel(const AttendParams p) {
+    constexpr int KS = D / 16;
+    constexpr int kWarps = kPrepThreads / 32;            // one n-tile of q_rot per warp (two at d = 256)
+    __shared__ float s_qr[8 * D];
+    __shared__ float s_red[kWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int G = p.group;
+    uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();
+    // q_rot[g][n] = sum_k q[g][k] Pi_op[n][k] on the tensor cores (fp16 inputs are exact products)
+    const __half* qg = p.q + (static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * G) * D;
+    for (int nt = warp; nt < D / 8; nt += kWarps) {
+        // every fragment of this n-tile is loaded before the first MMA, so the loads overlap
+        uint32_t bf[KS][2], af[KS][2];
+        const __half* prow = p.pi_op + (8 * nt + gid) * D + 2 * tig;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            bf[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(prow + 16 * ks));
+            bf[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(prow + 16 * ks + 8));
+            af[ks][0] = (gid < G) ? __ldg(reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig)) : 0u;
+            af[ks][1] = (gid < G) ? __ldg(reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig + 8)) : 0u;
+        }
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) mma_f16(c, make_uint4(af[ks][0], 0u, af[ks][1], 0u), bf[ks][0], bf[ks][1]);
+        s_qr[gid * D + 8 * nt + 2 * tig] = c[0];
+        s_qr[gid * D + 8 * nt + 2 * tig + 1] = c[1];
+    }
+    __syncthreads();
+    // power-of-two prescale so the fp16 hi/lo halves of the scaled query stay in the normal range
+    float amax = 0.f;
+    for (int i = threadIdx.x; i < G * D; i += 32 * kWarps) amax = fmaxf(amax, fabsf(s_qr[i] * p.scale_log2));
+#pragma unroll
+    for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) s_red[warp] = amax;
+    __syncthreads();
+    amax = s_red[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) amax = fmaxf(amax, s_red[w]);
+    int ex = 0;
+    if (amax > 0.f) frexpf(amax, &ex);
+    const float pre = (amax > 0.f) ? ldexpf(1.0f, 14 - ex) : 1.0f;     // max |q| * pre in [8192, 16384)
+    // score A fragments, coordinate-permuted so lane tig owns coords [tig*D/4, (tig+1)*D/4):
+    // k-slots (2tig, 2tig+1, 2tig+8, 2tig+9) of k-step ks <- coords tig*D/4 + 4ks + (0, 1, 2, 3)
+    for (int i = threadIdx.x; i < KS * 32; i += 32 * kWarps) {
+        const int ks = i >> 5, ln = i & 31, g = ln >> 2, tg = ln & 3;
+        const int cc = tg * (D / 4) + 4 * ks;
+        uint4 f = make_uint4(0u, 0u, 0u, 0u);
+        if (g < G) {
+            float x[4], hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x[e] = s_qr[g * D + cc + e] * p.scale_log2 * pre;
+                hi[e] = __half2float(__float2half_rn(x[e]));
+                lo[e] = x[e] - hi[e];
+            }
+            f.x = pack_f16(hi[0], hi[1]);
+            f.y = pack_f16(lo[0], lo[1]);
+            f.z = pack_f16(hi[2], hi[3]);
+            f.w = pack_f16(lo[2], lo[3]);
+        }
+        qf[i] = f;
+    }
+    if (threadIdx.x == 0) qf[KS * 32] = make_uint4(__float_as_uint(1.0f / pre), 0u, 0u, 0u);
+    // the attention grid may start streaming the cache; its consumers wait for this grid's completion
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Fused decode attention for one (split, kv head, sequence).  Per 16-token chunk and warp:
 //   scores  S[head][tok]  = (q hi/lo, fp16 A, rows gid / gid + 8) x (codebook pairs, fp16 B) on mma.sync
 //   values  O^T[col][head] += (value codes, bf16 A, exact) x (hi/lo of p * scale, bf16 B)
@@ -219,8 +298,6 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
     constexpr int kPExp = 80;
     extern __shared__ __align__(16) uint8_t smem[];
     uint4* s_qf = reinterpret_cast<uint4*>(smem + C::kQfOff);
-    float* s_qr = reinterpret_cast<float*>(smem + C::kQrOff);
-    float* s_red = reinterpret_cast<float*>(smem + C::kRedOff);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     const uint32_t b_full = smem_u32(bars), b_empty = b_full + 8 * S;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S);
@@ -289,67 +366,21 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                 mbar_wait_drain(b_full + 8 * static_cast<int>(ti % S), static_cast<uint32_t>((ti / S) & 1));
         }
     } else {
-        // ------------------------------------------------------------------ rotate the query
-        // q_rot[g][n] = sum_k q[g][k] Pi_op[n][k] on the tensor cores (fp16 inputs are exact products)
-        const __half* qg = p.q + (static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * G) * D;
-        for (int nt = warp; nt < D / 8; nt += C::kWarps) {
-            // every fragment of this n-tile is loaded before the first MMA, so the loads overlap
-            uint32_t bf[KS][2], af[KS][2];
-            const __half* prow = p.pi_op + (8 * nt + gid) * D + 2 * tig;
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                bf[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(prow + 16 * ks));
-                bf[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(prow + 16 * ks + 8));
-                af[ks][0] = (gid < G) ? __ldg(reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig)) : 0u;
-                af[ks][1] = (gid < G) ? __ldg(reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig + 8)) : 0u;
-            }
-            float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) mma_f16(c, make_uint4(af[ks][0], 0u, af[ks][1], 0u), bf[ks][0], bf[ks][1]);
-            s_qr[gid * D + 8 * nt + 2 * tig] = c[0];
-            s_qr[gid * D + 8 * nt + 2 * tig + 1] = c[1];
+        // ------------------------------------------------------------------ query fragments
+        // written by attend_prep_kernel, the grid this one depends on programmatically
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        const uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();
+        const float unpre = __uint_as_float(__ldcg(&qf[KS * 32].x));
+        if constexpr (!C::kQInRegs) {
+            for (int i = threadIdx.x; i < KS * 32; i += 32 * C::kWarps) s_qf[i] = __ldcg(qf + i);
+            named_bar_sync(1, 32 * C::kWarps);
         }
-        named_bar_sync(1, 32 * C::kWarps);
-        // power-of-two prescale so the fp16 hi/lo halves of the scaled query stay in the normal range
-        float amax = 0.f;
-        for (int i = threadIdx.x; i < G * D; i += 32 * C::kWarps) amax = fmaxf(amax, fabsf(s_qr[i] * p.scale_log2));
-#pragma unroll
-        for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        if (lane == 0) s_red[warp] = amax;
-        named_bar_sync(1, 32 * C::kWarps);
-        amax = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
-        int ex = 0;
-        if (amax > 0.f) frexpf(amax, &ex);
-        const float pre = (amax > 0.f) ? ldexpf(1.0f, 14 - ex) : 1.0f;     // max |q| * pre in [8192, 16384)
-        const float unpre = 1.0f / pre;
-        // score A fragments, coordinate-permuted so lane tig owns coords [tig*D/4, (tig+1)*D/4):
-        // k-slots (2tig, 2tig+1, 2tig+8, 2tig+9) of k-step ks <- coords tig*D/4 + 4ks + (0, 1, 2, 3)
-        for (int i = threadIdx.x; i < KS * 32; i += 32 * C::kWarps) {
-            const int ks = i >> 5, ln = i & 31, g = ln >> 2, tg = ln & 3;
-            const int cc = tg * (D / 4) + 4 * ks;
-            uint4 f = make_uint4(0u, 0u, 0u, 0u);
-            if (g < G) {
-                float x[4], hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    x[e] = s_qr[g * D + cc + e] * p.scale_log2 * pre;
-                    hi[e] = __half2float(__float2half_rn(x[e]));
-                    lo[e] = x[e] - hi[e];
-                }
-                f.x = pack_f16(hi[0], hi[1]);
-                f.y = pack_f16(lo[0], lo[1]);
-                f.z = pack_f16(hi[2], hi[3]);
-                f.w = pack_f16(lo[2], lo[3]);
-            }
-            s_qf[i] = f;
-        }
-        named_bar_sync(1, 32 * C::kWarps);
 
         // ------------------------------------------------------------------ token loop
         uint4 qa[C::kQInRegs ? KS : 1];
         if constexpr (C::kQInRegs) {
 #pragma unroll
-            for (int ks = 0; ks < KS; ++ks) qa[ks] = s_qf[ks * 32 + lane];
+            for (int ks = 0; ks < KS; ++ks) qa[ks] = __ldcg(qf + ks * 32 + lane);
         }
         const uint32_t lane_addr = lut_addr + 4u * lane;
         constexpr uint32_t kFieldMask = static_cast<uint32_t>(C::kPairs - 1) << 7;
@@ -560,8 +591,9 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
 }
 
 // Split-K merge: out[b][h*G+g][:] = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M), M = max_s m_s.
-// One CTA per (g, h, b); pass 1 gives every split's weight, pass 2 spreads the splits over
-// kMergeThreads / D slices so the partial loads are issued in parallel.
+// One CTA per (g, h, b).  Slice k of the CTA's threads (D threads, one per column) folds splits k, k + kSlices,
+// ... with every load issued before the first is used, so the partials cost one round trip; the slices are
+// then combined in shared memory the same way.
 constexpr int kMergeThreads = 512;
 constexpr int kMaxSplits = 256;
 
@@ -570,48 +602,59 @@ __global__ void __launch_bounds__(kMergeThreads) attend_merge_kernel(const Atten
     asm volatile("griddepcontrol.wait;" ::: "memory");
     constexpr int kPart = 16 + 8 * D;
     constexpr int kSlices = kMergeThreads / D;
-    __shared__ float s_f[kMaxSplits];
-    __shared__ float s_red[kMergeThreads / 32];
-    __shared__ float s_part[kSlices][D];
+    constexpr int kBatch = 16;                           // splits per slice per round of loads
+    __shared__ float s_o[kSlices][D];
+    __shared__ float s_ml[kSlices][2];
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    const int col = tid % D, slice = tid / D;
     const int S = p.num_splits;
     const float* base = p.partials + (static_cast<int64_t>(b) * p.num_kv_heads + h) * S * kPart;
-    const float m = (tid < S) ? __ldcg(base + static_cast<int64_t>(tid) * kPart + g) : -INFINITY;
-    float M = m;
+    float M = -INFINITY, L = 0.f, O = 0.f;
+    for (int s0 = slice; s0 < S; s0 += kSlices * kBatch) {
+        float mv[kBatch], lv[kBatch], ov[kBatch];
 #pragma unroll
-    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if ((tid & 31) == 0) s_red[tid >> 5] = M;
-    __syncthreads();
-    M = s_red[0];
+        for (int k = 0; k < kBatch; ++k) {
+            const int sp = s0 + k * kSlices;
+            const float* ps = base + static_cast<int64_t>(sp < S ? sp : 0) * kPart;
+            mv[k] = (sp < S) ? __ldcg(ps + g) : -INFINITY;
+            lv[k] = __ldcg(ps + 8 + g);
+            ov[k] = __ldcg(ps + 16 + g * D + col);
+        }
+        float Mn = M;
 #pragma unroll
-    for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, s_red[w]);
-    const float Mu = (M == -INFINITY) ? 0.f : M;
-    float lw = 0.f;
-    if (tid < S) {
-        const float f = exp2f(m - Mu);
-        s_f[tid] = f;
-        lw = __ldcg(base + static_cast<int64_t>(tid) * kPart + 8 + g) * f;
+        for (int k = 0; k < kBatch; ++k) Mn = fmaxf(Mn, mv[k]);
+        const float Mu = (Mn == -INFINITY) ? 0.f : Mn;
+        const float c = exp2f(M - Mu);
+        L *= c;
+        O *= c;
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            const float f = exp2f(mv[k] - Mu);                // 0 for the padding entries
+            L = fmaf(lv[k], f, L);
+            O = fmaf(ov[k], f, O);
+        }
+        M = Mn;
     }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
-    __syncthreads();
-    if ((tid & 31) == 0) s_red[tid >> 5] = lw;
-    __syncthreads();
-    float L = 0.f;
-#pragma unroll
-    for (int w = 0; w < kMergeThreads / 32; ++w) L += s_red[w];
-    const int col = tid % D, slice = tid / D;
-    float acc = 0.f;
-#pragma unroll 8
-    for (int sp = slice; sp < S; sp += kSlices)
-        acc += __ldcg(base + static_cast<int64_t>(sp) * kPart + 16 + g * D + col) * s_f[sp];
-    s_part[slice][col] = acc;
+    s_o[slice][col] = O;
+    if (col == 0) {
+        s_ml[slice][0] = M;
+        s_ml[slice][1] = L;
+    }
     __syncthreads();
     if (slice == 0) {
+        float Mt = s_ml[0][0];
 #pragma unroll
-        for (int k = 1; k < kSlices; ++k) acc += s_part[k][col];
+        for (int k = 1; k < kSlices; ++k) Mt = fmaxf(Mt, s_ml[k][0]);
+        const float Mu = (Mt == -INFINITY) ? 0.f : Mt;
+        float Lt = 0.f, Ot = 0.f;
+#pragma unroll
+        for (int k = 0; k < kSlices; ++k) {
+            const float f = exp2f(s_ml[k][0] - Mu);
+            Lt = fmaf(s_ml[k][1], f, Lt);
+            Ot = fmaf(s_o[k][col], f, Ot);
+        }
         p.out[(static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * p.group + g) * D + col] =
-            (L > 0.f) ? acc / L : 0.f;
+            (Lt > 0.f) ? Ot / Lt : 0.f;
     }
 }
 

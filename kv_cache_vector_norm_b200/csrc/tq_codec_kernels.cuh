@@ -7,10 +7,8 @@ namespace tq {
 namespace dev {
 
 // ------------------------------------------------------------------------------------ value codec
-// "KV Cache API", values.py quantize_values / dequantize_values.  One lane owns 8 consecutive elements of
-// a row (16 bytes of fp16), so every warp-wide load and store is contiguous; the lanes of one scale group
-// (4 for group 32, d/8 for the per-token layout) reduce min/max with shuffles.  Every arithmetic step is
-// the page's fp32 operation with one rounding.
+// "KV Cache API", values.py quantize_values / dequantize_values.  The lanes of one scale group reduce
+// min/max with shuffles.  Every arithmetic step is the page's fp32 operation with one rounding.
 
 // Codes of a group: round_half_even(a / s) with the page's IEEE fp32 division, 0 <= a <= (2^b - 1) s.
 // With r = RN(1/s), the products a RN(r (1 -+ 2^-21)) bracket RN(a / s) (each end is off by at most
@@ -20,32 +18,42 @@ namespace dev {
 constexpr float kCodeMagic = 12582912.0f;                   // 1.5 * 2^23
 constexpr uint32_t kCodeMagicBits = 0x4B400000u;
 
+// One lane owns 16 consecutive elements of a row (32 bytes of fp16), so a group of 32 spans 2 lanes (or d/16
+// lanes in the per-token layout), the per-group division and reciprocal of the encoder are shared by 16
+// elements, and every warp-wide load and store covers whole rows.
 template <int D, int GROUP>
 struct VLanes {
-    static constexpr int kRowLanes = D / 8;                       // lanes per row (8 elements each)
-    static constexpr int kRowsPerWarp = 32 / kRowLanes;           // 1, 2 or 4
-    static constexpr int kGroupLanes = GROUP / 8;                 // lanes per scale group (4 or D/8)
-};
-
-// Encode: one lane owns 16 consecutive elements (two 16-byte loads), so a group of 32 spans 2 lanes
-// (or d/16 lanes in the per-token layout) and the per-group division and reciprocal are shared by 16
-// elements.
-template <int D, int GROUP>
-struct VEncLanes {
     static constexpr int kRowLanes = D / 16;
     static constexpr int kRowsPerWarp = 32 / kRowLanes;           // 2, 4 or 8
     static constexpr int kGroupLanes = GROUP / 16;                // 2 or d/16
 };
 
+// f32(h) - c with one rounding (h exact in f32, so this is the page's fp32 subtraction of the fp16 input)
+__device__ __forceinline__ float sub_f16_f32(__half h, float c) {
+    float d;
+    asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(__half_as_ushort(h)), "f"(c));
+    return d;
+}
+
+// sum_k kMagicBits * 2^(BITS k) over the codes packed into one 32-bit word (mod 2^32): packing the raw bits
+// of the rounded values (kCodeMagicBits + code) with multiply-adds leaves exactly this constant on top
+template <int BITS>
+__host__ __device__ constexpr uint32_t magic_pack_offset() {
+    uint32_t c = 0u;
+    for (int k = 0; k < 32 / BITS; ++k) c += kCodeMagicBits << (BITS * k);
+    return c;
+}
+
 template <int D, int BITS, int GROUP>
 __global__ void __launch_bounds__(256) encode_v_kernel(const __half* __restrict__ x, int64_t n, int64_t stride,
                                                        const int64_t* __restrict__ slots, uint8_t* __restrict__ data,
                                                        __half* __restrict__ scales, __half* __restrict__ zeros) {
-    using L = VEncLanes<D, GROUP>;
+    using L = VLanes<D, GROUP>;
     constexpr int kRowBytes = D * BITS / 8;
     constexpr int kGroups = D / GROUP;
     constexpr uint32_t kLevels = (1u << BITS) - 1u;
     constexpr int kW = (16 * BITS + 31) / 32;                     // words holding this lane's 16 codes
+    constexpr bool kWordAligned = (32 % BITS == 0);               // codes never straddle a word (2, 4, 8 bits)
     const int lane = threadIdx.x & 31;
     const int j = lane % L::kRowLanes;                            // 16-element chunk index within the row
     const int gl = j % L::kGroupLanes;                            // lane index within the scale group
@@ -54,30 +62,26 @@ __global__ void __launch_bounds__(256) encode_v_kernel(const __half* __restrict_
          wrow < n; wrow += warps_total * L::kRowsPerWarp) {
         const int64_t row = wrow + lane / L::kRowLanes;
         const bool valid = row < n;
-        float v[16];
+        __half2 hv[8];
         if (valid) {
             const uint4* src = reinterpret_cast<const uint4*>(x + row * stride) + 2 * j;
             const uint4 w0 = __ldg(src), w1 = __ldg(src + 1);
-            const __half2* h0 = reinterpret_cast<const __half2*>(&w0);
-            const __half2* h1 = reinterpret_cast<const __half2*>(&w1);
+            const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 f0 = __half22float2(h0[k]), f1 = __half22float2(h1[k]);
-                v[2 * k] = f0.x;
-                v[2 * k + 1] = f0.y;
-                v[8 + 2 * k] = f1.x;
-                v[8 + 2 * k + 1] = f1.y;
-            }
+            for (int k = 0; k < 8; ++k) hv[k] = *reinterpret_cast<const __half2*>(&u[k]);
         } else {
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = 0.f;
+            for (int k = 0; k < 8; ++k) hv[k] = __floats2half2_rn(0.f, 0.f);
         }
-        float vmin = fminf(v[0], v[1]), vmax = fmaxf(v[0], v[1]);
+        // min / max on packed halves (exact; fp16 -> fp32 is exact afterwards)
+        __half2 mn2 = __hmin2(hv[0], hv[1]), mx2 = __hmax2(hv[0], hv[1]);
 #pragma unroll
-        for (int k = 2; k < 16; ++k) {
-            vmin = fminf(vmin, v[k]);
-            vmax = fmaxf(vmax, v[k]);
+        for (int k = 2; k < 8; ++k) {
+            mn2 = __hmin2(mn2, hv[k]);
+            mx2 = __hmax2(mx2, hv[k]);
         }
+        float vmin = fminf(__low2float(mn2), __high2float(mn2));
+        float vmax = fmaxf(__low2float(mx2), __high2float(mx2));
 #pragma unroll
         for (int off = 1; off < L::kGroupLanes; off <<= 1) {
             vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, off));
@@ -92,22 +96,34 @@ __global__ void __launch_bounds__(256) encode_v_kernel(const __half* __restrict_
         uint32_t chunk[kW];
 #pragma unroll
         for (int k = 0; k < kW; ++k) chunk[k] = 0u;
-        bool exact = true;
+        uint32_t differ = 0u;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            const float a = __fsub_rn(v[k], zero);
-            const float tlo = __fmaf_rn(a, r_lo, kCodeMagic);
-            const float thi = __fmaf_rn(a, r_hi, kCodeMagic);
-            exact &= (__float_as_uint(tlo) == __float_as_uint(thi));
-            // the code never exceeds 2^b - 1 (a <= max - min), so masking the low bits is the page's clamp
-            put_field<BITS>(chunk, k, __float_as_uint(tlo) & kLevels);
+            const __half hk = (k & 1) ? __high2half(hv[k >> 1]) : __low2half(hv[k >> 1]);
+            const float a = sub_f16_f32(hk, zero);
+            const uint32_t tlo = __float_as_uint(__fmaf_rn(a, r_lo, kCodeMagic));
+            const uint32_t thi = __float_as_uint(__fmaf_rn(a, r_hi, kCodeMagic));
+            differ |= tlo ^ thi;
+            // the code never exceeds 2^b - 1 (a <= max - min), so the low bits of tlo are the code and the
+            // bits above are the constant kCodeMagicBits
+            if constexpr (kWordAligned) {
+                constexpr int kPer = 32 / BITS;
+                chunk[k / kPer] += tlo << (BITS * (k % kPer));          // multiply-add; the magic is removed below
+            } else {
+                put_field<BITS>(chunk, k, tlo & kLevels);
+            }
         }
-        if (!exact) {
+        if constexpr (kWordAligned) {
+#pragma unroll
+            for (int k = 0; k < kW; ++k) chunk[k] -= magic_pack_offset<BITS>();
+        }
+        if (differ != 0u) {
 #pragma unroll
             for (int k = 0; k < kW; ++k) chunk[k] = 0u;
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                const float q = rintf(__fdiv_rn(__fsub_rn(v[k], zero), scale));
+                const __half hk = (k & 1) ? __high2half(hv[k >> 1]) : __low2half(hv[k >> 1]);
+                const float q = rintf(__fdiv_rn(sub_f16_f32(hk, zero), scale));
                 put_field<BITS>(chunk, k, static_cast<uint32_t>(fminf(fmaxf(q, 0.f), static_cast<float>(kLevels))));
             }
         }
@@ -136,80 +152,102 @@ __global__ void __launch_bounds__(256) encode_v_kernel(const __half* __restrict_
     }
 }
 
+// The 16 codes (16 BITS bits) of 16-element chunk j of a value row.
 template <int D, int BITS>
-__device__ __forceinline__ void load_vchunk(const uint8_t* src, int j, uint32_t (&c)[2]) {
-    if constexpr (BITS == 4) {
-        c[0] = reinterpret_cast<const uint32_t*>(src)[j];
-        c[1] = 0u;
+__device__ __forceinline__ void load_vchunk16(const uint8_t* src, int j, uint32_t (&c)[4]) {
+    if constexpr (BITS == 2) {
+        c[0] = __ldg(reinterpret_cast<const uint32_t*>(src) + j);
+    } else if constexpr (BITS == 4) {
+        const uint2 t = __ldg(reinterpret_cast<const uint2*>(src) + j);
+        c[0] = t.x; c[1] = t.y;
     } else if constexpr (BITS == 8) {
-        const uint2 t = reinterpret_cast<const uint2*>(src)[j];
-        c[0] = t.x;
-        c[1] = t.y;
-    } else if constexpr (BITS == 2) {
-        c[0] = reinterpret_cast<const uint16_t*>(src)[j];
-        c[1] = 0u;
+        const uint4 t = __ldg(reinterpret_cast<const uint4*>(src) + j);
+        c[0] = t.x; c[1] = t.y; c[2] = t.z; c[3] = t.w;
     } else {
-        // 24 bits at byte 3j: the aligned 32-bit word holding its start, plus the next one when needed
-        const int byte = 3 * j, wi = byte >> 2, sh = 8 * (byte & 3);
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(src);
-        const uint64_t both = static_cast<uint64_t>(w[wi]) | (sh > 8 ? static_cast<uint64_t>(w[wi + 1]) << 32 : 0ull);
-        c[0] = static_cast<uint32_t>(both >> sh) & 0xFFFFFFu;
-        c[1] = 0u;
+        // 48 bits at byte 6j (2-byte aligned)
+        const uint16_t* h = reinterpret_cast<const uint16_t*>(src) + 3 * j;
+        c[0] = static_cast<uint32_t>(__ldg(h)) | (static_cast<uint32_t>(__ldg(h + 1)) << 16);
+        c[1] = __ldg(h + 2);
     }
 }
 
-// Decode: one lane owns 8 consecutive elements of a row (kU rows per lane per iteration, loads first).
+// Decode: one lane owns 16 consecutive elements of a row, so a warp's rows are one contiguous block of 512
+// output elements.  The lane writes its 16 results to the warp's shared-memory buffer and one lane sends the
+// block to global memory with a bulk copy (double-buffered), so the output bypasses the load/store queue; the
+// next rows' codes, scale and zero are loaded before the current rows are converted.
 template <int D, int BITS, int GROUP, bool OUT_F32>
 __global__ void __launch_bounds__(256) decode_v_kernel(const uint8_t* __restrict__ data, const __half* __restrict__ scales,
                                                        const __half* __restrict__ zeros, int64_t n, void* __restrict__ out) {
     using L = VLanes<D, GROUP>;
-    constexpr int kU = 1;                                         // rows per lane per iteration
     constexpr int kRowBytes = D * BITS / 8;
     constexpr int kGroups = D / GROUP;
-    const int lane = threadIdx.x & 31;
+    constexpr int kElt = OUT_F32 ? 4 : 2;
+    constexpr int kBlockBytes = 32 * 16 * kElt;                    // one warp iteration of output
+    __shared__ __align__(128) uint8_t s_out[8][2][kBlockBytes];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int j = lane % L::kRowLanes;
     const int gi = j / L::kGroupLanes;
     const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
     const int64_t step = warps_total * L::kRowsPerWarp;
-    for (int64_t wrow = (static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5)) * L::kRowsPerWarp;
-         wrow < n; wrow += step * kU) {
-        uint32_t c[kU][2];
-        float s[kU], z[kU];
-        int64_t rows[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            rows[u] = wrow + u * step + lane / L::kRowLanes;
-            if (rows[u] < n) {
-                load_vchunk<D, BITS>(data + rows[u] * kRowBytes, j, c[u]);
-                s[u] = __half2float(scales[rows[u] * kGroups + gi]);
-                z[u] = __half2float(zeros[rows[u] * kGroups + gi]);
-            }
+    int64_t wrow = (static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + warp) * L::kRowsPerWarp;
+    const int rl = lane / L::kRowLanes;
+    uint32_t c[4] = {0u, 0u, 0u, 0u};
+    __half s16 = __float2half_rn(0.f), z16 = s16;
+    if (wrow + rl < n) {
+        load_vchunk16<D, BITS>(data + (wrow + rl) * kRowBytes, j, c);
+        s16 = __ldg(scales + (wrow + rl) * kGroups + gi);
+        z16 = __ldg(zeros + (wrow + rl) * kGroups + gi);
+    }
+    for (int it = 0; wrow < n; wrow += step, ++it) {
+        const int64_t nrow = wrow + step + rl;
+        uint32_t cn[4] = {0u, 0u, 0u, 0u};
+        __half sn = s16, zn = z16;
+        if (nrow < n) {
+            load_vchunk16<D, BITS>(data + nrow * kRowBytes, j, cn);
+            sn = __ldg(scales + nrow * kGroups + gi);
+            zn = __ldg(zeros + nrow * kGroups + gi);
         }
+        const float s = __half2float(s16), z = __half2float(z16);
+        float y[16];
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            if (rows[u] >= n) continue;
-            float y[8];
+        for (int k = 0; k < 16; ++k) {
+            const uint32_t q = get_bits<BITS>(c, k * BITS);
+            y[k] = __fadd_rn(__fmul_rn(static_cast<float>(q), s), z);
+        }
+        const int buf = it & 1;
+        if (it >= 2) {
+            if (lane == 0) bulk_wait_read<1>();                      // the copy that last read this buffer is done
+            __syncwarp();
+        }
+        uint8_t* sb = &s_out[warp][buf][0];
+        if constexpr (OUT_F32) {
+            float4* o = reinterpret_cast<float4*>(sb) + 4 * lane;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) o[k] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+        } else {
+            uint32_t pk[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const uint32_t q = get_bits<BITS>(c[u], k * BITS);
-                y[k] = __fadd_rn(__fmul_rn(static_cast<float>(q), s[u]), z[u]);
+                __half2 hh = __floats2half2_rn(y[2 * k], y[2 * k + 1]);
+                pk[k] = *reinterpret_cast<uint32_t*>(&hh);
             }
-            if constexpr (OUT_F32) {
-                float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + rows[u] * D) + 2 * j;
-                o[0] = make_float4(y[0], y[1], y[2], y[3]);
-                o[1] = make_float4(y[4], y[5], y[6], y[7]);
-            } else {
-                uint4 pk;
-                __half2 h0 = __floats2half2_rn(y[0], y[1]), h1 = __floats2half2_rn(y[2], y[3]);
-                __half2 h2 = __floats2half2_rn(y[4], y[5]), h3 = __floats2half2_rn(y[6], y[7]);
-                pk.x = *reinterpret_cast<uint32_t*>(&h0);
-                pk.y = *reinterpret_cast<uint32_t*>(&h1);
-                pk.z = *reinterpret_cast<uint32_t*>(&h2);
-                pk.w = *reinterpret_cast<uint32_t*>(&h3);
-                reinterpret_cast<uint4*>(static_cast<__half*>(out) + rows[u] * D)[j] = pk;
-            }
+            uint4* o = reinterpret_cast<uint4*>(sb) + 2 * lane;
+            o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            const int64_t rows = (n - wrow < L::kRowsPerWarp) ? n - wrow : L::kRowsPerWarp;
+            bulk_store(static_cast<uint8_t*>(out) + wrow * D * kElt, smem_u32(sb), static_cast<uint32_t>(rows * D * kElt));
+            bulk_commit();
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) c[k] = cn[k];
+        s16 = sn;
+        z16 = zn;
     }
+    if (lane == 0) bulk_wait_all();
 }
 
 // -------------------------------------------------------------------------------------- key codec
@@ -245,16 +283,6 @@ struct KeyCfg {
 constexpr float kGridScale = 512.0f;
 constexpr float kGridMagic = 12583552.0f;   // 1.5 * 2^23 + 640
 
-__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Encode CTA: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-3 compute the row norms of
 // each X stage ahead of the epilogue, warps 4.. are the epilogue (kEncEpiWarps: warp w reads TMEM lanes

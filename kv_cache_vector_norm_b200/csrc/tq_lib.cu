@@ -321,7 +321,7 @@ tq_status launch_encode_v(const void* x, int64_t n, int64_t stride, const int64_
 template <int D, int BITS, int GROUP>
 tq_status launch_decode_v(const uint8_t* data, const void* scales, const void* zeros, int64_t n, void* out, int dtype,
                           cudaStream_t st) {
-    const int grid = grid_for(n * (D / 8));
+    const int grid = grid_for(n * (D / 16));
     if (dtype == TQ_F32)
         decode_v_kernel<D, BITS, GROUP, true><<<grid, 256, 0, st>>>(data, static_cast<const __half*>(scales),
                                                                     static_cast<const __half*>(zeros), n, out);
@@ -397,7 +397,9 @@ constexpr int kAttendCtasPerSm = 3;
 
 struct AttendPlan {
     int num_splits;
-    size_t partial_bytes;
+    size_t qfrag_bytes;        // query fragments, one block per (sequence, kv head)
+    size_t partial_bytes;      // split-K partials (0 with one split)
+    size_t workspace_bytes;    // qfrag_bytes + partial_bytes
 };
 
 tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan) {
@@ -432,6 +434,8 @@ tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan) {
     if (splits < 1) splits = 1;
     plan->num_splits = static_cast<int>(splits);
     plan->partial_bytes = (splits > 1) ? static_cast<size_t>(bh) * splits * (16 + 8 * a->head_dim) * 4 : 0;
+    plan->qfrag_bytes = static_cast<size_t>(bh) * ((a->head_dim / 16) * 32 + 1) * 16;
+    plan->workspace_bytes = plan->qfrag_bytes + plan->partial_bytes;
     return TQ_OK;
 }
 
@@ -461,23 +465,28 @@ tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const Attend
     p.v_scales = static_cast<const __half*>(a->v_scales);
     p.v_zeros = static_cast<const __half*>(a->v_zeros);
     p.out = a->out;
-    p.partials = static_cast<float*>(a->workspace);
+    p.qfrag = static_cast<uint4*>(a->workspace);
+    p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(a->workspace) + plan.qfrag_bytes);
     p.num_splits = plan.num_splits;
-    dim3 grid(plan.num_splits, a->num_kv_heads, a->batch);
-    kern<<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(p);
-    TQ_CUDA(cudaGetLastError(), "tq_attend_decode: launch");
+    attend_prep_kernel<D><<<dim3(a->num_kv_heads, a->batch), kPrepThreads, 0, st>>>(p);
+    TQ_CUDA(cudaGetLastError(), "tq_attend_decode: query preparation launch");
+    // the attention grid and the split merge are programmatic dependents of the grid before them: each is
+    // scheduled while its predecessor drains and waits for it (griddepcontrol.wait) before reading its output
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan.num_splits, a->num_kv_heads, a->batch);
+    cfg.blockDim = dim3(Cfg::kThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    TQ_CUDA(cudaLaunchKernelEx(&cfg, kern, p), "tq_attend_decode: launch");
     if (plan.num_splits > 1) {
-        // merge the splits in a programmatic dependent launch: it is scheduled while the main grid drains
-        cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(p.group, a->num_kv_heads, a->batch);
         cfg.blockDim = dim3(kMergeThreads);
         cfg.dynamicSmemBytes = 0;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
         TQ_CUDA(cudaLaunchKernelEx(&cfg, attend_merge_kernel<D>, p), "tq_attend_decode: merge launch");
     }
     return TQ_OK;
@@ -508,7 +517,7 @@ extern "C" tq_status tq_attend_workspace_bytes(const tq_attend_args* a, size_t* 
     AttendPlan plan;
     tq_status s = plan_attend(a, &plan);
     if (s != TQ_OK) return s;
-    *bytes = plan.partial_bytes;
+    *bytes = plan.workspace_bytes;
     return TQ_OK;
 }
 
@@ -521,9 +530,9 @@ extern "C" tq_status tq_attend_decode(const tq_codec* c, const tq_attend_args* a
     if (a->head_dim != c->d) return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: head_dim=%d but the codec has d=%d", a->head_dim, c->d);
     if (!a->q || !a->k_packed || !a->k_norms || !a->v_data || !a->v_scales || !a->v_zeros || !a->out)
         return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: NULL pointer in args");
-    if (plan.partial_bytes && (!a->workspace || a->workspace_bytes < plan.partial_bytes))
+    if (!a->workspace || a->workspace_bytes < plan.workspace_bytes)
         return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: workspace of %zu bytes required (got %zu)",
-                    plan.partial_bytes, a->workspace ? a->workspace_bytes : static_cast<size_t>(0));
+                    plan.workspace_bytes, a->workspace ? a->workspace_bytes : static_cast<size_t>(0));
     if (!aligned(a->q, 16) || !aligned(a->k_packed, 16) || !aligned(a->k_norms, 16) || !aligned(a->v_data, 16) ||
         !aligned(a->v_scales, 16) || !aligned(a->v_zeros, 16) || !aligned(a->out, 16) || !aligned(a->workspace, 16))
         return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: every pointer must be 16-byte aligned");
@@ -579,11 +588,11 @@ extern "C" tq_status tq_attend_decode_noalloc(const tq_codec* c, const tq_attend
     AttendPlan plan;
     tq_status s = plan_attend(a, &plan);
     if (s != TQ_OK) return s;
-    if (plan.partial_bytes > TQ_ATTEND_SCRATCH_BYTES)
+    if (plan.workspace_bytes > TQ_ATTEND_SCRATCH_BYTES)
         return fail(TQ_ERR_INVALID_ARG,
-                    "tq_attend_decode_noalloc: this launch needs %zu bytes of split-K scratch but the static scratch "
+                    "tq_attend_decode_noalloc: this launch needs %zu bytes of scratch but the static scratch "
                     "holds %u; use tq_attend_decode with a workspace",
-                    plan.partial_bytes, TQ_ATTEND_SCRATCH_BYTES);
+                    plan.workspace_bytes, TQ_ATTEND_SCRATCH_BYTES);
     void* scratch = nullptr;
     if ((s = attend_scratch(&scratch)) != TQ_OK) return s;
     tq_attend_args with_scratch = *a;
