@@ -437,12 +437,11 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                 for (int c = 0; c < D / 8; ++c) {
                     // squares of fp16 values are exact in fp32; eight partial sums keep the rounding small
                     const uint4 v = *reinterpret_cast<const uint4*>(xs + (c >> 3) * C::kTileBlockBytes + sw128_offset(r, c & 7));
-                    const __half2* h = reinterpret_cast<const __half2*>(&v);
+                    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const float2 f = __half22float2(h[k]);
-                        acc[2 * k] = fmaf(f.x, f.x, acc[2 * k]);
-                        acc[2 * k + 1] = fmaf(f.y, f.y, acc[2 * k + 1]);
+                        acc[2 * k] = fma_f16_f32(static_cast<uint16_t>(u[k]), acc[2 * k]);
+                        acc[2 * k + 1] = fma_f16_f32(static_cast<uint16_t>(u[k] >> 16), acc[2 * k + 1]);
                     }
                 }
                 const float nrm = sqrtf(((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
@@ -500,8 +499,10 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                     const float y = __uint_as_float(v[j]) * inv;
                     const float g = fmaf(y, kGridScale, kGridMagic);
                     const uint32_t e = s_lut[__float_as_uint(g) & (C::kLutEntries - 1)];
-                    const uint32_t idx = (e & 15u) + (y > __uint_as_float(e & ~15u) ? 1u : 0u);
-                    put_field<BITS>(w, j, idx);
+                    // the entry read as a float is the cell's boundary moved by at most 15 ulps (its low 4 bits hold
+                    // the count; the boundary's own low bits are zero), or a NaN / +inf when the cell has none
+                    const uint32_t idx = (e & 15u) + (y > __uint_as_float(e) ? 1u : 0u);
+                    add_field<BITS>(w, j, idx);
                 }
                 const int boff = (c0 + k * 32) * BITS / 8;
                 if (staged) {

@@ -203,6 +203,22 @@ __device__ __forceinline__ void put_field(uint32_t (&w)[NW], int j, uint32_t v) 
     if (sh + BITS > 32) w[wi + 1] |= v >> (32 - sh);
 }
 
+// Add value v (< 2^BITS) into field j of the zero-initialised bitstream `w` (fields do not overlap, so this is
+// the same as OR-ing it in, as a shift-add).
+template <int BITS, int NW>
+__device__ __forceinline__ void add_field(uint32_t (&w)[NW], int j, uint32_t v) {
+    const int bit = j * BITS, wi = bit >> 5, sh = bit & 31;
+    w[wi] += v << sh;
+    if (sh + BITS > 32) w[wi + 1] += v >> (32 - sh);
+}
+
+// acc + h * h for an fp16 h (given by its bits) with one rounding: h * h is exact in fp32
+__device__ __forceinline__ float fma_f16_f32(uint16_t h, float acc) {
+    float d;
+    asm("fma.rn.f32.f16 %0, %1, %1, %2;" : "=f"(d) : "h"(h), "f"(acc));
+    return d;
+}
+
 // Field of width W starting at bit `bit` of the little-endian bitstream `w`.
 template <int W, int NW>
 __device__ __forceinline__ uint32_t get_bits(const uint32_t (&w)[NW], int bit) {
