@@ -311,6 +311,7 @@ struct EncLayout {
     static constexpr int kBars = 4 * C::kEncStages + 10;
     static constexpr uint32_t kMisc = kBar + 8 * kBars;
     static constexpr uint32_t kBytes = kMisc + 16 + 1024;                  // + alignment slack
+    static_assert(kBytes <= 227 * 1024, "encode layout exceeds the shared memory of one CTA");
 };
 
 template <int D, int BITS>
@@ -560,16 +561,22 @@ struct DecLayout {
     using E = DecCfg<D>;
     static constexpr int kRowBytes = D * BITS / 8;
     static constexpr int kInBytes = 128 * kRowBytes + 128 * 4;            // packed rows + norms
+    // code-pair table: one copy per shared-memory bank (entry e of lane l at 128 e + 4 l) where it fits
+    static constexpr bool kReplPairs = (D <= 128);
+    static constexpr int kPairBytes = (1 << (2 * BITS)) * (kReplPairs ? 128 : 4);
     static constexpr uint32_t kPit = 0;
     static constexpr uint32_t kA = kPit + C::kPiBytes;
     static constexpr uint32_t kIn = kA + C::kDecBufs * C::kTileBytes;
     static constexpr uint32_t kPair = kIn + C::kDecInBufs * kInBytes;
-    static constexpr uint32_t kPatch = (kPair + 256 * 4 + 127) & ~127u;   // per-warp output transpose
-    static constexpr uint32_t kPatchBytes = 32 * 64;                      // 32 rows x 64 bytes
-    static constexpr uint32_t kBar = kPatch + E::kEpiWarps * kPatchBytes;
+    // per-warp output patches: 32 rows x 64 bytes, 64B-swizzled, the source of one tensor store each
+    static constexpr int kPatchBufs = (D <= 128) ? 2 : 1;
+    static constexpr uint32_t kPatchBytes = 32 * 64;
+    static constexpr uint32_t kPatch = (kPair + kPairBytes + 511) & ~511u;     // 64B swizzle repeats every 512 bytes
+    static constexpr uint32_t kBar = kPatch + E::kEpiWarps * kPatchBufs * kPatchBytes;
     static constexpr int kBars = 2 * C::kDecBufs + 2 * C::kDecInBufs + 8;
     static constexpr uint32_t kMisc = kBar + 8 * kBars;
     static constexpr uint32_t kBytes = kMisc + 16 + 1024;
+    static_assert(kBytes <= 227 * 1024, "decode layout exceeds the shared memory of one CTA");
 };
 
 template <int D, int BITS>
@@ -579,9 +586,9 @@ __host__ __device__ constexpr uint32_t dec_smem_bytes() {
 
 template <int D, int BITS, bool OUT_F32>
 __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
-    decode_k_kernel(const __grid_constant__ CUtensorMap tmap_pit, const uint32_t* __restrict__ pair_lut_g,
-                    const uint8_t* __restrict__ packed, const float* __restrict__ norms, int64_t n,
-                    void* __restrict__ out) {
+    decode_k_kernel(const __grid_constant__ CUtensorMap tmap_pit, const __grid_constant__ CUtensorMap tmap_out,
+                    const uint32_t* __restrict__ pair_lut_g, const uint8_t* __restrict__ packed,
+                    const float* __restrict__ norms, int64_t n) {
     using C = KeyCfg<D>;
     using E = DecCfg<D>;
     using Lo = DecLayout<D, BITS>;
@@ -630,7 +637,11 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
-    for (int i = threadIdx.x; i < kPairs; i += blockDim.x) s_pair[i] = pair_lut_g[i];
+    if constexpr (Lo::kReplPairs) {
+        for (int i = threadIdx.x; i < kPairs * 32; i += blockDim.x) s_pair[i] = pair_lut_g[i >> 5];
+    } else {
+        for (int i = threadIdx.x; i < kPairs; i += blockDim.x) s_pair[i] = pair_lut_g[i];
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -693,7 +704,8 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
         const int quarter = warp & 3;
         const int c0 = (ew >> 2) * E::kCols;               // first column of this warp
         const int r = quarter * 32 + lane;
-        uint8_t* patch = smem + Lo::kPatch + ew * Lo::kPatchBytes;
+        uint8_t* patches = smem + Lo::kPatch + ew * Lo::kPatchBufs * Lo::kPatchBytes;
+        int pcount = 0;                                    // tensor stores issued by this warp
         float nrm_next = 0.f;
 
         // build the A tile (c_op[idx] as fp16, 128B-swizzled K-major) for local tile index lt
@@ -726,7 +738,10 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
             for (int c = 0; c < E::kCols / 8; ++c) {
                 uint32_t h[4];
 #pragma unroll
-                for (int p = 0; p < 4; ++p) h[p] = s_pair[get_bits<2 * BITS>(w, (c * 8 + 2 * p) * BITS)];
+                for (int p = 0; p < 4; ++p) {
+                    const uint32_t key = get_bits<2 * BITS>(w, (c * 8 + 2 * p) * BITS);
+                    h[p] = Lo::kReplPairs ? s_pair[key * 32 + lane] : s_pair[key];
+                }
                 const int col = c0 + c * 8;
                 *reinterpret_cast<uint4*>(as + (col >> 6) * C::kTileBlockBytes + sw128_offset(r, (col & 63) >> 3)) =
                     make_uint4(h[0], h[1], h[2], h[3]);
@@ -746,7 +761,6 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
             const int64_t next = tile + gridDim.x;
             if (next < num_tiles && !build(li + 1, next)) break;
             const int a = li & 1;
-            const int64_t rows = tile_rows(tile);
             if (!mbar_wait(b_accfull + 8 * a, (li >> 1) & 1, abort_flag)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + a * D + c0;
@@ -760,12 +774,20 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(b_accempty + 8 * a);
                 }
-                // per 64-byte segment of this row's chunk: scale, convert, write it into the warp's patch as
-                // four 16-byte pieces (swizzled by row), then read the patch back row-contiguously (4 lanes per
-                // row, 8 rows per instruction) so each warp store covers whole 64-byte row segments
+                // per 64-byte segment of this row's chunk: scale, convert and write it as row r of the warp's
+                // 64B-swizzled patch (32 rows x 64 bytes); one lane then stores the patch with a tensor store
+                // (rows past n are clipped by the tensor map)
                 const int col0 = c0 + ch * 32;
 #pragma unroll
                 for (int ps = 0; ps < kPasses; ++ps) {
+                    uint8_t* patch = patches + (pcount % Lo::kPatchBufs) * Lo::kPatchBytes;
+                    if (pcount >= Lo::kPatchBufs) {
+                        // the store that last read this patch is done reading it
+                        if (lane == 0) {
+                            if constexpr (Lo::kPatchBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();
+                        }
+                        __syncwarp();
+                    }
 #pragma unroll
                     for (int pc = 0; pc < 4; ++pc) {
                         uint4 pk;
@@ -787,22 +809,18 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
                         }
                         *reinterpret_cast<uint4*>(patch + lane * 64 + ((pc ^ ((lane >> 1) & 3)) * 16)) = pk;
                     }
+                    fence_proxy_async_smem();
                     __syncwarp();
-#pragma unroll
-                    for (int it = 0; it < 4; ++it) {
-                        const int rr = it * 8 + (lane >> 2), pc = lane & 3;
-                        const uint4 val = *reinterpret_cast<const uint4*>(patch + rr * 64 + ((pc ^ ((rr >> 1) & 3)) * 16));
-                        const int trow = quarter * 32 + rr;
-                        if (trow < rows) {
-                            uint8_t* gdst = static_cast<uint8_t*>(out) + ((tile * 128 + trow) * D + col0) * kOutBytes +
-                                            ps * 64 + pc * 16;
-                            *reinterpret_cast<uint4*>(gdst) = val;
-                        }
+                    if (lane == 0) {
+                        tma_store_2d(&tmap_out, smem_u32(patch), col0 + ps * (64 / kOutBytes),
+                                     static_cast<int>(tile * 128 + quarter * 32));
+                        bulk_commit();
                     }
-                    __syncwarp();
+                    ++pcount;
                 }
             }
         }
+        if (lane == 0) bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();

@@ -76,6 +76,23 @@ tq_status make_tmap_f16(CUtensorMap* map, const void* base, uint64_t rows, uint6
     return TQ_OK;
 }
 
+// 2-D tensor map for the decoded keys: rows x cols of fp16 or fp32 (dense rows), 64B swizzle, box of
+// 64 bytes x 32 rows (one warp's patch).
+tq_status make_tmap_out(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, bool f32) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return fail(TQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+    const uint64_t elt = f32 ? 4 : 2;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * elt};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(64 / elt), 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+    return TQ_OK;
+}
+
 // Raise the dynamic shared-memory limit of a kernel once per device.
 template <typename K>
 cudaError_t allow_smem(K kernel, uint32_t bytes, std::atomic<uint64_t>& done_mask) {
@@ -234,14 +251,17 @@ tq_status launch_decode_k(const tq_codec* c, const uint8_t* packed, const float*
     constexpr uint32_t smem = dec_smem_bytes<D, BITS>();
     const int64_t tiles = (n + 127) / 128;
     const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+    CUtensorMap tmap_out;
+    tq_status s = make_tmap_out(&tmap_out, out, static_cast<uint64_t>(n), D, dtype == TQ_F32);
+    if (s != TQ_OK) return s;
     if (dtype == TQ_F32) {
         auto kern = decode_k_kernel<D, BITS, true>;
         TQ_CUDA(allow_smem(kern, smem, mask32), "tq_decode_k: cudaFuncSetAttribute");
-        kern<<<grid, DecCfg<D>::kThreads, smem, st>>>(c->tmap_pit, c->pair_lut, packed, norms, n, out);
+        kern<<<grid, DecCfg<D>::kThreads, smem, st>>>(c->tmap_pit, tmap_out, c->pair_lut, packed, norms, n);
     } else {
         auto kern = decode_k_kernel<D, BITS, false>;
         TQ_CUDA(allow_smem(kern, smem, mask16), "tq_decode_k: cudaFuncSetAttribute");
-        kern<<<grid, DecCfg<D>::kThreads, smem, st>>>(c->tmap_pit, c->pair_lut, packed, norms, n, out);
+        kern<<<grid, DecCfg<D>::kThreads, smem, st>>>(c->tmap_pit, tmap_out, c->pair_lut, packed, norms, n);
     }
     TQ_CUDA(cudaGetLastError(), "tq_decode_k: launch");
     return TQ_OK;
@@ -295,6 +315,8 @@ extern "C" tq_status tq_decode_k(const tq_codec* c, const uint8_t* packed, const
     if (!packed || !norms || !out) return fail(TQ_ERR_INVALID_ARG, "tq_decode_k: packed, norms and out must be non-NULL");
     if (!aligned(packed, 16) || !aligned(norms, 16) || !aligned(out, 16))
         return fail(TQ_ERR_INVALID_ARG, "tq_decode_k: packed, norms and out must be 16-byte aligned");
+    if (n > INT32_MAX) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_k: n=%lld rows (at most 2^31 - 1 per call)",
+                                   static_cast<long long>(n));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     TQ_DISPATCH_DB(c->d, c->bits, launch_decode_k, c, packed, norms, n, out, out_dtype, st);
 }
