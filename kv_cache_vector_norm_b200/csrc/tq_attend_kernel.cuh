@@ -65,9 +65,11 @@ struct AttCfg {
     static constexpr int kQuarterBits = D * KB / 4;  // one lane's quarter of a key row (16-bit multiple)
     static constexpr int kQuarterHalves = kQuarterBits / 16;
     static constexpr int kQuarterWords = (kQuarterHalves + 1) / 2 + 1;
-    static constexpr int kMinBlocks = (D == 256) ? 1 : 3;
+    static constexpr int kMinBlocks = (D == 256) ? 1 : 4;
     static constexpr int kPartFloats = 16 + 8 * D;
-    static constexpr bool kQInRegs = (D <= 128);     // score A fragments held in registers
+    // score A fragments from shared memory (one 16-byte load per k-step): keeping them in registers would
+    // cost 32 registers and one resident CTA per SM
+    static constexpr bool kQInRegs = false;
     // key table: a pair of codes (2 KB bits, first code in the low bits) -> half2 of codebook values, with one
     // copy per shared-memory bank (entry e of lane l at byte 128 e + 4 l), so lookups never conflict
     static constexpr int kPairs = 1 << (2 * KB);

@@ -415,7 +415,7 @@ extern "C" tq_status tq_decode_v(int d, int bits, int group, const uint8_t* data
 
 namespace {
 
-constexpr int kAttendCtasPerSm = 3;
+constexpr int kAttendCtasPerSm = 4;
 
 struct AttendPlan {
     int num_splits;
