@@ -51,7 +51,7 @@ struct AttCfg {
     static constexpr int kThreads = 32 * (kWarps + 1);
     static constexpr int kChunkTok = 16;             // tokens per chunk (= one paged block)
     static constexpr int kTileTok = kWarps * kChunkTok;
-    static constexpr int kStages = 4;
+    static constexpr int kStages = 4;               // a power of two
     static constexpr int kKRow = D * KB / 8;
     static constexpr int kVRow = D * VB / 8;
     static constexpr int kVGroups = D / VG;
@@ -128,11 +128,13 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // hi/lo bf16 split of two values: hi = x truncated to bf16 (the upper 16 bits), lo = bf16(x - hi);
-// hi + lo is within 2^-16 |x| of x
-__device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-    const uint32_t u0 = __float_as_uint(x0), u1 = __float_as_uint(x1);
+// hi + lo is within 2^-16 |x| of x.  x - hi is exact; it is one packed f32x2 FMA (-1 * hi + x).
+__device__ __forceinline__ void split_bf16(float2 x, uint32_t& hi, uint32_t& lo) {
+    const uint32_t u0 = __float_as_uint(x.x), u1 = __float_as_uint(x.y);
     hi = __byte_perm(u0, u1, 0x7632);
-    lo = pack_bf16(x0 - __uint_as_float(u0 & 0xFFFF0000u), x1 - __uint_as_float(u1 & 0xFFFF0000u));
+    const float2 h = make_float2(__uint_as_float(u0 & 0xFFFF0000u), __uint_as_float(u1 & 0xFFFF0000u));
+    const float2 r = __ffma2_rn(h, make_float2(-1.0f, -1.0f), x);
+    lo = pack_bf16(r.x, r.y);
 }
 
 // n fp16 values at p (n in {1, 2, 4, 8}, naturally aligned) as floats
@@ -223,6 +225,9 @@ __global__ void __launch_bounds__(kPrepThreads) attend_prep_kernel(const AttendP
     const int h = blockIdx.x, b = blockIdx.y;
     const int G = p.group;
     uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();
+    // the attention grid may be scheduled at once and start streaming the cache; its consumers wait for this
+    // grid's completion (griddepcontrol.wait) before they read the fragments
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // q_rot[g][n] = sum_k q[g][k] Pi_op[n][k] on the tensor cores (fp16 inputs are exact products)
     const __half* qg = p.q + (static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * G) * D;
     for (int nt = warp; nt < D / 8; nt += kWarps) {
@@ -278,8 +283,6 @@ __global__ void __launch_bounds__(kPrepThreads) attend_prep_kernel(const AttendP
         qf[i] = f;
     }
     if (threadIdx.x == 0) qf[KS * 32] = make_uint4(__float_as_uint(1.0f / pre), 0u, 0u, 0u);
-    // the attention grid may start streaming the cache; its consumers wait for this grid's completion
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Fused decode attention for one (split, kv head, sequence).  Per 16-token chunk and warp:
@@ -395,11 +398,14 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         float m_run = -INFINITY, l_run = 0.f;
         const int tok[4] = {2 * tig, 2 * tig + 1, 8 + 2 * tig, 9 + 2 * tig};
 
-        for (int64_t ti = 0; ti < ntiles; ++ti) {
-            const int s = static_cast<int>(ti % S);
+        // 32-bit loop state: a split holds fewer than 2^31 chunks
+        const int ntiles32 = static_cast<int>(ntiles);
+        const int nrel = static_cast<int>(c_end - c_begin);
+        for (int ti = 0; ti < ntiles32; ++ti) {
+            const int s = ti % S;
             if (!mbar_wait(b_full + 8 * s, static_cast<uint32_t>((ti / S) & 1), abort_flag)) break;
-            const int64_t chunk = c_begin + ti * C::kWarps + warp;
-            if (chunk < c_end) {
+            const int rel = ti * C::kWarps + warp;        // chunk index within the split
+            if (rel < nrel) {
                 const uint8_t* st = smem + s * C::kStageBytes;
                 const uint8_t* kch = st + C::kKOff + warp * 16 * C::kKRow;
                 // ---- scores: S'[16 x 8 tokens] per n-tile, rows gid (hi part) and gid+8 (lo part)
@@ -437,7 +443,8 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                 }
                 // ---- logits (log2 domain) of head gid for tokens 2tig, 2tig+1, 8+2tig, 9+2tig
                 const float* nrm = reinterpret_cast<const float*>(st + C::kNOff) + warp * 16;
-                const int64_t valid = T - chunk * 16;
+                const int64_t rem = T - (c_begin + rel) * 16;
+                const int valid = (rem < 16) ? static_cast<int>(rem) : 16;
                 float lg[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -478,8 +485,19 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                 for (int e = 0; e < 4; ++e) {
                     float zr[G8];
                     load_halves<G8>(zch + tok[e] * G8, zr);
+                    if constexpr (G8 % 2 == 0) {
+                        // two groups per packed f32x2 FMA
 #pragma unroll
-                    for (int g = 0; g < G8; ++g) zacc[g] = fmaf(pr[e], zr[g], zacc[g]);
+                        for (int g = 0; g < G8; g += 2) {
+                            const float2 t = __ffma2_rn(make_float2(pr[e], pr[e]), make_float2(zr[g], zr[g + 1]),
+                                                        make_float2(zacc[g], zacc[g + 1]));
+                            zacc[g] = t.x;
+                            zacc[g + 1] = t.y;
+                        }
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < G8; ++g) zacc[g] = fmaf(pr[e], zr[g], zacc[g]);
+                    }
                 }
                 // ---- values: A = codes (exact bf16), B = hi/lo of p * scale; per 32-column slice
                 uint32_t bh0 = 0, bh1 = 0, bl0 = 0, bl1 = 0;
@@ -487,11 +505,12 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                 for (int sl = 0; sl < NSL; ++sl) {
                     const int g = (32 * sl) / VG;
                     if (sl == 0 || (32 * sl) % VG == 0) {
-                        float x[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) x[e] = pr[e] * __half2float(sch[tok[e] * G8 + g]);
-                        split_bf16(x[0], x[1], bh0, bl0);
-                        split_bf16(x[2], x[3], bh1, bl1);
+                        const float2 x01 = __fmul2_rn(make_float2(pr[0], pr[1]),
+                                                      make_float2(__half2float(sch[tok[0] * G8 + g]), __half2float(sch[tok[1] * G8 + g])));
+                        const float2 x23 = __fmul2_rn(make_float2(pr[2], pr[3]),
+                                                      make_float2(__half2float(sch[tok[2] * G8 + g]), __half2float(sch[tok[3] * G8 + g])));
+                        split_bf16(x01, bh0, bl0);
+                        split_bf16(x23, bh1, bl1);
                     }
                     uint32_t f[4];
 #pragma unroll

@@ -97,20 +97,26 @@ __global__ void __launch_bounds__(256) encode_v_kernel(const __half* __restrict_
 #pragma unroll
         for (int k = 0; k < kW; ++k) chunk[k] = 0u;
         uint32_t differ = 0u;
+        const float2 rlo2 = make_float2(r_lo, r_lo), rhi2 = make_float2(r_hi, r_hi);
+        const float2 mag2 = make_float2(kCodeMagic, kCodeMagic);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const __half hk = (k & 1) ? __high2half(hv[k >> 1]) : __low2half(hv[k >> 1]);
-            const float a = sub_f16_f32(hk, zero);
-            const uint32_t tlo = __float_as_uint(__fmaf_rn(a, r_lo, kCodeMagic));
-            const uint32_t thi = __float_as_uint(__fmaf_rn(a, r_hi, kCodeMagic));
-            differ |= tlo ^ thi;
-            // the code never exceeds 2^b - 1 (a <= max - min), so the low bits of tlo are the code and the
-            // bits above are the constant kCodeMagicBits
-            if constexpr (kWordAligned) {
-                constexpr int kPer = 32 / BITS;
-                chunk[k / kPer] += tlo << (BITS * (k % kPer));          // multiply-add; the magic is removed below
-            } else {
-                put_field<BITS>(chunk, k, tlo & kLevels);
+        for (int k2 = 0; k2 < 8; ++k2) {
+            // two elements per packed f32x2 FMA (each lane of the pair is the scalar IEEE operation)
+            const float2 a = make_float2(sub_f16_f32(__low2half(hv[k2]), zero), sub_f16_f32(__high2half(hv[k2]), zero));
+            const float2 lo2 = __ffma2_rn(a, rlo2, mag2), hi2 = __ffma2_rn(a, rhi2, mag2);
+            const uint32_t tlo[2] = {__float_as_uint(lo2.x), __float_as_uint(lo2.y)};
+            differ |= (tlo[0] ^ __float_as_uint(hi2.x)) | (tlo[1] ^ __float_as_uint(hi2.y));
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int k = 2 * k2 + e;
+                // the code never exceeds 2^b - 1 (a <= max - min), so the low bits of tlo are the code and the
+                // bits above are the constant kCodeMagicBits
+                if constexpr (kWordAligned) {
+                    constexpr int kPer = 32 / BITS;
+                    chunk[k / kPer] += tlo[e] << (BITS * (k % kPer));   // shift-add; the magic is removed below
+                } else {
+                    put_field<BITS>(chunk, k, tlo[e] & kLevels);
+                }
             }
         }
         if constexpr (kWordAligned) {
@@ -208,11 +214,18 @@ __global__ void __launch_bounds__(256) decode_v_kernel(const uint8_t* __restrict
             zn = __ldg(zeros + nrow * kGroups + gi);
         }
         const float s = __half2float(s16), z = __half2float(z16);
+        // q * s is exact in fp32 (q < 2^8, s an fp16), so (2^23 + q) s - 2^23 s in one FMA is exactly q s and the
+        // page's two roundings reduce to the one of the final addition: y = RN(RN(q s) + z) = RN(q s + z)
+        const float2 s2 = make_float2(s, s), z2 = make_float2(z, z);
+        const float2 off2 = make_float2(-8388608.0f * s, -8388608.0f * s);
         float y[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const uint32_t q = get_bits<BITS>(c, k * BITS);
-            y[k] = __fadd_rn(__fmul_rn(static_cast<float>(q), s), z);
+        for (int k2 = 0; k2 < 8; ++k2) {
+            const float2 qm = make_float2(__uint_as_float(0x4B000000u | get_bits<BITS>(c, 2 * k2 * BITS)),
+                                          __uint_as_float(0x4B000000u | get_bits<BITS>(c, (2 * k2 + 1) * BITS)));
+            const float2 yy = __fadd2_rn(__ffma2_rn(qm, s2, off2), z2);
+            y[2 * k2] = yy.x;
+            y[2 * k2 + 1] = yy.y;
         }
         const int buf = it & 1;
         if (it >= 2) {
@@ -495,15 +508,23 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                 uint32_t w[BITS];
 #pragma unroll
                 for (int i = 0; i < BITS; ++i) w[i] = 0u;
+                const float2 inv2 = make_float2(inv, inv);
+                const float2 gs2 = make_float2(kGridScale, kGridScale), gm2 = make_float2(kGridMagic, kGridMagic);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float y = __uint_as_float(v[j]) * inv;
-                    const float g = fmaf(y, kGridScale, kGridMagic);
-                    const uint32_t e = s_lut[__float_as_uint(g) & (C::kLutEntries - 1)];
-                    // the entry read as a float is the cell's boundary moved by at most 15 ulps (its low 4 bits hold
-                    // the count; the boundary's own low bits are zero), or a NaN / +inf when the cell has none
-                    const uint32_t idx = (e & 15u) + (y > __uint_as_float(e) ? 1u : 0u);
-                    add_field<BITS>(w, j, idx);
+                for (int j2 = 0; j2 < 16; ++j2) {
+                    // two coordinates per packed f32x2 multiply and FMA
+                    const float2 y2 = __fmul2_rn(make_float2(__uint_as_float(v[2 * j2]), __uint_as_float(v[2 * j2 + 1])), inv2);
+                    const float2 g2 = __ffma2_rn(y2, gs2, gm2);
+                    const float yv[2] = {y2.x, y2.y};
+                    const uint32_t cell[2] = {__float_as_uint(g2.x), __float_as_uint(g2.y)};
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const uint32_t e = s_lut[cell[e2] & (C::kLutEntries - 1)];
+                        // the entry read as a float is the cell's boundary moved by at most 15 ulps (its low 4 bits
+                        // hold the count; the boundary's own low bits are zero), or a NaN / +inf when it has none
+                        const uint32_t idx = (e & 15u) + (yv[e2] > __uint_as_float(e) ? 1u : 0u);
+                        add_field<BITS>(w, 2 * j2 + e2, idx);
+                    }
                 }
                 const int boff = (c0 + k * 32) * BITS / 8;
                 if (staged) {
