@@ -115,12 +115,6 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
-    uint32_t v;
-    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
-
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -215,7 +209,7 @@ __device__ __forceinline__ uint32_t vfield(const uint8_t* row, int sl, int gid) 
 constexpr int kPrepThreads = 512;
 
 template <int D>
-__global__ void __launch_bounds__(kPrepThreads) attend_prep_kernel(const AttendParams p) {
+__global__ void __launch_bounds__(kPrepThreads, 1) attend_prep_kernel(const AttendParams p) {
     constexpr int KS = D / 16;
     constexpr int kWarps = kPrepThreads / 32;            // one n-tile of q_rot per warp (two at d = 256)
     __shared__ float s_qr[8 * D];
@@ -258,9 +252,10 @@ __global__ void __launch_bounds__(kPrepThreads) attend_prep_kernel(const AttendP
     amax = s_red[0];
 #pragma unroll
     for (int w = 1; w < kWarps; ++w) amax = fmaxf(amax, s_red[w]);
-    int ex = 0;
-    if (amax > 0.f) frexpf(amax, &ex);
-    const float pre = (amax > 0.f) ? ldexpf(1.0f, 14 - ex) : 1.0f;     // max |q| * pre in [8192, 16384)
+    // amax = m 2^ex with m in [0.5, 1) (read from the exponent field; clamped for tiny or zero queries)
+    int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 255u) - 126;
+    ex = (amax > 0.f) ? max(ex, -100) : 14;
+    const float pre = __uint_as_float(static_cast<uint32_t>(127 + 14 - ex) << 23);   // max |q| * pre in [8192, 16384)
     // score A fragments, coordinate-permuted so lane tig owns coords [tig*D/4, (tig+1)*D/4):
     // k-slots (2tig, 2tig+1, 2tig+8, 2tig+9) of k-step ks <- coords tig*D/4 + 4ks + (0, 1, 2, 3)
     for (int i = threadIdx.x; i < KS * 32; i += 32 * kWarps) {

@@ -6,6 +6,12 @@
 namespace tq {
 namespace dev {
 
+// Grid of the key encoder's nearest-level search (built on the host, see tq_lib.cu build_grid_lut):
+// kGridCells cells of width 1 / kGridRes, cell = rint(kGridRes * y + kGridOffset).
+constexpr int kGridRes = 64;
+constexpr int kGridOffset = 128;
+constexpr int kGridCells = 256;
+
 // ------------------------------------------------------------------------------------ value codec
 // "KV Cache API", values.py quantize_values / dequantize_values.  The lanes of one scale group reduce
 // min/max with shuffles.  Every arithmetic step is the page's fp32 operation with one rounding.
@@ -285,16 +291,16 @@ struct KeyCfg {
     static constexpr int kTmemCols = 2 * D;                  // two accumulator buffers
     static constexpr int kHalfCols = D / 2;
     static constexpr int kChunks = kHalfCols / 32;           // 32-column TMEM loads per thread per tile
-    static constexpr int kLutEntries = 2048;                 // encode grid table
+    static constexpr int kLutEntries = kGridCells;           // encode grid table, replicated once per bank
     static constexpr bool kEncStaged = (D <= 128);           // packed output staged for a bulk store
     static constexpr uint32_t kIdesc = idesc_f16_f32(128, D);
 };
 
-// Encode-side search: y maps to grid cell rint(512 y + 640) (an exact FMA into the 1.5*2^23 magic
-// range); the cell's entry holds the count L of boundaries below the cell and the one boundary B that
-// may fall inside it (+inf if none): index = L + (y > B).
-constexpr float kGridScale = 512.0f;
-constexpr float kGridMagic = 12583552.0f;   // 1.5 * 2^23 + 640
+// Encode-side search: y maps to grid cell rint(64 y + 128) (an exact FMA into the 1.5*2^23 magic range);
+// the cell's entry holds the count L of boundaries below the cell and the one boundary B that may fall
+// inside it (+inf if none): index = L + (y > B).
+constexpr float kGridScale = static_cast<float>(kGridRes);
+constexpr float kGridMagic = 12582912.0f + kGridOffset;   // 1.5 * 2^23 + 128
 
 
 // Encode CTA: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-3 compute the row norms of
@@ -318,7 +324,7 @@ struct EncLayout {
     static constexpr uint32_t kPi = 0;
     static constexpr uint32_t kX = kPi + C::kPiBytes;
     static constexpr uint32_t kLut = kX + C::kEncStages * C::kTileBytes;
-    static constexpr uint32_t kPk = kLut + C::kLutEntries * 4;
+    static constexpr uint32_t kPk = kLut + C::kLutEntries * 128;            // entry e of lane l at 128 e + 4 l
     static constexpr uint32_t kNorm = kPk + 2 * kPkBytes;                   // [stage][128] {norm, 1/(norm+1e-8)}
     static constexpr uint32_t kBar = kNorm + C::kEncStages * 128 * 8;
     static constexpr int kBars = 4 * C::kEncStages + 10;
@@ -382,8 +388,8 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
-    for (int i = threadIdx.x; i < C::kLutEntries; i += blockDim.x)
-        reinterpret_cast<uint32_t*>(smem + Lo::kLut)[i] = lut_g[i];
+    for (int i = threadIdx.x; i < C::kLutEntries * 32; i += blockDim.x)
+        reinterpret_cast<uint32_t*>(smem + Lo::kLut)[i] = lut_g[i >> 5];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -479,6 +485,7 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         const int c0 = (ew >> 2) * E::kCols;                  // first column of this warp
         const int r = quarter * 32 + lane;
         const bool issuer = (ew == 0 && lane == 0);           // issues the bulk stores of staged tiles
+        const uint32_t lut_lane = smem_u32(s_lut) + 4u * lane; // this lane's copy of the grid table (its own bank)
         int li = 0;
         for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
             const int s = li % S, a = li & 1, pb = li & 1;
@@ -519,7 +526,7 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                     const uint32_t cell[2] = {__float_as_uint(g2.x), __float_as_uint(g2.y)};
 #pragma unroll
                     for (int e2 = 0; e2 < 2; ++e2) {
-                        const uint32_t e = s_lut[cell[e2] & (C::kLutEntries - 1)];
+                        const uint32_t e = lds_u32(lut_lane + (cell[e2] & (C::kLutEntries - 1)) * 128u);
                         // the entry read as a float is the cell's boundary moved by at most 15 ulps (its low 4 bits
                         // hold the count; the boundary's own low bits are zero), or a NaN / +inf when it has none
                         const uint32_t idx = (e & 15u) + (yv[e2] > __uint_as_float(e) ? 1u : 0u);
@@ -726,6 +733,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
         const int c0 = (ew >> 2) * E::kCols;               // first column of this warp
         const int r = quarter * 32 + lane;
         uint8_t* patches = smem + Lo::kPatch + ew * Lo::kPatchBufs * Lo::kPatchBytes;
+        const uint32_t pair_lane = smem_u32(s_pair) + 4u * lane;   // this lane's copy of the pair table
         int pcount = 0;                                    // tensor stores issued by this warp
         float nrm_next = 0.f;
 
@@ -761,7 +769,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
                     const uint32_t key = get_bits<2 * BITS>(w, (c * 8 + 2 * p) * BITS);
-                    h[p] = Lo::kReplPairs ? s_pair[key * 32 + lane] : s_pair[key];
+                    h[p] = Lo::kReplPairs ? lds_u32(pair_lane + key * 128u) : s_pair[key];
                 }
                 const int col = c0 + c * 8;
                 *reinterpret_cast<uint4*>(as + (col >> 6) * C::kTileBlockBytes + sw128_offset(r, (col & 63) >> 3)) =

@@ -212,6 +212,14 @@ __device__ __forceinline__ void put_field(uint32_t (&w)[NW], int j, uint32_t v) 
     if (sh + BITS > 32) w[wi + 1] |= v >> (32 - sh);
 }
 
+// 32-bit load from a shared-space address (no memory clobber: callers order it after the barrier or wait
+// that made the data visible, through the address's data dependence).
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
 // Add value v (< 2^BITS) into field j of the zero-initialised bitstream `w` (fields do not overlap, so this is
 // the same as OR-ing it in, as a shift-add).
 template <int BITS, int NW>

@@ -116,21 +116,23 @@ struct tq_codec {
     uint64_t seed = 0;
     __half* pi_op = nullptr;        // d x d, rotated = Pi_op x
     __half* pi_op_t = nullptr;      // Pi_op^T, the decode-side B operand
-    uint32_t* enc_lut = nullptr;    // 2048 grid cells: boundary bits | count below (low 4 bits)
+    uint32_t* enc_lut = nullptr;    // kGridCells grid cells: boundary bits | count below (low 4 bits)
     uint32_t* pair_lut = nullptr;   // 2^(2 bits) half2 pairs
     CUtensorMap tmap_pi, tmap_pit;
 };
 
 namespace {
 
-// Grid table of the encode search (see encode_k_kernel): cell c holds the y with rint(512 y + 640) = c.
-// Entry = bits of the one boundary inside the cell (+inf if none) OR the count of boundaries below the
-// cell; the boundaries, midpoints of fp16 levels, have at least 4 zero low bits in fp32 (checked).
+// Grid table of the encode search (see encode_k_kernel): cell c holds the y with rint(64 y + 128) = c, so the
+// 256 cells cover y in [-2, 2) (|y| <= ||Pi_op|| < 1.01).  Entry = bits of the one boundary inside the cell
+// (+inf if none) OR the count of boundaries below the cell; the boundaries, midpoints of fp16 levels, have at
+// least 4 zero low bits in fp32 (checked), and no cell holds two of them for any supported d and bits
+// (checked: the closest pair, d = 256 at 4 bits, is 0.016 apart, above the 1/64 cell width).
 tq_status build_grid_lut(int bits, const float* t, std::vector<uint32_t>& lut) {
     const int nb = (1 << bits) - 1;
-    lut.assign(2048, 0x7F800000u | static_cast<uint32_t>(nb));
-    for (int c = 0; c <= 1280; ++c) {
-        const double lo = (c - 640.5) / 512.0, hi = (c - 639.5) / 512.0;
+    lut.assign(kGridCells, 0);
+    for (int c = 0; c < kGridCells; ++c) {
+        const double lo = (c - kGridOffset - 0.5) / kGridRes, hi = (c - kGridOffset + 0.5) / kGridRes;
         uint32_t below = 0;
         int inside = 0;
         float b = INFINITY;
@@ -186,12 +188,12 @@ extern "C" tq_status tq_codec_create(int d, int k_bits, uint64_t seed, tq_codec*
         return s;
     };
     if (cudaMalloc(&c->pi_op, dd * 2) != cudaSuccess || cudaMalloc(&c->pi_op_t, dd * 2) != cudaSuccess ||
-        cudaMalloc(&c->enc_lut, 2048 * sizeof(uint32_t)) != cudaSuccess ||
+        cudaMalloc(&c->enc_lut, kGridCells * sizeof(uint32_t)) != cudaSuccess ||
         cudaMalloc(&c->pair_lut, pairs.size() * 4) != cudaSuccess)
         return cleanup(fail(TQ_ERR_CUDA, "tq_codec_create: cudaMalloc failed"));
     if (cudaMemcpy(c->pi_op, pi16.data(), dd * 2, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(c->pi_op_t, pit16.data(), dd * 2, cudaMemcpyHostToDevice) != cudaSuccess ||
-        cudaMemcpy(c->enc_lut, lut.data(), 2048 * sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->enc_lut, lut.data(), kGridCells * sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(c->pair_lut, pairs.data(), pairs.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
         return cleanup(fail(TQ_ERR_CUDA, "tq_codec_create: cudaMemcpy failed"));
     if ((st = make_tmap_f16(&c->tmap_pi, c->pi_op, d, d, d, d)) != TQ_OK) return cleanup(st);
