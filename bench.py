@@ -283,7 +283,7 @@ def gpu_arm(args, w, rank, world, local_rank):
         raise RuntimeError("a kernel raised the device error flag during timing")
     # kernels per call: one each for the codec calls; attention = query preparation + split kernel
     # (+ the split merge when the workspace holds split-K partials beyond the query fragments)
-    qfrag_bytes = b * hkv * ((d // 16) * 32 + 1) * 16
+    qfrag_bytes = b * hkv * ((d // 16) * 32 + 2) * 16
     per_call = {"attend": 3 if ws.numel() > qfrag_bytes else 2}
     launches = sum(per_call.get(name, 1) for name, _, _ in events)
     return dict(per=per, ms_per_step=ms_per_step, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, n=n,

@@ -209,7 +209,7 @@ typedef struct tq_attend_args {
 
 /*
  * tq_attend_workspace_bytes -- bytes of workspace tq_attend_decode needs for these arguments on the current
- * device: (head_dim / 16 * 32 + 1) * 16 bytes per (sequence, kv head) for the prepared query, plus the split-K
+ * device: (head_dim / 16 * 32 + 2) * 16 bytes per (sequence, kv head) for the prepared query, plus the split-K
  * partials when the sequence axis is split.  Only the shape fields of args are read.
  * Errors: the same argument checks as tq_attend_decode (TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED).
  */

@@ -37,13 +37,13 @@ struct AttendParams {
     const __half* v_zeros;
     float* out;
     float* partials;                                 // [B][H_kv][splits][16 + 8 d]
-    uint4* qfrag;                                    // [B][H_kv][d/16 * 32 + 1]: score A fragments, 1 / prescale
+    uint4* qfrag;                                    // [B][H_kv][d/16 * 32 + 2]: score A fragments, 1 / prescale
     int num_splits;
 };
 
-// uint4 slots per (sequence, kv head) of the query-fragment array
+// uint4 slots per (sequence, kv head) of the query-fragment array: the fragments, then 1 / prescale of 8 heads
 template <int D>
-__host__ __device__ constexpr int qfrag_slots() { return (D / 16) * 32 + 1; }
+__host__ __device__ constexpr int qfrag_slots() { return (D / 16) * 32 + 2; }
 
 template <int D, int KB, int VB, int VG>
 struct AttCfg {
@@ -202,82 +202,76 @@ __device__ __forceinline__ uint32_t vfield(const uint8_t* row, int sl, int gid) 
     }
 }
 
-// Query preparation for one (kv head, sequence): the rotated query q_rot[g] = Pi_op q[g] of each of the
-// group's heads, scaled by softmax scale * log2(e) and a power-of-two prescale, split into fp16 hi/lo halves and
-// laid out as the score A fragments (rows gid = hi, gid + 8 = lo); slot d/16 * 32 holds 1 / prescale.
-// Done once per (kv head, sequence) instead of once per split; the attention grid is its programmatic dependent.
-constexpr int kPrepThreads = 512;
+// Query preparation: the rotated query q_rot[g] = Pi_op q[g] of each of the group's heads, scaled by softmax
+// scale * log2(e) and a per-head power-of-two prescale, split into fp16 hi/lo halves and laid out as the score A
+// fragments (rows gid = hi, gid + 8 = lo); slots d/16 * 32 and + 1 hold 1 / prescale of heads 0..7.
+// The prescale comes from a bound, |q_rot_j| <= ||Pi_op|| ||q|| < 1.0625 ||q||, so max |x * pre| < 2^15 and
+// no reduction over q_rot is needed: CTA x of grid (d / 32, H_kv, B) computes n-tiles 4x .. 4x + 3 (one per
+// warp) and writes their fragments straight from the MMA accumulators.  The attention grid is its
+// programmatic dependent.
+constexpr int kPrepThreads = 128;
 
 template <int D>
-__global__ void __launch_bounds__(kPrepThreads, 1) attend_prep_kernel(const AttendParams p) {
+__global__ void __launch_bounds__(kPrepThreads) attend_prep_kernel(const AttendParams p) {
     constexpr int KS = D / 16;
-    constexpr int kWarps = kPrepThreads / 32;            // one n-tile of q_rot per warp (two at d = 256)
-    __shared__ float s_qr[8 * D];
-    __shared__ float s_red[kWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;
-    const int h = blockIdx.x, b = blockIdx.y;
+    const int nt = blockIdx.x * (kPrepThreads / 32) + warp;      // n-tile: columns 8 nt .. 8 nt + 7
+    const int h = blockIdx.y, b = blockIdx.z;
     const int G = p.group;
     uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();
     // the attention grid may be scheduled at once and start streaming the cache; its consumers wait for this
     // grid's completion (griddepcontrol.wait) before they read the fragments
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    // q_rot[g][n] = sum_k q[g][k] Pi_op[n][k] on the tensor cores (fp16 inputs are exact products)
     const __half* qg = p.q + (static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * G) * D;
-    for (int nt = warp; nt < D / 8; nt += kWarps) {
-        // every fragment of this n-tile is loaded before the first MMA, so the loads overlap
-        uint32_t bf[KS][2], af[KS][2];
-        const __half* prow = p.pi_op + (8 * nt + gid) * D + 2 * tig;
+    // every fragment is loaded before the first MMA, so the loads overlap
+    uint32_t bf[KS][2], af[KS][2];
+    const __half* prow = p.pi_op + (8 * nt + gid) * D + 2 * tig;
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            bf[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(prow + 16 * ks));
-            bf[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(prow + 16 * ks + 8));
-            af[ks][0] = (gid < G) ? __ldg(reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig)) : 0u;
-            af[ks][1] = (gid < G) ? __ldg(reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig + 8)) : 0u;
-        }
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) mma_f16(c, make_uint4(af[ks][0], 0u, af[ks][1], 0u), bf[ks][0], bf[ks][1]);
-        s_qr[gid * D + 8 * nt + 2 * tig] = c[0];
-        s_qr[gid * D + 8 * nt + 2 * tig + 1] = c[1];
+    for (int ks = 0; ks < KS; ++ks) {
+        bf[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(prow + 16 * ks));
+        bf[ks][1] = __ldg(reinterpret_cast<const uint32_t*>(prow + 16 * ks + 8));
+        af[ks][0] = (gid < G) ? __ldg(reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig)) : 0u;
+        af[ks][1] = (gid < G) ? __ldg(reinterpret_cast<const uint32_t*>(qg + gid * D + 16 * ks + 2 * tig + 8)) : 0u;
     }
-    __syncthreads();
-    // power-of-two prescale so the fp16 hi/lo halves of the scaled query stay in the normal range
-    float amax = 0.f;
-    for (int i = threadIdx.x; i < G * D; i += 32 * kWarps) amax = fmaxf(amax, fabsf(s_qr[i] * p.scale_log2));
+    // ||q_gid||^2 from the fragments this quad holds (lane tig: coordinates 16 ks + 2 tig + {0, 1, 8, 9})
+    float ss = 0.f;
 #pragma unroll
-    for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (lane == 0) s_red[warp] = amax;
-    __syncthreads();
-    amax = s_red[0];
+    for (int ks = 0; ks < KS; ++ks) {
 #pragma unroll
-    for (int w = 1; w < kWarps; ++w) amax = fmaxf(amax, s_red[w]);
-    // amax = m 2^ex with m in [0.5, 1) (read from the exponent field; clamped for tiny or zero queries)
-    int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 255u) - 126;
-    ex = (amax > 0.f) ? max(ex, -100) : 14;
-    const float pre = __uint_as_float(static_cast<uint32_t>(127 + 14 - ex) << 23);   // max |q| * pre in [8192, 16384)
-    // score A fragments, coordinate-permuted so lane tig owns coords [tig*D/4, (tig+1)*D/4):
-    // k-slots (2tig, 2tig+1, 2tig+8, 2tig+9) of k-step ks <- coords tig*D/4 + 4ks + (0, 1, 2, 3)
-    for (int i = threadIdx.x; i < KS * 32; i += 32 * kWarps) {
-        const int ks = i >> 5, ln = i & 31, g = ln >> 2, tg = ln & 3;
-        const int cc = tg * (D / 4) + 4 * ks;
-        uint4 f = make_uint4(0u, 0u, 0u, 0u);
-        if (g < G) {
-            float x[4], hi[4], lo[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                x[e] = s_qr[g * D + cc + e] * p.scale_log2 * pre;
-                hi[e] = __half2float(__float2half_rn(x[e]));
-                lo[e] = x[e] - hi[e];
-            }
-            f.x = pack_f16(hi[0], hi[1]);
-            f.y = pack_f16(lo[0], lo[1]);
-            f.z = pack_f16(hi[2], hi[3]);
-            f.w = pack_f16(lo[2], lo[3]);
+        for (int j = 0; j < 2; ++j) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&af[ks][j]));
+            ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
         }
-        qf[i] = f;
     }
-    if (threadIdx.x == 0) qf[KS * 32] = make_uint4(__float_as_uint(1.0f / pre), 0u, 0u, 0u);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    const float bound = sqrtf(ss) * fabsf(p.scale_log2) * 1.0625f;
+    // bound = m 2^ex with m in [0.5, 1); pre = 2^(14 - ex), so |x| * pre < 2^15 (zero or tiny queries clamped)
+    int ex = static_cast<int>((__float_as_uint(bound) >> 23) & 255u) - 126;
+    ex = (bound > 0.f) ? max(ex, -100) : 14;
+    const float pre = __uint_as_float(static_cast<uint32_t>(127 + 14 - ex) << 23);
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) mma_f16(c, make_uint4(af[ks][0], 0u, af[ks][1], 0u), bf[ks][0], bf[ks][1]);
+    // c0, c1 = q_rot[gid][8 nt + 2 tig + {0, 1}]; the fragment of (head gid, k-step ks) holds coordinates
+    // tg * D/4 + 4 ks + (0..3), so columns 8 nt .. + 3 and + 4 .. + 7 are two whole fragments: lanes tig = 0, 2
+    // assemble them with the halves of lanes tig = 1, 3
+    float hi[2], lo[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const float x = c[e] * p.scale_log2 * pre;
+        hi[e] = __half2float(__float2half_rn(x));
+        lo[e] = x - hi[e];
+    }
+    const uint32_t h01 = pack_f16(hi[0], hi[1]), l01 = pack_f16(lo[0], lo[1]);
+    const uint32_t h23 = __shfl_down_sync(0xffffffffu, h01, 1), l23 = __shfl_down_sync(0xffffffffu, l01, 1);
+    if ((tig & 1) == 0) {
+        const int col = 8 * nt + 2 * tig;                         // first of this fragment's four coordinates
+        const int tg = col / (D / 4), ks = (col % (D / 4)) / 4;
+        qf[ks * 32 + gid * 4 + tg] = make_uint4(h01, l01, h23, l23);
+    }
+    if (blockIdx.x == 0 && warp == 0 && tig == 0) reinterpret_cast<float*>(qf + KS * 32)[gid] = 1.0f / pre;
 }
 
 // Fused decode attention for one (split, kv head, sequence).  Per 16-token chunk and warp:
@@ -370,7 +364,7 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         // written by attend_prep_kernel, the grid this one depends on programmatically
         asm volatile("griddepcontrol.wait;" ::: "memory");
         const uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();
-        const float unpre = __uint_as_float(__ldcg(&qf[KS * 32].x));
+        const float unpre = __ldcg(reinterpret_cast<const float*>(qf + KS * 32) + gid);   // head gid's
         if constexpr (!C::kQInRegs) {
             for (int i = threadIdx.x; i < KS * 32; i += 32 * C::kWarps) s_qf[i] = __ldcg(qf + i);
             named_bar_sync(1, 32 * C::kWarps);
@@ -610,7 +604,7 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
 // One CTA per (g, h, b).  Slice k of the CTA's threads (D threads, one per column) folds splits k, k + kSlices,
 // ... with every load issued before the first is used, so the partials cost one round trip; the slices are
 // then combined in shared memory the same way.
-constexpr int kMergeThreads = 512;
+constexpr int kMergeThreads = 1024;
 constexpr int kMaxSplits = 256;
 
 template <int D>
@@ -618,7 +612,7 @@ __global__ void __launch_bounds__(kMergeThreads) attend_merge_kernel(const Atten
     asm volatile("griddepcontrol.wait;" ::: "memory");
     constexpr int kPart = 16 + 8 * D;
     constexpr int kSlices = kMergeThreads / D;
-    constexpr int kBatch = 16;                           // splits per slice per round of loads
+    constexpr int kBatch = 12;                           // splits per slice per round of loads
     __shared__ float s_o[kSlices][D];
     __shared__ float s_ml[kSlices][2];
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;

@@ -830,8 +830,11 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
                             uint32_t hw[4];
 #pragma unroll
                             for (int k = 0; k < 4; ++k) {
-                                __half2 h2 = __floats2half2_rn(__uint_as_float(v[8 * pc + 2 * k]) * nrm,
-                                                               __uint_as_float(v[8 * pc + 2 * k + 1]) * nrm);
+                                // two elements per packed f32x2 multiply, then one paired conversion
+                                const float2 y2 = __fmul2_rn(make_float2(__uint_as_float(v[8 * pc + 2 * k]),
+                                                                         __uint_as_float(v[8 * pc + 2 * k + 1])),
+                                                             make_float2(nrm, nrm));
+                                __half2 h2 = __floats2half2_rn(y2.x, y2.y);
                                 hw[k] = *reinterpret_cast<uint32_t*>(&h2);
                             }
                             pk = make_uint4(hw[0], hw[1], hw[2], hw[3]);

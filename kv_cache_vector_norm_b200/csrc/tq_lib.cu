@@ -458,7 +458,7 @@ tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan) {
     if (splits < 1) splits = 1;
     plan->num_splits = static_cast<int>(splits);
     plan->partial_bytes = (splits > 1) ? static_cast<size_t>(bh) * splits * (16 + 8 * a->head_dim) * 4 : 0;
-    plan->qfrag_bytes = static_cast<size_t>(bh) * ((a->head_dim / 16) * 32 + 1) * 16;
+    plan->qfrag_bytes = static_cast<size_t>(bh) * ((a->head_dim / 16) * 32 + 2) * 16;
     plan->workspace_bytes = plan->qfrag_bytes + plan->partial_bytes;
     return TQ_OK;
 }
@@ -492,7 +492,7 @@ tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const Attend
     p.qfrag = static_cast<uint4*>(a->workspace);
     p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(a->workspace) + plan.qfrag_bytes);
     p.num_splits = plan.num_splits;
-    attend_prep_kernel<D><<<dim3(a->num_kv_heads, a->batch), kPrepThreads, 0, st>>>(p);
+    attend_prep_kernel<D><<<dim3(D / 32, a->num_kv_heads, a->batch), kPrepThreads, 0, st>>>(p);
     TQ_CUDA(cudaGetLastError(), "tq_attend_decode: query preparation launch");
     // the attention grid and the split merge are programmatic dependents of the grid before them: each is
     // scheduled while its predecessor drains and waits for it (griddepcontrol.wait) before reading its output

@@ -77,7 +77,7 @@ def test_argument_errors_are_reported():
     assert nb.value > 0                                                     # one sequence: split over the SMs
     a.batch, a.num_kv_heads, a.max_seq_len = 3, 2, 16                       # one chunk per sequence: one split
     assert tq.LIB.tq_attend_workspace_bytes(ctypes.byref(a), ctypes.byref(nb)) == tq.TQ_OK
-    assert nb.value == 3 * 2 * (128 // 16 * 32 + 1) * 16                   # only the prepared query fragments
+    assert nb.value == 3 * 2 * (128 // 16 * 32 + 2) * 16                   # only the prepared query fragments
     assert tq.LIB.tq_attend_decode(None, ctypes.byref(a), None) == tq.TQ_ERR_INVALID_ARG
     assert tq.LIB.tq_codec_create(96, 4, 0, ctypes.byref(ctypes.c_void_p())) == tq.TQ_ERR_UNSUPPORTED
     assert tq.LIB.tq_codec_create(128, 5, 0, ctypes.byref(ctypes.c_void_p())) == tq.TQ_ERR_UNSUPPORTED
