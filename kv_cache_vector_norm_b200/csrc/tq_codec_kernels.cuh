@@ -17,12 +17,30 @@ constexpr int kGridCells = 256;
 // min/max with shuffles.  Every arithmetic step is the page's fp32 operation with one rounding.
 
 // Codes of a group: round_half_even(a / s) with the page's IEEE fp32 division, 0 <= a <= (2^b - 1) s.
-// With r = RN(1/s), the products a RN(r (1 -+ 2^-21)) bracket RN(a / s) (each end is off by at most
-// 3 * 2^-23 relative, inside the 2^-21 bracket); an FMA adding 1.5 * 2^23 rounds each end to the nearest
-// integer (ties to even) in its low mantissa bits.  Rounding is monotonic, so when both ends give the same
-// integer, RN(a / s) rounds to it as well; otherwise the caller recomputes with the exact quotient.
+// With r an approximate reciprocal of s (relative error <= 2^-21; the hardware's is about 2^-23), the
+// products a RN(r (1 -+ 2^-20)) bracket both a / s and RN(a / s): each end lies at least 2^-21 (a/s) away
+// from a / s on its side, beyond the half ulp (<= 2^-24 (a/s)) that separates a / s from RN(a / s).  An FMA
+// adding 1.5 * 2^23 rounds each end to the nearest integer (ties to even) in its low mantissa bits.  Rounding
+// is monotonic, so when both ends give the same integer, RN(a / s) rounds to it as well; otherwise the caller
+// recomputes with the exact quotient.
 constexpr float kCodeMagic = 12582912.0f;                   // 1.5 * 2^23
 constexpr uint32_t kCodeMagicBits = 0x4B400000u;
+
+// RN(x / L) for x >= 0 and L in {3, 7, 15, 255}: q = RN(x RN(1/L)), then one FMA correction with the exact
+// residual x - q L.  Checked exhaustively against IEEE division for every non-negative finite fp32 x and each
+// of the four L (all 2^31 - 2^23 values, on the host with hardware FMA).
+template <int L>
+__device__ __forceinline__ float div_by_levels(float x) {
+    constexpr float y = 1.0f / static_cast<float>(L);
+    const float q = __fmul_rn(x, y);
+    return __fmaf_rn(__fmaf_rn(-q, static_cast<float>(L), x), y, q);
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
 
 // One lane owns 16 consecutive elements of a row (32 bytes of fp16), so a group of 32 spans 2 lanes (or d/16
 // lanes in the per-token layout), the per-group division and reciprocal of the encoder are shared by 16
@@ -93,12 +111,12 @@ __global__ void __launch_bounds__(256) encode_v_kernel(const __half* __restrict_
             vmin = fminf(vmin, __shfl_xor_sync(0xffffffffu, vmin, off));
             vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
         }
-        float scale = __fdiv_rn(__fsub_rn(vmax, vmin), static_cast<float>(kLevels));
-        scale = fmaxf(scale, 1e-12f);
+        float scale = div_by_levels<static_cast<int>(kLevels)>(__fsub_rn(vmax, vmin));   // = IEEE (max - min) / L
+        scale = fmaxf(scale, 1e-12f);                                 // a normal number from here on
         const float zero = vmin;
-        const float rcp = __frcp_rn(scale);
-        const float r_lo = __fmul_rn(rcp, 0.99999952316284180f);   // 1 - 2^-21
-        const float r_hi = __fmul_rn(rcp, 1.00000047683715820f);   // 1 + 2^-21
+        const float rcp = rcp_approx(scale);
+        const float r_lo = __fmul_rn(rcp, 0.99999904632568359375f);   // 1 - 2^-20
+        const float r_hi = __fmul_rn(rcp, 1.00000095367431640625f);   // 1 + 2^-20
         uint32_t chunk[kW];
 #pragma unroll
         for (int k = 0; k < kW; ++k) chunk[k] = 0u;
@@ -504,6 +522,11 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
             if (staged && !mbar_wait(b_pkempty + 8 * pb, ((li >> 1) & 1) ^ 1, abort_flag)) break;
 #pragma unroll
             for (int k = 0; k < E::kChunks; ++k) {
+                uint32_t w[BITS];
+#pragma unroll
+                for (int i = 0; i < BITS; ++i) w[i] = 0u;
+                const float2 inv2 = make_float2(inv, inv);
+                const float2 gs2 = make_float2(kGridScale, kGridScale), gm2 = make_float2(kGridMagic, kGridMagic);
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(taddr + k * 32, v);
                 tmem_ld_wait();
@@ -512,11 +535,6 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(b_accempty + 8 * a);   // TMEM buffer a is free for tile li + 2
                 }
-                uint32_t w[BITS];
-#pragma unroll
-                for (int i = 0; i < BITS; ++i) w[i] = 0u;
-                const float2 inv2 = make_float2(inv, inv);
-                const float2 gs2 = make_float2(kGridScale, kGridScale), gm2 = make_float2(kGridMagic, kGridMagic);
 #pragma unroll
                 for (int j2 = 0; j2 < 16; ++j2) {
                     // two coordinates per packed f32x2 multiply and FMA
