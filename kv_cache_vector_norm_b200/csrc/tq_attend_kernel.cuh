@@ -436,10 +436,17 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                 const int valid = (rem < 16) ? static_cast<int>(rem) : 16;
                 float lg[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int nt = e >> 1, k = e & 1;
-                    const float raw = (sc[nt][k] + sc[nt][k + 2]) * unpre * nrm[tok[e]];
-                    lg[e] = (tok[e] < valid) ? raw : -INFINITY;
+                for (int nt = 0; nt < 2; ++nt) {
+                    // tokens 8 nt + 2 tig, + 1: (hi row + lo row) * unpre * n_t, two per packed f32x2 operation
+                    const float2 sum = __fadd2_rn(make_float2(sc[nt][0], sc[nt][1]), make_float2(sc[nt][2], sc[nt][3]));
+                    const float2 nn = __fmul2_rn(make_float2(nrm[tok[2 * nt]], nrm[tok[2 * nt + 1]]), make_float2(unpre, unpre));
+                    const float2 raw = __fmul2_rn(sum, nn);
+                    lg[2 * nt] = raw.x;
+                    lg[2 * nt + 1] = raw.y;
+                }
+                if (valid < 16) {                                  // the sequence's last, partial chunk
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) lg[e] = (tok[e] < valid) ? lg[e] : -INFINITY;
                 }
                 float mt = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
                 mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
@@ -449,8 +456,11 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                 // probabilities carry the factor 2^kPExp (so do l_run and zacc; removed at the end)
                 const float m_off = m_use - static_cast<float>(kPExp);
                 float pr[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) pr[e] = ex2(lg[e] - m_off);
+                {
+                    const float2 a01 = __fadd2_rn(make_float2(lg[0], lg[1]), make_float2(-m_off, -m_off));
+                    const float2 a23 = __fadd2_rn(make_float2(lg[2], lg[3]), make_float2(-m_off, -m_off));
+                    pr[0] = ex2(a01.x); pr[1] = ex2(a01.y); pr[2] = ex2(a23.x); pr[3] = ex2(a23.y);
+                }
                 if (__any_sync(0xffffffffu, m_new != m_run)) {     // some head's running max moved
                     const float corr = ex2(m_run - m_use);
                     // the accumulator columns are heads 2tig and 2tig+1: their factors sit in lanes 8tig, 8tig+4
