@@ -82,21 +82,33 @@ __global__ void __launch_bounds__(256) encode_v_kernel(const __half* __restrict_
     const int j = lane % L::kRowLanes;                            // 16-element chunk index within the row
     const int gl = j % L::kGroupLanes;                            // lane index within the scale group
     const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
-    for (int64_t wrow = (static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5)) * L::kRowsPerWarp;
-         wrow < n; wrow += warps_total * L::kRowsPerWarp) {
+    const int64_t step = warps_total * L::kRowsPerWarp;
+    // this lane's 16 inputs of row r (zeros past n); the next row's are loaded before the current one is encoded
+    auto load = [&](int64_t r, uint4& w0, uint4& w1) {
+        if (r < n) {
+            const uint4* src = reinterpret_cast<const uint4*>(x + r * stride) + 2 * j;
+            w0 = __ldg(src);
+            w1 = __ldg(src + 1);
+        } else {
+            w0 = w1 = make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    int64_t wrow = (static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5)) * L::kRowsPerWarp;
+    uint4 c0, c1;
+    load(wrow + lane / L::kRowLanes, c0, c1);
+    for (; wrow < n; wrow += step) {
         const int64_t row = wrow + lane / L::kRowLanes;
         const bool valid = row < n;
+        uint4 n0, n1;
+        load(row + step, n0, n1);
         __half2 hv[8];
-        if (valid) {
-            const uint4* src = reinterpret_cast<const uint4*>(x + row * stride) + 2 * j;
-            const uint4 w0 = __ldg(src), w1 = __ldg(src + 1);
-            const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        {
+            const uint32_t u[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
             for (int k = 0; k < 8; ++k) hv[k] = *reinterpret_cast<const __half2*>(&u[k]);
-        } else {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) hv[k] = __floats2half2_rn(0.f, 0.f);
         }
+        c0 = n0;
+        c1 = n1;
         // min / max on packed halves (exact; fp16 -> fp32 is exact afterwards)
         __half2 mn2 = __hmin2(hv[0], hv[1]), mx2 = __hmax2(hv[0], hv[1]);
 #pragma unroll
