@@ -315,7 +315,6 @@ struct KeyCfg {
     static constexpr int kPiBlockBytes = D * 128;            // one 64-column block of the d x d matrix
     static constexpr int kEncStages = (D == 256) ? 1 : (D == 128 ? 4 : 6);
     static constexpr int kDecBufs = (D == 256) ? 1 : 2;
-    static constexpr int kDecInBufs = (D == 256) ? 1 : 2;    // packed-row staging buffers (decode)
     static constexpr int kEpiWarps = 8;
     static constexpr int kThreads = 32 * (2 + kEpiWarps);
     static constexpr int kTmemCols = 2 * D;                  // two accumulator buffers
@@ -619,19 +618,21 @@ struct DecLayout {
     using E = DecCfg<D>;
     static constexpr int kRowBytes = D * BITS / 8;
     static constexpr int kInBytes = 128 * kRowBytes + 128 * 4;            // packed rows + norms
+    // staging buffers for the packed rows: the producer runs up to kInBufs - 1 tiles ahead of the builders
+    static constexpr int kInBufs = (D == 256) ? 1 : ((D == 128 && BITS == 4) ? 3 : 4);
     // code-pair table: one copy per shared-memory bank (entry e of lane l at 128 e + 4 l) where it fits
     static constexpr bool kReplPairs = (D <= 128);
     static constexpr int kPairBytes = (1 << (2 * BITS)) * (kReplPairs ? 128 : 4);
     static constexpr uint32_t kPit = 0;
     static constexpr uint32_t kA = kPit + C::kPiBytes;
     static constexpr uint32_t kIn = kA + C::kDecBufs * C::kTileBytes;
-    static constexpr uint32_t kPair = kIn + C::kDecInBufs * kInBytes;
+    static constexpr uint32_t kPair = kIn + kInBufs * kInBytes;
     // per-warp output patches: 32 rows x 64 bytes, 64B-swizzled, the source of one tensor store each
     static constexpr int kPatchBufs = (D <= 128) ? 2 : 1;
     static constexpr uint32_t kPatchBytes = 32 * 64;
     static constexpr uint32_t kPatch = (kPair + kPairBytes + 511) & ~511u;     // 64B swizzle repeats every 512 bytes
     static constexpr uint32_t kBar = kPatch + E::kEpiWarps * kPatchBufs * kPatchBytes;
-    static constexpr int kBars = 2 * C::kDecBufs + 2 * C::kDecInBufs + 8;
+    static constexpr int kBars = 2 * C::kDecBufs + 2 * kInBufs + 8;
     static constexpr uint32_t kMisc = kBar + 8 * kBars;
     static constexpr uint32_t kBytes = kMisc + 16 + 1024;
     static_assert(kBytes <= 227 * 1024, "decode layout exceeds the shared memory of one CTA");
@@ -651,7 +652,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
     using E = DecCfg<D>;
     using Lo = DecLayout<D, BITS>;
     constexpr int NB = C::kDecBufs;
-    constexpr int NI = C::kDecInBufs;
+    constexpr int NI = Lo::kInBufs;
     constexpr int kRowBytes = Lo::kRowBytes;
     constexpr int kPartWords = E::kCols * BITS / 32;   // 32-bit words of this warp's columns of a packed row
     constexpr int kPairs = 1 << (2 * BITS);
