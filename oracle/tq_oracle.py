@@ -107,13 +107,49 @@ def to_fp16_values(a: np.ndarray) -> np.ndarray:
     return np.asarray(a, dtype=np.float64).astype(np.float16).astype(np.float64)
 
 
-def operational_rotation(d: int, seed: int) -> np.ndarray:
+def sylvester_hadamard(d: int) -> np.ndarray:
+    """The d x d Walsh-Hadamard matrix of +-1 entries (d a power of two) by Sylvester's doubling:
+    H_1 = [1], H_2m = [[H_m, H_m], [H_m, -H_m]]."""
+    if d < 1 or d & (d - 1):
+        raise ValueError(f"d={d} is not a power of two")
+    h = np.ones((1, 1), dtype=np.float64)
+    while h.shape[0] < d:
+        h = np.block([[h, h], [h, -h]])
+    return h
+
+
+def hadamard_signs(d: int, seed: int) -> np.ndarray:
+    """Seeded signs s_j = -1 if the top bit of SplitMix64(seed) output j is set, else +1."""
+    top = (splitmix64(seed, d) >> _U64(63)).astype(np.int64)
+    return 1.0 - 2.0 * top
+
+
+def hadamard_rotation(d: int, seed: int) -> np.ndarray:
+    """The randomized Walsh-Hadamard rotation Pi = H diag(s) / sqrt(d) (d x d, fp64): rotated = Pi @ x.
+
+    [P4] "turbo-attn", The codec, "Hadamard rotation": a Walsh-Hadamard transform spreads outlier channels
+    over the vector, and queries are rotated the same way.  Reading: the page fixes neither the signs nor
+    the scale; this build takes the usual randomized, orthonormal form -- seeded signs (so the coordinates
+    of a rotated isotropic vector follow the same marginal and the same data-independent codebook
+    applies) and 1/sqrt(d) (so Pi is orthogonal and norms are kept).
+    """
+    return sylvester_hadamard(d) * hadamard_signs(d, seed)[None, :] / math.sqrt(d)
+
+
+ROTATIONS = ("haar", "hadamard")
+
+
+def operational_rotation(d: int, seed: int, kind: str = "haar") -> np.ndarray:
     """Pi_op = fp16(Pi): the rotation the tensor-core path multiplies by (values as fp64).
 
     Reading: the pages keep Pi in fp32; this build rounds it once to fp16 so that fp16 inputs times
     Pi_op are exact products in an fp32 accumulator, and states the deviation separately.
     """
-    return to_fp16_values(haar_rotation(d, seed))
+    if kind == "haar":
+        return to_fp16_values(haar_rotation(d, seed))
+    if kind == "hadamard":
+        return to_fp16_values(hadamard_rotation(d, seed))
+    raise ValueError(f"unknown rotation {kind!r}")
 
 
 # ----------------------------------------------------------------------------------------------

@@ -76,3 +76,48 @@ def test_operational_rotation_deviation(d):
     # entries are O(1/sqrt d); fp16 relative rounding is 2^-11, so Pi_op^T Pi_op stays within 2e-3 of I
     assert np.max(np.abs(op.T @ op - np.eye(d))) < 2e-3
     assert np.max(np.abs(op - pi)) <= 2.0 ** -11 * np.max(np.abs(pi))
+
+
+# ---- randomized Walsh-Hadamard rotation ("turbo-attn", The codec, "Hadamard rotation")
+
+@pytest.mark.parametrize("d", [2, 4, 64, 128, 256])
+def test_sylvester_hadamard_is_the_library_hadamard(d):
+    from scipy import linalg
+    assert np.array_equal(o.sylvester_hadamard(d), linalg.hadamard(d).astype(np.float64))
+
+
+def _fwht(v: np.ndarray) -> np.ndarray:
+    """Fast Walsh-Hadamard transform by butterflies (pairs (a + b, a - b) at strides 1, 2, 4, ...), the
+    O(d log d) algorithm, independent of the matrix construction."""
+    v = np.array(v, dtype=np.float64)
+    h = 1
+    while h < v.shape[-1]:
+        a = v.reshape(*v.shape[:-1], -1, 2, h)
+        v = np.concatenate([a[..., 0, :] + a[..., 1, :], a[..., 0, :] - a[..., 1, :]], axis=-1).reshape(v.shape)
+        h *= 2
+    return v
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_hadamard_rotation_is_orthogonal_and_is_the_fast_transform(d):
+    pi = o.hadamard_rotation(d, 5)
+    assert np.abs(pi @ pi.T - np.eye(d)).max() < 1e-14
+    x = np.random.default_rng(0).standard_normal((16, d))
+    s = o.hadamard_signs(d, 5)
+    assert np.abs(x @ pi.T - _fwht(x * s) / math.sqrt(d)).max() < 1e-12
+    assert set(np.unique(s)) == {-1.0, 1.0}
+    assert abs(int((s < 0).sum()) - d / 2) < 4 * math.sqrt(d)     # fair signs
+    assert not np.array_equal(s, o.hadamard_signs(d, 6))
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_hadamard_rotation_keeps_the_codebook_distortion(bits):
+    # an orthogonal map sends an isotropic Gaussian to an isotropic Gaussian, so the rotated unit vector is
+    # uniform on the sphere and the measured distortion is the codebook's D(b, d)
+    d, n = 128, 20000
+    pi = o.operational_rotation(d, 9, "hadamard")
+    c, t = o.operational_codebook(d, bits)
+    x = o.to_fp16_values(np.random.default_rng(bits).standard_normal((n, d)))
+    idx, nrm, y = o.encode_k(x, pi, t)
+    measured = float(np.mean(np.sum((y - c[idx]) ** 2, axis=1)))
+    assert abs(measured - o.sphere_distortion(d, c, t)) <= 0.02 * o.sphere_distortion(d, c, t)
