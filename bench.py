@@ -176,7 +176,7 @@ def gpu_arm(args, w, rank, world, local_rank):
     k = synth.kv_tensor(seed, synth.STREAM_K, b, hkv, t, d, device=dev, scales=ks).view(n, d)
     v = synth.kv_tensor(seed, synth.STREAM_V, b, hkv, t, d, device=dev, scales=vs).view(n, d)
     q = synth.normal_fp16(seed, synth.STREAM_Q, (b, hq, d), device=dev)
-    codec = tq.Codec(d, kb, 0)
+    codec = tq.Codec(d, kb, 0, rotation=args.rotation)
     kp = torch.empty(n, d * kb // 8, dtype=torch.uint8, device=dev)
     kn = torch.empty(n, dtype=torch.float32, device=dev)
     vd = torch.empty(n, (d * vb + 7) // 8, dtype=torch.uint8, device=dev)
@@ -355,6 +355,8 @@ def main():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--workload", default="70b_decode_128k", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rotation", default="haar", choices=["haar", "hadamard"],
+                    help="key rotation: seeded Haar (default) or randomized Walsh-Hadamard; same kernels")
     ap.add_argument("--only", choices=["encode_k", "encode_v", "decode_k", "decode_v", "attend"],
                     help="time one kernel of the path alone (profiling aid; prints its per-launch times)")
     args = ap.parse_args()
@@ -367,7 +369,7 @@ def main():
     bpv = algorithmic_bytes(w)
     config = {"workload": args.workload, "description": w["desc"], "batch": w["batch"], "kv_heads": w["kv_heads"],
               "q_heads": w["q_heads"], "tokens": w["tokens"], "head_dim": w["d"], "k_bits": w["k_bits"],
-              "v_bits": w["v_bits"], "v_group": w["v_group"],
+              "v_bits": w["v_bits"], "v_group": w["v_group"], "rotation": args.rotation,
               "vector": "one (token, kv head) key/value pair through encode + decode + attention",
               "l2": "flushed by a 256 MiB write before every kernel launch (outside the timed interval)",
               "parallelism": f"replicas x{world} (independent caches, no collective on the data path)"}

@@ -76,6 +76,25 @@ int tq_version(void);
  */
 tq_status tq_make_rotation(int d, uint64_t seed, double* pi, uint16_t* pi_f16);
 
+/* Rotation kinds of tq_make_rotation_ex / tq_codec_create_ex. */
+typedef enum tq_rotation {
+    TQ_ROT_HAAR = 0,          /* the seeded Haar rotation of tq_make_rotation */
+    TQ_ROT_HADAMARD = 1       /* the seeded randomized Walsh-Hadamard rotation below */
+} tq_rotation;
+
+/*
+ * tq_make_rotation_ex -- tq_make_rotation for either rotation kind.  TQ_ROT_HADAMARD ("turbo-attn", The
+ * codec, "Hadamard rotation": a Walsh-Hadamard transform spreads outlier channels across the vector and the
+ * queries are rotated the same way) is Pi = H diag(s) / sqrt(d): H the Sylvester Hadamard matrix
+ * (H[i][j] = (-1)^popcount(i & j)), s_j = -1 if the top bit of SplitMix64(seed) output j (0-based) is set,
+ * else +1.  The page fixes neither the signs nor the scale; these make Pi orthogonal and the rotated
+ * coordinates of an isotropic vector follow the same marginal, so the same codebook applies.
+ *   rotation  TQ_ROT_HAAR or TQ_ROT_HADAMARD (then d must be a power of two).
+ * Errors: TQ_ERR_INVALID_ARG for a bad kind, d out of range or not a power of two (Hadamard), or both
+ * outputs NULL.
+ */
+tq_status tq_make_rotation_ex(int d, uint64_t seed, int rotation, double* pi, uint16_t* pi_f16);
+
 /*
  * tq_build_codebook -- data-independent Lloyd-Max levels for one rotated coordinate ("KV Cache API",
  * compressors.py calls _solve_codebook(head_dim, bits), body not shown; "TurboQuant: A KV Cache
@@ -107,6 +126,16 @@ typedef struct tq_codec tq_codec;
  * Errors: TQ_ERR_UNSUPPORTED for other d / bits, TQ_ERR_CUDA if the device allocation fails.
  */
 tq_status tq_codec_create(int d, int k_bits, uint64_t seed, tq_codec** out);
+
+/*
+ * tq_codec_create_ex -- tq_codec_create with the rotation kind (tq_rotation).  Every kernel is the same:
+ * the rotation is a d x d fp16 matrix multiplied on the tensor cores whichever kind it is.
+ * Errors: as tq_codec_create, plus TQ_ERR_INVALID_ARG for an unknown kind.
+ */
+tq_status tq_codec_create_ex(int d, int k_bits, uint64_t seed, int rotation, tq_codec** out);
+
+/* The rotation kind a codec was created with (TQ_ROT_HAAR for tq_codec_create). */
+tq_status tq_codec_rotation(const tq_codec* codec, int* rotation);
 
 /* Free a codec (NULL is accepted).  The caller must ensure no enqueued work still uses it. */
 tq_status tq_codec_destroy(tq_codec* codec);

@@ -1,4 +1,5 @@
-// Host-side parameter builders of libtq: the seeded Haar rotation and the Lloyd-Max codebook.
+// Host-side parameter builders of libtq: the seeded Haar (or Walsh-Hadamard) rotation and the Lloyd-Max
+// codebook.
 //
 // Rotation: "KV Cache API" (TurboQuant docs), compressors.py MSECompressor.__init__ -- a Gaussian d x d
 // matrix G, its QR factorisation, Pi = Q * sign(diag R).  The Gaussian draws come from SplitMix64
@@ -101,6 +102,32 @@ void host_rotation(int d, uint64_t seed, double* pi) {
     // Pi = Q diag(sign(R_jj)), sign(0) := +1
     for (size_t i = 0; i < n; ++i)
         for (size_t j = 0; j < n; ++j) pi[i * n + j] = (rdiag[j] < 0.0 ? -1.0 : 1.0) * q[i * n + j];
+}
+
+// "turbo-attn", The codec, "Hadamard rotation": a Walsh-Hadamard transform spreads outlier channels over the
+// vector; queries are rotated the same way.  H by Sylvester's doubling (H_1 = [1], H_2m = [[H, H], [H, -H]]),
+// i.e. H[i][j] = (-1)^popcount(i & j); columns scaled by the seeded signs and by 1/sqrt(d).
+void host_hadamard(int d, uint64_t seed, double* pi) {
+    const double inv = 1.0 / std::sqrt(static_cast<double>(d));
+    for (int j = 0; j < d; ++j) {
+        const double sj = (splitmix64_at(seed, static_cast<uint64_t>(j)) >> 63) ? -inv : inv;
+        for (int i = 0; i < d; ++i) {
+            const bool odd = __builtin_popcount(static_cast<unsigned>(i & j)) & 1;
+            pi[static_cast<size_t>(i) * d + j] = odd ? -sj : sj;
+        }
+    }
+}
+
+bool host_rotation_of(int kind, int d, uint64_t seed, double* pi) {
+    if (kind == TQ_ROT_HAAR) {
+        host_rotation(d, seed, pi);
+        return true;
+    }
+    if (kind == TQ_ROT_HADAMARD) {
+        host_hadamard(d, seed, pi);
+        return true;
+    }
+    return false;
 }
 
 // ------------------------------------------------------------------------------------------ codebook
@@ -272,18 +299,26 @@ double f16_to_f64(uint16_t h) {
 
 extern "C" const char* tq_last_error(void) { return tq::g_last_error.c_str(); }
 
-extern "C" int tq_version(void) { return 100; }
+extern "C" int tq_version(void) { return 101; }
 
-extern "C" tq_status tq_make_rotation(int d, uint64_t seed, double* pi, uint16_t* pi_f16) {
+extern "C" tq_status tq_make_rotation_ex(int d, uint64_t seed, int rotation, double* pi, uint16_t* pi_f16) {
     tq::clear_error();
     if (d < 2 || d > 1024) return tq::fail(TQ_ERR_INVALID_ARG, "tq_make_rotation: d=%d outside [2, 1024]", d);
     if (!pi && !pi_f16) return tq::fail(TQ_ERR_INVALID_ARG, "tq_make_rotation: pi and pi_f16 are both NULL");
+    if (rotation != TQ_ROT_HAAR && rotation != TQ_ROT_HADAMARD)
+        return tq::fail(TQ_ERR_INVALID_ARG, "tq_make_rotation: rotation=%d (TQ_ROT_HAAR or TQ_ROT_HADAMARD)", rotation);
+    if (rotation == TQ_ROT_HADAMARD && (d & (d - 1)))
+        return tq::fail(TQ_ERR_INVALID_ARG, "tq_make_rotation: d=%d is not a power of two (Hadamard)", d);
     std::vector<double> m(static_cast<size_t>(d) * d);
-    tq::host_rotation(d, seed, m.data());
+    tq::host_rotation_of(rotation, d, seed, m.data());
     if (pi) std::memcpy(pi, m.data(), m.size() * sizeof(double));
     if (pi_f16)
         for (size_t i = 0; i < m.size(); ++i) pi_f16[i] = tq::f64_to_f16(m[i]);
     return TQ_OK;
+}
+
+extern "C" tq_status tq_make_rotation(int d, uint64_t seed, double* pi, uint16_t* pi_f16) {
+    return tq_make_rotation_ex(d, seed, TQ_ROT_HAAR, pi, pi_f16);
 }
 
 extern "C" tq_status tq_build_codebook(int d, int bits, double* centroids, uint16_t* centroids_f16,

@@ -15,6 +15,14 @@ void clear_error();
 // Householder reflections, Q's columns multiplied by sign(diag R) (zero taken as +1).
 void host_rotation(int d, uint64_t seed, double* pi);
 
+// Seeded randomized Walsh-Hadamard rotation (row-major d*d doubles, d a power of two):
+// Pi = H diag(s) / sqrt(d), H the Sylvester Hadamard matrix, s_j = -1 if the top bit of SplitMix64(seed)
+// output j is set, else +1.
+void host_hadamard(int d, uint64_t seed, double* pi);
+
+// Either rotation by kind (TQ_ROT_HAAR / TQ_ROT_HADAMARD); false for an unknown kind.
+bool host_rotation_of(int kind, int d, uint64_t seed, double* pi);
+
 // Lloyd-Max levels (ascending, 2^bits) of the sphere-coordinate density for dimension d, fp64.
 void host_codebook(int d, int bits, double* levels);
 

@@ -112,7 +112,7 @@ bool supported_d(int d) { return d == 64 || d == 128 || d == 256; }
 // ------------------------------------------------------------------------------------------- codec
 
 struct tq_codec {
-    int d = 0, bits = 0, device = 0;
+    int d = 0, bits = 0, device = 0, rotation = TQ_ROT_HAAR;
     uint64_t seed = 0;
     __half* pi_op = nullptr;        // d x d, rotated = Pi_op x
     __half* pi_op_t = nullptr;      // Pi_op^T, the decode-side B operand
@@ -152,16 +152,18 @@ tq_status build_grid_lut(int bits, const float* t, std::vector<uint32_t>& lut) {
 
 }  // namespace
 
-extern "C" tq_status tq_codec_create(int d, int k_bits, uint64_t seed, tq_codec** out) {
+extern "C" tq_status tq_codec_create_ex(int d, int k_bits, uint64_t seed, int rotation, tq_codec** out) {
     clear_error();
     if (!out) return fail(TQ_ERR_INVALID_ARG, "tq_codec_create: out is NULL");
     *out = nullptr;
     if (!supported_d(d)) return fail(TQ_ERR_UNSUPPORTED, "tq_codec_create: d=%d (supported: 64, 128, 256)", d);
     if (k_bits < 1 || k_bits > 4) return fail(TQ_ERR_UNSUPPORTED, "tq_codec_create: k_bits=%d (supported: 1..4)", k_bits);
+    if (rotation != TQ_ROT_HAAR && rotation != TQ_ROT_HADAMARD)
+        return fail(TQ_ERR_INVALID_ARG, "tq_codec_create: rotation=%d (TQ_ROT_HAAR or TQ_ROT_HADAMARD)", rotation);
     const size_t dd = static_cast<size_t>(d) * d;
     std::vector<uint16_t> pi16(dd), pit16(dd);
     std::vector<double> pi(dd);
-    host_rotation(d, seed, pi.data());
+    host_rotation_of(rotation, d, seed, pi.data());
     for (int i = 0; i < d; ++i)
         for (int j = 0; j < d; ++j) {
             pi16[static_cast<size_t>(i) * d + j] = f64_to_f16(pi[static_cast<size_t>(i) * d + j]);
@@ -182,6 +184,7 @@ extern "C" tq_status tq_codec_create(int d, int k_bits, uint64_t seed, tq_codec*
     c->d = d;
     c->bits = k_bits;
     c->seed = seed;
+    c->rotation = rotation;
     cudaGetDevice(&c->device);
     auto cleanup = [&](tq_status s) {
         tq_codec_destroy(c);
@@ -200,6 +203,10 @@ extern "C" tq_status tq_codec_create(int d, int k_bits, uint64_t seed, tq_codec*
     if ((st = make_tmap_f16(&c->tmap_pit, c->pi_op_t, d, d, d, d)) != TQ_OK) return cleanup(st);
     *out = c;
     return TQ_OK;
+}
+
+extern "C" tq_status tq_codec_create(int d, int k_bits, uint64_t seed, tq_codec** out) {
+    return tq_codec_create_ex(d, k_bits, seed, TQ_ROT_HAAR, out);
 }
 
 extern "C" tq_status tq_codec_destroy(tq_codec* c) {
@@ -222,6 +229,13 @@ extern "C" tq_status tq_codec_info(const tq_codec* c, int* d, int* k_bits, uint6
     if (d) *d = c->d;
     if (k_bits) *k_bits = c->bits;
     if (seed) *seed = c->seed;
+    return TQ_OK;
+}
+
+extern "C" tq_status tq_codec_rotation(const tq_codec* c, int* rotation) {
+    clear_error();
+    if (!c || !rotation) return fail(TQ_ERR_INVALID_ARG, "tq_codec_rotation: codec and rotation must be non-NULL");
+    *rotation = c->rotation;
     return TQ_OK;
 }
 

@@ -18,6 +18,8 @@ LIB_PATH = os.path.join(_PKG, "libtq.so")
 
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_DEVICE_FLAG = range(5)
 TQ_F16, TQ_F32 = 0, 1
+TQ_ROT_HAAR, TQ_ROT_HADAMARD = 0, 1
+ROTATIONS = {"haar": TQ_ROT_HAAR, "hadamard": TQ_ROT_HADAMARD}
 
 _c_i64p = ctypes.POINTER(ctypes.c_int64)
 
@@ -41,9 +43,14 @@ SIGNATURES = {
     "tq_last_error": (ctypes.c_char_p, []),
     "tq_version": (ctypes.c_int, []),
     "tq_make_rotation": (ctypes.c_int, [ctypes.c_int, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]),
+    "tq_make_rotation_ex": (ctypes.c_int, [ctypes.c_int, ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p,
+                                           ctypes.c_void_p]),
     "tq_build_codebook": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_void_p]),
     "tq_codec_create": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_uint64, ctypes.POINTER(ctypes.c_void_p)]),
+    "tq_codec_create_ex": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_uint64, ctypes.c_int,
+                                          ctypes.POINTER(ctypes.c_void_p)]),
+    "tq_codec_rotation": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)]),
     "tq_codec_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "tq_codec_info": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "tq_encode_k": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
@@ -106,11 +113,12 @@ def _need_cuda(t: torch.Tensor, name: str, dtype=None):
 
 # ------------------------------------------------------------------------------- host parameters
 
-def make_rotation(d: int, seed: int):
-    """(Pi fp64 [d, d], Pi_op fp16 [d, d]) from tq_make_rotation."""
+def make_rotation(d: int, seed: int, rotation: str = "haar"):
+    """(Pi fp64 [d, d], Pi_op fp16 [d, d]) from tq_make_rotation_ex."""
     pi = np.empty((d, d), np.float64)
     pi16 = np.empty((d, d), np.uint16)
-    _check("tq_make_rotation", LIB.tq_make_rotation(d, seed, pi.ctypes.data, pi16.ctypes.data))
+    _check("tq_make_rotation_ex", LIB.tq_make_rotation_ex(d, seed, ROTATIONS[rotation], pi.ctypes.data,
+                                                          pi16.ctypes.data))
     return pi, pi16.view(np.float16)
 
 
@@ -129,13 +137,14 @@ def build_codebook(d: int, bits: int):
 # ------------------------------------------------------------------------------------ key codec
 
 class Codec:
-    """A key codec (rotation + codebook resident on the current CUDA device)."""
+    """A key codec (rotation + codebook resident on the current CUDA device).  rotation: "haar" (the seeded
+    Haar rotation) or "hadamard" (the seeded randomized Walsh-Hadamard rotation)."""
 
-    def __init__(self, d: int, bits: int, seed: int = 0):
+    def __init__(self, d: int, bits: int, seed: int = 0, rotation: str = "haar"):
         h = ctypes.c_void_p()
-        _check("tq_codec_create", LIB.tq_codec_create(d, bits, seed, ctypes.byref(h)))
+        _check("tq_codec_create_ex", LIB.tq_codec_create_ex(d, bits, seed, ROTATIONS[rotation], ctypes.byref(h)))
         self._h = h
-        self.d, self.bits, self.seed = d, bits, seed
+        self.d, self.bits, self.seed, self.rotation = d, bits, seed, rotation
         self.row_bytes = d * bits // 8
 
     @property

@@ -22,8 +22,8 @@ L2_RTOL = 1e-3
 
 
 @functools.lru_cache(maxsize=None)
-def params(d: int, bits: int, seed: int):
-    pi_op = o.operational_rotation(d, seed)
+def params(d: int, bits: int, seed: int, rotation: str = "haar"):
+    pi_op = o.operational_rotation(d, seed, rotation)
     c_op, t = o.operational_codebook(d, bits)
     return pi_op, c_op, t
 

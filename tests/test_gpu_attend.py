@@ -17,18 +17,18 @@ DEV = "cuda:0"
 _CODECS = {}
 
 
-def codec(d, bits, seed=0):
-    if (d, bits, seed) not in _CODECS:
-        _CODECS[(d, bits, seed)] = tq.Codec(d, bits, seed)
-    return _CODECS[(d, bits, seed)]
+def codec(d, bits, seed=0, rotation="haar"):
+    if (d, bits, seed, rotation) not in _CODECS:
+        _CODECS[(d, bits, seed, rotation)] = tq.Codec(d, bits, seed, rotation=rotation)
+    return _CODECS[(d, bits, seed, rotation)]
 
 
-def build_contiguous(b, hkv, t, d, kb, vb, vg, seed=0, scaled=True):
+def build_contiguous(b, hkv, t, d, kb, vb, vg, seed=0, scaled=True, rotation="haar"):
     ks = synth.channel_scales(seed, hkv, d, "k") if scaled else None
     vs = synth.channel_scales(seed, hkv, d, "v") if scaled else None
     k = synth.kv_tensor(seed, synth.STREAM_K, b, hkv, t, d, device=DEV, scales=ks).view(-1, d)
     v = synth.kv_tensor(seed, synth.STREAM_V, b, hkv, t, d, device=DEV, scales=vs).view(-1, d)
-    cd = codec(d, kb, seed)
+    cd = codec(d, kb, seed, rotation)
     kp, kn = cd.encode_k(k)
     vd, vsc, vz = tq.encode_v(v, vb, vg)
     return cd, tq.Cache(kp, kn, vd, vsc, vz)
@@ -37,7 +37,7 @@ def build_contiguous(b, hkv, t, d, kb, vb, vg, seed=0, scaled=True):
 def oracle_heads(cd, cache, q16, b, h, rows, vb, vg, hq_per_kv, scale=None):
     """Oracle outputs of the query heads of kv head h of sequence b over pool rows `rows`."""
     d, kb = cd.d, cd.bits
-    pi, c, _ = params(d, kb, cd.seed)
+    pi, c, _ = params(d, kb, cd.seed, cd.rotation)
     r = torch.as_tensor(rows, device=DEV)
     idx = o.unpack_lsb(to_np(cache.k_packed[r]), kb, d)
     nrm = to_np(cache.k_norms[r]).astype(np.float64)
@@ -50,8 +50,8 @@ def oracle_heads(cd, cache, q16, b, h, rows, vb, vg, hq_per_kv, scale=None):
     return o.attend(qs, idx[None, None], nrm[None, None], vh[None, None], pi, c, scale)[0]
 
 
-def _run_contiguous(b, hkv, hq, t, d, kb, vb, vg, seq_lens=None, seed=0, check_bh=None):
-    cd, cache = build_contiguous(b, hkv, t, d, kb, vb, vg, seed)
+def _run_contiguous(b, hkv, hq, t, d, kb, vb, vg, seq_lens=None, seed=0, check_bh=None, rotation="haar"):
+    cd, cache = build_contiguous(b, hkv, t, d, kb, vb, vg, seed, rotation=rotation)
     q16 = synth.normal_fp16(seed, synth.STREAM_Q, (b, hq, d))
     sl = torch.tensor(seq_lens, dtype=torch.int32, device=DEV) if seq_lens is not None else None
     out = tq.attend_decode(cd, q16.to(DEV), cache, num_kv_heads=hkv, v_bits=vb, v_group=vg, max_seq_len=t,
@@ -77,6 +77,12 @@ def _run_contiguous(b, hkv, hq, t, d, kb, vb, vg, seq_lens=None, seed=0, check_b
                                         (256, 2, 2, 256)])
 def test_attend_contiguous_formats(d, kb, vb, vg):
     _run_contiguous(2, 2, 8, 320, d, kb, vb, vg, seq_lens=[320, 157])
+
+
+@pytest.mark.parametrize("d,kb,vb,vg", [(128, 3, 2, 32), (64, 4, 4, 64), (256, 2, 4, 32)])
+def test_attend_hadamard_rotation(d, kb, vb, vg):
+    # the query is rotated by the codec's (Walsh-Hadamard) rotation like the keys: scores need no un-rotation
+    _run_contiguous(2, 2, 8, 320, d, kb, vb, vg, seq_lens=[320, 157], rotation="hadamard")
 
 
 @pytest.mark.parametrize("hkv,hq", [(4, 4), (2, 16), (1, 8), (3, 6)])

@@ -2,6 +2,7 @@
 
 Indices bit-exact except in-band neighbour flips (< 1e-4 of coordinates); norms within 1e-6 relative;
 decode within 1e-3 relative L2 of the oracle's decode of the GPU's own indices and norms."""
+import ctypes
 import math
 
 import numpy as np
@@ -119,3 +120,23 @@ def test_key_full_size_sampled():
     ref_dec = o.decode_k(gidx, gn.astype(np.float64), pi, c)
     assert rel_l2(to_np(out[rows.to(DEV)]), ref_dec) <= L2_RTOL
     assert tq.read_device_flag() == 0
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("bits", [2, 4])
+def test_key_codec_parity_hadamard_rotation(d, bits):
+    # the randomized Walsh-Hadamard rotation ("turbo-attn", The codec) through the same tensor-core kernels
+    cd = tq.Codec(d, bits, 3, rotation="hadamard")
+    pi, c, t = params(d, bits, 3, "hadamard")
+    for n in (1, 300, 4097):
+        x16 = synth.normal_fp16(n + bits, synth.STREAM_K, (n, d))
+        packed, norms = cd.encode_k(x16.to(DEV))
+        out = cd.decode_k(packed, norms)
+        ref_idx, ref_n, y = o.encode_k(x16.numpy(), pi, t)
+        gidx = o.unpack_lsb(to_np(packed), bits, d)
+        check_key_indices(gidx, ref_idx, y, t)
+        gn = to_np(norms)
+        assert np.all(np.abs(gn - ref_n) <= NORM_RTOL * ref_n)
+        assert rel_l2(to_np(out), o.decode_k(gidx, gn.astype(np.float64), pi, c)) <= L2_RTOL
+    rot = ctypes.c_int(-1)
+    assert tq.LIB.tq_codec_rotation(cd.handle, ctypes.byref(rot)) == tq.TQ_OK and rot.value == tq.TQ_ROT_HADAMARD

@@ -39,6 +39,24 @@ def test_rotation_matches_oracle(d):
         assert np.array_equal(pi16.astype(np.float64), o.to_fp16_values(ref))
 
 
+@pytest.mark.parametrize("d", [2, 64, 128, 256, 1024])
+def test_hadamard_rotation_matches_oracle(d):
+    pi, pi16 = tq.make_rotation(d, 17, "hadamard")
+    ref = o.hadamard_rotation(d, 17)
+    assert np.array_equal(pi, ref)
+    assert np.array_equal(pi16.astype(np.float64), o.to_fp16_values(ref))
+    assert np.array_equal(pi16.astype(np.float64), o.operational_rotation(d, 17, "hadamard"))
+
+
+def test_rotation_kind_errors():
+    out = np.empty(96 * 96)
+    assert tq.LIB.tq_make_rotation_ex(96, 0, tq.TQ_ROT_HADAMARD, out.ctypes.data, None) == tq.TQ_ERR_INVALID_ARG
+    assert b"power of two" in tq.LIB.tq_last_error()
+    assert tq.LIB.tq_make_rotation_ex(64, 0, 7, out.ctypes.data, None) == tq.TQ_ERR_INVALID_ARG
+    assert tq.LIB.tq_codec_create_ex(128, 4, 0, 7, ctypes.byref(ctypes.c_void_p())) == tq.TQ_ERR_INVALID_ARG
+    assert tq.LIB.tq_version() == 101
+
+
 @pytest.mark.parametrize("d", [3, 64, 128, 256, 1024])
 @pytest.mark.parametrize("bits", [1, 2, 3, 4])
 def test_codebook_matches_oracle(d, bits):
