@@ -556,6 +556,45 @@ def attend(q16: np.ndarray, k_idx: np.ndarray, k_norms: np.ndarray, v_hat: np.nd
     return out
 
 
+def attend_window(q16: np.ndarray, k_idx: np.ndarray, k_norms: np.ndarray, v_hat: np.ndarray,
+                  win_k16: np.ndarray, win_v16: np.ndarray, pi_op: np.ndarray, c_op: np.ndarray,
+                  scale: float | None = None, seq_lens: np.ndarray | None = None,
+                  win_lens: np.ndarray | None = None) -> np.ndarray:
+    """Decode attention over the compressed cache plus a window of recent uncompressed tokens.
+
+    [P3] store.py ``TurboQuantKVCache``: ``attention_scores`` concatenates scale * (the quantized part's
+    scores) with scale * query @ key_buffer^T; the caller's softmax runs over all of them; ``attend`` adds
+    the quantized part's weights times the dequantized values and the buffer's weights times the buffer's
+    values, which are used as stored (fp16).  The compressed part's scores are those of ``attend_one``
+    (path A, the decoded keys).
+
+    q16 [B][H_q][d]; k_idx [B][H_kv][T][d]; k_norms [B][H_kv][T]; v_hat [B][H_kv][T][d];
+    win_k16, win_v16 [B][H_kv][W][d] fp16; optional seq_lens / win_lens [B] (tokens 0..len-1 of each part).
+    Returns o [B][H_q][d] fp64 (zeros where both parts are empty).
+    """
+    bsz, hq, d = q16.shape
+    hkv = k_idx.shape[1]
+    grp = hq // hkv
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = np.zeros((bsz, hq, d), dtype=np.float64)
+    for b in range(bsz):
+        tl = k_idx.shape[2] if seq_lens is None else int(seq_lens[b])
+        wl = win_k16.shape[2] if win_lens is None else int(win_lens[b])
+        for h in range(hq):
+            kv = h // grp
+            q = np.asarray(q16[b, h]).astype(np.float64)
+            k_all = np.concatenate([decode_k(k_idx[b, kv, :tl], k_norms[b, kv, :tl], pi_op, c_op),
+                                    np.asarray(win_k16[b, kv, :wl]).astype(np.float64)], axis=0)
+            v_all = np.concatenate([np.asarray(v_hat[b, kv, :tl], dtype=np.float64),
+                                    np.asarray(win_v16[b, kv, :wl]).astype(np.float64)], axis=0)
+            if k_all.shape[0] == 0:
+                continue
+            s = scale * (k_all @ q)
+            p = np.exp(s - s.max())
+            out[b, h] = (p / p.sum()) @ v_all
+    return out
+
+
 def paged_rows(block_table: np.ndarray, b: int, h: int, length: int, num_kv_heads: int,
                block_size: int) -> np.ndarray:
     """Pool rows of sequence b, kv head h, positions 0..length-1 in the paged layout.

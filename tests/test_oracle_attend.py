@@ -99,3 +99,50 @@ def test_seq_lens_and_paged_layout():
     for bi in range(b):
         for h in range(hkv):
             assert np.array_equal(pool_idx[o.paged_rows(table, bi, h, t, hkv, bs)], idx[bi, h])
+
+
+# ---- recent uncompressed window ("KV Cache API", store.py TurboQuantKVCache: quantized part + fp16 buffer)
+
+def _window_case(seed, tl, wl, d=64, kb=3, vb=2):
+    rng = np.random.default_rng(seed)
+    pi = o.operational_rotation(d, seed)
+    c, t = o.operational_codebook(d, kb)
+    q16 = rng.standard_normal((1, 4, d)).astype(np.float16)
+    k16 = rng.standard_normal((1, 2, tl, d)).astype(np.float16)
+    v16 = rng.standard_normal((1, 2, tl, d)).astype(np.float16)
+    idx, nrm, _ = o.encode_k(k16.reshape(-1, d), pi, t)
+    idx = idx.reshape(1, 2, tl, d)
+    nrm = nrm.reshape(1, 2, tl)
+    dat, sc, zr, _ = o.encode_v(v16.reshape(-1, d), vb)
+    vh = o.decode_v(dat, sc, zr, vb, d).reshape(1, 2, tl, d)
+    wk = rng.standard_normal((1, 2, wl, d)).astype(np.float16)
+    wv = rng.standard_normal((1, 2, wl, d)).astype(np.float16)
+    return q16, idx, nrm, vh, wk, wv, pi, c
+
+
+def test_window_attention_is_softmax_over_the_concatenation():
+    # pinned against the library's scaled-dot-product attention on the explicitly concatenated keys and values
+    q16, idx, nrm, vh, wk, wv, pi, c = _window_case(1, 37, 21)
+    got = o.attend_window(q16, idx, nrm, vh, wk, wv, pi, c)
+    for h in range(4):
+        kv = h // 2
+        k_all = np.concatenate([o.decode_k(idx[0, kv], nrm[0, kv], pi, c), wk[0, kv].astype(np.float64)])
+        v_all = np.concatenate([vh[0, kv].astype(np.float64), wv[0, kv].astype(np.float64)])
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q16[0, h].astype(np.float64))[None, None, None],
+            torch.from_numpy(k_all)[None, None], torch.from_numpy(v_all)[None, None])[0, 0, 0].numpy()
+        assert np.abs(got[0, h] - ref).max() < 1e-12
+
+
+def test_window_attention_reduces_to_its_parts():
+    q16, idx, nrm, vh, wk, wv, pi, c = _window_case(2, 40, 16)
+    # an empty window is the compressed attention; an empty compressed part is attention over the window alone
+    assert np.abs(o.attend_window(q16, idx, nrm, vh, wk, wv, pi, c, win_lens=np.array([0]))
+                  - o.attend(q16, idx, nrm, vh, pi, c)).max() < 1e-12
+    only_w = o.attend_window(q16, idx, nrm, vh, wk, wv, pi, c, seq_lens=np.array([0]))
+    for h in range(4):
+        s = wk[0, h // 2].astype(np.float64) @ q16[0, h].astype(np.float64) / np.sqrt(64)
+        p = np.exp(s - s.max())
+        assert np.abs(only_w[0, h] - (p / p.sum()) @ wv[0, h // 2].astype(np.float64)).max() < 1e-12
+    both_empty = o.attend_window(q16, idx, nrm, vh, wk, wv, pi, c, seq_lens=np.array([0]), win_lens=np.array([0]))
+    assert np.all(both_empty == 0)
