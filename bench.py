@@ -187,7 +187,15 @@ def gpu_arm(args, w, rank, world, local_rank):
     out = torch.empty(b, hq, d, dtype=torch.float32, device=dev)
     cache = tq.Cache(kp, kn, vd, vsc, vz)
     akw = dict(num_kv_heads=hkv, v_bits=vb, v_group=vg, max_seq_len=t, block_table=None, seq_lens=None, scale=0.0)
-    ws = tq.attend_workspace(codec, q, cache, **akw)
+    if args.window > 0:
+        # recent uncompressed tokens beside the compressed cache ("KV Cache API" store.py buffer)
+        win_k = synth.normal_fp16(0, 21, (b, hkv, args.window, d), device=dev)
+        win_v = synth.normal_fp16(0, 22, (b, hkv, args.window, d), device=dev)
+        akw.update(win_k=win_k, win_v=win_v)
+        ws = tq.attend_window_workspace(codec, q, cache, win_k, win_v, None,
+                                        **{k: v for k, v in akw.items() if not k.startswith("win_")})
+    else:
+        ws = tq.attend_workspace(codec, q, cache, **akw)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     kernels = [
@@ -355,6 +363,8 @@ def main():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--workload", default="70b_decode_128k", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--window", type=int, default=0,
+                    help="recent uncompressed tokens per (sequence, kv head) attended beside the compressed cache")
     ap.add_argument("--rotation", default="haar", choices=["haar", "hadamard"],
                     help="key rotation: seeded Haar (default) or randomized Walsh-Hadamard; same kernels")
     ap.add_argument("--only", choices=["encode_k", "encode_v", "decode_k", "decode_v", "attend"],
@@ -369,7 +379,7 @@ def main():
     bpv = algorithmic_bytes(w)
     config = {"workload": args.workload, "description": w["desc"], "batch": w["batch"], "kv_heads": w["kv_heads"],
               "q_heads": w["q_heads"], "tokens": w["tokens"], "head_dim": w["d"], "k_bits": w["k_bits"],
-              "v_bits": w["v_bits"], "v_group": w["v_group"], "rotation": args.rotation,
+              "v_bits": w["v_bits"], "v_group": w["v_group"], "rotation": args.rotation, "window": args.window,
               "vector": "one (token, kv head) key/value pair through encode + decode + attention",
               "l2": "flushed by a 256 MiB write before every kernel launch (outside the timed interval)",
               "parallelism": f"replicas x{world} (independent caches, no collective on the data path)"}

@@ -258,6 +258,42 @@ tq_status tq_attend_workspace_bytes(const tq_attend_args* args, size_t* bytes);
  */
 tq_status tq_attend_decode(const tq_codec* codec, const tq_attend_args* args, void* stream);
 
+/* --------------------------------------------------------------------------------------------------
+ * Attention with a window of recent uncompressed tokens.
+ * ------------------------------------------------------------------------------------------------ */
+
+/* Largest window per (sequence, kv head) tq_attend_decode_window accepts. */
+#define TQ_ATTEND_WINDOW_MAX 256
+
+typedef struct tq_attend_window {
+    const void* k;             /* device binary16 [batch][num_kv_heads][max_len][head_dim]: recent keys as stored */
+    const void* v;             /* device binary16, same layout: recent values as stored */
+    const int32_t* lens;       /* device int32 [batch]: window tokens of each sequence (clamped to 0..max_len);
+                                  NULL: max_len for every sequence */
+    int max_len;               /* 1..TQ_ATTEND_WINDOW_MAX */
+} tq_attend_window;
+
+/*
+ * tq_attend_window_workspace_bytes -- workspace bytes tq_attend_decode_window needs (as
+ * tq_attend_workspace_bytes, with one more partial per (sequence, kv head) for the window).
+ */
+tq_status tq_attend_window_workspace_bytes(const tq_attend_args* args, const tq_attend_window* window,
+                                           size_t* bytes);
+
+/*
+ * tq_attend_decode_window -- tq_attend_decode over the compressed cache plus a window of recent tokens kept
+ * uncompressed ("KV Cache API", store.py TurboQuantKVCache: attention_scores concatenates the quantized
+ * part's scores with scale * query @ key_buffer^T; the softmax runs over both; attend adds the quantized
+ * part's weights times the dequantized values and the buffer's weights times the buffer's values).  The
+ * window's scores are fp32 dot products of the fp16 query and keys, times the same scale; one extra CTA per
+ * (sequence, kv head) computes them and its partial (max, sum, weighted values) enters the same split merge.
+ * A sequence whose compressed part and window are both empty yields zeros.
+ * Errors: as tq_attend_decode, plus TQ_ERR_INVALID_ARG for a NULL window, NULL k or v, max_len outside
+ * 1..TQ_ATTEND_WINDOW_MAX or misaligned (16-byte) k / v.
+ */
+tq_status tq_attend_decode_window(const tq_codec* codec, const tq_attend_args* args, const tq_attend_window* window,
+                                  void* stream);
+
 /*
  * TQ_ATTEND_SCRATCH_BYTES -- size of the library-owned scratch used by tq_attend_decode_noalloc (4 MiB).
  * That array lives in the library's device image, so every GPU that loads libtq holds it until the process

@@ -38,8 +38,22 @@ struct AttendParams {
     float* out;
     float* partials;                                 // [B][H_kv][splits][16 + 8 d]
     uint4* qfrag;                                    // [B][H_kv][d/16 * 32 + 2]: score A fragments, 1 / prescale
-    int num_splits;
+    int num_splits;                                  // CTAs along the compressed sequence
+    int num_parts;                                   // partials per (sequence, kv head): splits (+ 1 window)
+    const __half* win_k;                             // nullable: [B][H_kv][win_max][d] recent keys, uncompressed
+    const __half* win_v;
+    const int32_t* win_lens;                         // nullable: win_max for every sequence
+    int win_max;
 };
+
+constexpr int kWinMax = 256;                         // largest window per (sequence, kv head)
+constexpr int kWinChunk = 32;                        // window tokens staged in shared memory at a time
+
+// shared memory of the window path (floats): query, scores, max/sum, one staged chunk, two partial sums
+template <int D>
+__host__ __device__ constexpr int window_smem_floats() {
+    return 8 * D + 8 * kWinMax + 16 + kWinChunk * (D + 2) / 2 + 2 * 8 * D;
+}
 
 // uint4 slots per (sequence, kv head) of the query-fragment array: the fragments, then 1 / prescale of 8 heads
 template <int D>
@@ -83,7 +97,9 @@ struct AttCfg {
     static constexpr int kLutOff = kQfOff + (kQInRegs ? 0 : (D / 16) * 32 * 16);
     static constexpr int kZsOff = kLutOff + 2 * kLutBytes;
     static constexpr int kBarOff = (kZsOff + kWarps * 8 * kVGroups * 4 + 15) & ~15;
-    static constexpr int kSmem = kBarOff + 8 * (2 * kStages) + 16;
+    static constexpr int kSmemMain = kBarOff + 8 * (2 * kStages) + 16;
+    // the window CTA reuses the same allocation
+    static constexpr int kSmem = (kSmemMain > window_smem_floats<D>() * 4) ? kSmemMain : window_smem_floats<D>() * 4;
     static_assert(kNOff % 16 == 0 && kVOff % 16 == 0 && kSOff % 16 == 0 && kZOff % 16 == 0 && kStageBytes % 16 == 0,
                   "bulk copies need 16-byte multiples");
     static_assert(VG % 32 == 0, "a 32-column slice of the value row lies in one scale group");
@@ -274,6 +290,117 @@ __global__ void __launch_bounds__(kPrepThreads) attend_prep_kernel(const AttendP
     if (blockIdx.x == 0 && warp == 0 && tig == 0) reinterpret_cast<float*>(qf + KS * 32)[gid] = 1.0f / pre;
 }
 
+// The window part of one (sequence, kv head): scores of the group's queries against the recent uncompressed
+// keys (fp32 dot products of the fp16 inputs, in the log2 domain like the compressed part's), their maximum m,
+// l = sum 2^(s - m) and O = sum 2^(s - m) v -- one partial of the split merge.  All threads of the CTA.  Keys
+// and values go through shared memory in chunks of kWinChunk tokens, loaded with coalesced 16-byte reads; key
+// rows are padded by 4 bytes so the per-token dot products read distinct banks.
+template <int D>
+__device__ void attend_window_partial(const AttendParams& p, int b, int h, uint8_t* smem, float* part) {
+    const int G = p.group, tid = threadIdx.x, nth = blockDim.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int KR = D + 2;                              // padded key row, in halves
+    float* qs = reinterpret_cast<float*>(smem);            // [8][D]  query * scale * log2(e)
+    float* ss = qs + 8 * D;                                // [8][kWinMax]  scores, then weights
+    float* ml = ss + 8 * kWinMax;                          // [16]  per-head max and sum
+    __half* kv = reinterpret_cast<__half*>(ml + 16);       // one chunk of keys [kWinChunk][KR] or values [kWinChunk][D]
+    float* red = ml + 16 + kWinChunk * KR / 2;             // [2][8][D] partial sums of up to two token groups
+    int L = p.win_lens ? p.win_lens[b] : p.win_max;
+    L = L < 0 ? 0 : (L > p.win_max ? p.win_max : L);
+    const __half* qg = p.q + (static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * G) * D;
+    const int64_t base = (static_cast<int64_t>(b) * p.num_kv_heads + h) * p.win_max * D;
+    const __half* wk = p.win_k + base;
+    const __half* wv = p.win_v + base;
+    for (int i = tid; i < G * D; i += nth) qs[i] = __half2float(qg[i]) * p.scale_log2;
+    // ---- scores, chunk by chunk: thread (g, t) of the chunk
+    for (int t0 = 0; t0 < L; t0 += kWinChunk) {
+        const int cl = (L - t0 < kWinChunk) ? L - t0 : kWinChunk;
+        __syncthreads();                                   // the previous chunk's readers are done (and qs is set)
+        for (int i = tid; i < cl * (D / 8); i += nth) {
+            const int t = i / (D / 8), c8 = i % (D / 8);
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(wk + static_cast<int64_t>(t0 + t) * D) + c8);
+            uint32_t* dst = reinterpret_cast<uint32_t*>(kv + t * KR + 8 * c8);
+            dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+        }
+        __syncthreads();
+        for (int i = tid; i < G * cl; i += nth) {
+            const int g = i / cl, t = i % cl;
+            const __half2* kr = reinterpret_cast<const __half2*>(kv + t * KR);
+            const float2* qr = reinterpret_cast<const float2*>(qs + g * D);
+            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+            for (int c = 0; c < D / 2; ++c) {
+                const float2 k2 = __half22float2(kr[c]);
+                const float2 q2 = qr[c];
+                acc0 = fmaf(q2.x, k2.x, acc0);
+                acc1 = fmaf(q2.y, k2.y, acc1);
+            }
+            ss[g * kWinMax + t0 + t] = acc0 + acc1;
+        }
+    }
+    __syncthreads();
+    // ---- per head: max, weights 2^(s - m), their sum
+    for (int g = warp; g < G; g += nth / 32) {
+        float m = -INFINITY;
+        for (int t = lane; t < L; t += 32) m = fmaxf(m, ss[g * kWinMax + t]);
+#pragma unroll
+        for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float l = 0.f;
+        for (int t = lane; t < L; t += 32) {
+            const float w = exp2f(ss[g * kWinMax + t] - m);
+            ss[g * kWinMax + t] = w;
+            l += w;
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+        if (lane == 0) {
+            ml[g] = m;
+            ml[8 + g] = l;
+        }
+    }
+    // ---- O = sum_t w_t v_t: thread (grp, c2) accumulates column pair c2 of every head over every ngrp-th token
+    const int ngrp = (nth / (D / 2) >= 2) ? 2 : 1;
+    const int grp = tid / (D / 2), c2 = tid % (D / 2);
+    float acc[8][2];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) acc[g][0] = acc[g][1] = 0.f;
+    for (int t0 = 0; t0 < L; t0 += kWinChunk) {
+        const int cl = (L - t0 < kWinChunk) ? L - t0 : kWinChunk;
+        __syncthreads();
+        for (int i = tid; i < cl * (D / 8); i += nth) {
+            const int t = i / (D / 8), c8 = i % (D / 8);
+            reinterpret_cast<uint4*>(kv + t * D)[c8] =
+                __ldg(reinterpret_cast<const uint4*>(wv + static_cast<int64_t>(t0 + t) * D) + c8);
+        }
+        __syncthreads();
+        if (grp < ngrp) {
+            for (int t = grp; t < cl; t += ngrp) {
+                const float2 v2 = __half22float2(reinterpret_cast<const __half2*>(kv + t * D)[c2]);
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    if (g < G) {
+                        const float w = ss[g * kWinMax + t0 + t];
+                        acc[g][0] = fmaf(w, v2.x, acc[g][0]);
+                        acc[g][1] = fmaf(w, v2.y, acc[g][1]);
+                    }
+                }
+            }
+        }
+    }
+    if (grp < ngrp) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g) reinterpret_cast<float2*>(red + (grp * 8 + g) * D)[c2] = make_float2(acc[g][0], acc[g][1]);
+    }
+    __syncthreads();
+    for (int i = tid; i < G * D; i += nth) {
+        const int g = i / D, c = i % D;
+        part[16 + g * D + c] = (ngrp == 2) ? red[g * D + c] + red[(8 + g) * D + c] : red[g * D + c];
+    }
+    if (tid < G) {
+        part[tid] = ml[tid];
+        part[8 + tid] = ml[8 + tid];
+    }
+}
+
 // Fused decode attention for one (split, kv head, sequence).  Per 16-token chunk and warp:
 //   scores  S[head][tok]  = (q hi/lo, fp16 A, rows gid / gid + 8) x (codebook pairs, fp16 B) on mma.sync
 //   values  O^T[col][head] += (value codes, bf16 A, exact) x (hi/lo of p * scale, bf16 B)
@@ -303,6 +430,16 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
     const int gid = lane >> 2, tig = lane & 3;
     const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int G = p.group;
+    static_assert(window_smem_floats<D>() * 4 <= C::kSmem, "the window path fits the CTA's shared memory");
+    static_assert(C::kThreads >= D / 2, "one thread per column pair in the window's value pass");
+    if (split == p.num_splits) {
+        // the extra CTA of a call with a window of recent uncompressed tokens: its own partial, then done
+        attend_window_partial<D>(p, b, h, smem,
+                                 p.partials + ((static_cast<int64_t>(b) * p.num_kv_heads + h) * p.num_parts + split) *
+                                                  C::kPartFloats);
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+        return;
+    }
     const int64_t T = p.seq_lens ? static_cast<int64_t>(p.seq_lens[b]) : p.max_seq_len;
     const int64_t nchunks = (T + 15) / 16;
     const int64_t cps = (nchunks + p.num_splits - 1) / p.num_splits;
@@ -580,7 +717,7 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         // ------------------------------------------------------------------ merge the four warps
         const int tid = threadIdx.x;
         float* part = p.partials +
-                      ((static_cast<int64_t>(b) * p.num_kv_heads + h) * p.num_splits + split) * C::kPartFloats;
+                      ((static_cast<int64_t>(b) * p.num_kv_heads + h) * p.num_parts + split) * C::kPartFloats;
         for (int i = tid; i < G * D; i += 32 * C::kWarps) {
             const int g = i / D, col = i % D;
             float M = -INFINITY;
@@ -594,7 +731,7 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                 L += comb[w * C::kPartFloats + 8 + g] * f;
                 O += comb[w * C::kPartFloats + 16 + g * D + col] * f;
             }
-            if (p.num_splits == 1) {
+            if (p.num_parts == 1) {
                 p.out[(static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * G + g) * D + col] =
                     (L > 0.f) ? O / L : 0.f;
             } else {
@@ -627,7 +764,7 @@ __global__ void __launch_bounds__(kMergeThreads) attend_merge_kernel(const Atten
     __shared__ float s_ml[kSlices][2];
     const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
     const int col = tid % D, slice = tid / D;
-    const int S = p.num_splits;
+    const int S = p.num_parts;
     const float* base = p.partials + (static_cast<int64_t>(b) * p.num_kv_heads + h) * S * kPart;
     float M = -INFINITY, L = 0.f, O = 0.f;
     for (int s0 = slice; s0 < S; s0 += kSlices * kBatch) {

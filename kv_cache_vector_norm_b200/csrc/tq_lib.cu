@@ -435,12 +435,13 @@ constexpr int kAttendCtasPerSm = 4;
 
 struct AttendPlan {
     int num_splits;
+    int num_parts;             // num_splits, + 1 with a window
     size_t qfrag_bytes;        // query fragments, one block per (sequence, kv head)
     size_t partial_bytes;      // split-K partials (0 with one split)
     size_t workspace_bytes;    // qfrag_bytes + partial_bytes
 };
 
-tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan) {
+tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan, bool window = false) {
     if (!a) return fail(TQ_ERR_INVALID_ARG, "tq_attend: args is NULL");
     if (a->batch < 1 || a->num_kv_heads < 1 || a->num_q_heads < 1)
         return fail(TQ_ERR_INVALID_ARG, "tq_attend: batch, num_q_heads, num_kv_heads must be >= 1");
@@ -465,20 +466,24 @@ tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan) {
         max_chunks = a->max_seq_len / 16;
     }
     const int64_t bh = static_cast<int64_t>(a->batch) * a->num_kv_heads;
-    int64_t splits = (static_cast<int64_t>(sm_count()) * kAttendCtasPerSm + bh - 1) / bh;
+    // fill every SM's resident CTAs once; a window's extra CTA per (sequence, kv head) takes one of them
+    int64_t splits = (static_cast<int64_t>(sm_count()) * kAttendCtasPerSm - (window ? bh : 0) + bh - 1) / bh;
     const int64_t by_len = (max_chunks + 7) / 8;            // at least ~8 chunks (128 tokens) per split
     if (splits > by_len) splits = by_len;
     if (splits > kMaxSplits) splits = kMaxSplits;
     if (splits < 1) splits = 1;
     plan->num_splits = static_cast<int>(splits);
-    plan->partial_bytes = (splits > 1) ? static_cast<size_t>(bh) * splits * (16 + 8 * a->head_dim) * 4 : 0;
+    plan->num_parts = static_cast<int>(splits) + (window ? 1 : 0);
+    plan->partial_bytes =
+        (plan->num_parts > 1) ? static_cast<size_t>(bh) * plan->num_parts * (16 + 8 * a->head_dim) * 4 : 0;
     plan->qfrag_bytes = static_cast<size_t>(bh) * ((a->head_dim / 16) * 32 + 2) * 16;
     plan->workspace_bytes = plan->qfrag_bytes + plan->partial_bytes;
     return TQ_OK;
 }
 
 template <int D, int KB, int VB, int VG>
-tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const AttendPlan& plan, cudaStream_t st) {
+tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const tq_attend_window* win, const AttendPlan& plan,
+                        cudaStream_t st) {
     using Cfg = AttCfg<D, KB, VB, VG>;
     static std::atomic<uint64_t> mask{0};
     auto kern = attend_kernel<D, KB, VB, VG>;
@@ -506,6 +511,17 @@ tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const Attend
     p.qfrag = static_cast<uint4*>(a->workspace);
     p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(a->workspace) + plan.qfrag_bytes);
     p.num_splits = plan.num_splits;
+    p.num_parts = plan.num_parts;
+    p.win_k = nullptr;
+    p.win_v = nullptr;
+    p.win_lens = nullptr;
+    p.win_max = 0;
+    if (win) {
+        p.win_k = static_cast<const __half*>(win->k);
+        p.win_v = static_cast<const __half*>(win->v);
+        p.win_lens = win->lens;
+        p.win_max = win->max_len;
+    }
     attend_prep_kernel<D><<<dim3(D / 32, a->num_kv_heads, a->batch), kPrepThreads, 0, st>>>(p);
     TQ_CUDA(cudaGetLastError(), "tq_attend_decode: query preparation launch");
     // the attention grid and the split merge are programmatic dependents of the grid before them: each is
@@ -514,14 +530,14 @@ tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const Attend
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(plan.num_splits, a->num_kv_heads, a->batch);
+    cfg.gridDim = dim3(plan.num_parts, a->num_kv_heads, a->batch);   // split CTAs, then the window's
     cfg.blockDim = dim3(Cfg::kThreads);
     cfg.dynamicSmemBytes = Cfg::kSmem;
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     TQ_CUDA(cudaLaunchKernelEx(&cfg, kern, p), "tq_attend_decode: launch");
-    if (plan.num_splits > 1) {
+    if (plan.num_parts > 1) {
         cfg.gridDim = dim3(p.group, a->num_kv_heads, a->batch);
         cfg.blockDim = dim3(kMergeThreads);
         cfg.dynamicSmemBytes = 0;
@@ -531,18 +547,69 @@ tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const Attend
 }
 
 template <int D, int KB>
-tq_status attend_v(const tq_codec* c, const tq_attend_args* a, const AttendPlan& plan, cudaStream_t st) {
+tq_status attend_v(const tq_codec* c, const tq_attend_args* a, const tq_attend_window* win, const AttendPlan& plan,
+                   cudaStream_t st) {
     const bool tok = a->v_group == D;
     switch (a->v_bits * 2 + (tok ? 1 : 0)) {
-        case 4: return launch_attend<D, KB, 2, 32>(c, a, plan, st);
-        case 5: return launch_attend<D, KB, 2, D>(c, a, plan, st);
-        case 6: return launch_attend<D, KB, 3, 32>(c, a, plan, st);
-        case 7: return launch_attend<D, KB, 3, D>(c, a, plan, st);
-        case 8: return launch_attend<D, KB, 4, 32>(c, a, plan, st);
-        case 9: return launch_attend<D, KB, 4, D>(c, a, plan, st);
-        case 16: return launch_attend<D, KB, 8, 32>(c, a, plan, st);
-        case 17: return launch_attend<D, KB, 8, D>(c, a, plan, st);
+        case 4: return launch_attend<D, KB, 2, 32>(c, a, win, plan, st);
+        case 5: return launch_attend<D, KB, 2, D>(c, a, win, plan, st);
+        case 6: return launch_attend<D, KB, 3, 32>(c, a, win, plan, st);
+        case 7: return launch_attend<D, KB, 3, D>(c, a, win, plan, st);
+        case 8: return launch_attend<D, KB, 4, 32>(c, a, win, plan, st);
+        case 9: return launch_attend<D, KB, 4, D>(c, a, win, plan, st);
+        case 16: return launch_attend<D, KB, 8, 32>(c, a, win, plan, st);
+        case 17: return launch_attend<D, KB, 8, D>(c, a, win, plan, st);
         default: return fail(TQ_ERR_UNSUPPORTED, "tq_attend_decode: v_bits=%d", a->v_bits);
+    }
+}
+
+}  // namespace
+
+namespace {
+
+tq_status check_window(const char* fn, const tq_attend_window* w) {
+    if (!w) return fail(TQ_ERR_INVALID_ARG, "%s: window is NULL", fn);
+    if (w->max_len < 1 || w->max_len > TQ_ATTEND_WINDOW_MAX)
+        return fail(TQ_ERR_INVALID_ARG, "%s: window max_len=%d outside 1..%d", fn, w->max_len, TQ_ATTEND_WINDOW_MAX);
+    return TQ_OK;
+}
+
+tq_status attend_decode_impl(const char* fn, const tq_codec* c, const tq_attend_args* a, const tq_attend_window* win,
+                             void* stream) {
+    if (!c) return fail(TQ_ERR_INVALID_ARG, "%s: codec is NULL", fn);
+    AttendPlan plan;
+    tq_status s = plan_attend(a, &plan, win != nullptr);
+    if (s != TQ_OK) return s;
+    if (a->head_dim != c->d) return fail(TQ_ERR_INVALID_ARG, "%s: head_dim=%d but the codec has d=%d", fn, a->head_dim, c->d);
+    if (!a->q || !a->k_packed || !a->k_norms || !a->v_data || !a->v_scales || !a->v_zeros || !a->out)
+        return fail(TQ_ERR_INVALID_ARG, "%s: NULL pointer in args", fn);
+    if (!a->workspace || a->workspace_bytes < plan.workspace_bytes)
+        return fail(TQ_ERR_INVALID_ARG, "%s: workspace of %zu bytes required (got %zu)", fn, plan.workspace_bytes,
+                    a->workspace ? a->workspace_bytes : static_cast<size_t>(0));
+    if (!aligned(a->q, 16) || !aligned(a->k_packed, 16) || !aligned(a->k_norms, 16) || !aligned(a->v_data, 16) ||
+        !aligned(a->v_scales, 16) || !aligned(a->v_zeros, 16) || !aligned(a->out, 16) || !aligned(a->workspace, 16))
+        return fail(TQ_ERR_INVALID_ARG, "%s: every pointer must be 16-byte aligned", fn);
+    if (win) {
+        if ((s = check_window(fn, win)) != TQ_OK) return s;
+        if (!win->k || !win->v) return fail(TQ_ERR_INVALID_ARG, "%s: window k and v must be non-NULL", fn);
+        if (!aligned(win->k, 16) || !aligned(win->v, 16) || (win->lens && !aligned(win->lens, 4)))
+            return fail(TQ_ERR_INVALID_ARG, "%s: window k and v must be 16-byte aligned", fn);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (c->d * 10 + c->bits) {
+        case 641: return attend_v<64, 1>(c, a, win, plan, st);
+        case 642: return attend_v<64, 2>(c, a, win, plan, st);
+        case 643: return attend_v<64, 3>(c, a, win, plan, st);
+        case 644: return attend_v<64, 4>(c, a, win, plan, st);
+        case 1281: return attend_v<128, 1>(c, a, win, plan, st);
+        case 1282: return attend_v<128, 2>(c, a, win, plan, st);
+        case 1283: return attend_v<128, 3>(c, a, win, plan, st);
+        case 1284: return attend_v<128, 4>(c, a, win, plan, st);
+        case 2561: return attend_v<256, 1>(c, a, win, plan, st);
+        case 2562: return attend_v<256, 2>(c, a, win, plan, st);
+        case 2563: return attend_v<256, 3>(c, a, win, plan, st);
+        case 2564: return attend_v<256, 4>(c, a, win, plan, st);
+        default: return fail(TQ_ERR_UNSUPPORTED, "%s: d=%d bits=%d", fn, c->d, c->bits);
     }
 }
 
@@ -559,37 +626,28 @@ extern "C" tq_status tq_attend_workspace_bytes(const tq_attend_args* a, size_t* 
     return TQ_OK;
 }
 
+extern "C" tq_status tq_attend_window_workspace_bytes(const tq_attend_args* a, const tq_attend_window* w, size_t* bytes) {
+    clear_error();
+    if (!bytes) return fail(TQ_ERR_INVALID_ARG, "tq_attend_window_workspace_bytes: bytes is NULL");
+    *bytes = 0;
+    tq_status s = check_window("tq_attend_window_workspace_bytes", w);
+    if (s != TQ_OK) return s;
+    AttendPlan plan;
+    if ((s = plan_attend(a, &plan, true)) != TQ_OK) return s;
+    *bytes = plan.workspace_bytes;
+    return TQ_OK;
+}
+
 extern "C" tq_status tq_attend_decode(const tq_codec* c, const tq_attend_args* a, void* stream) {
     clear_error();
-    if (!c) return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: codec is NULL");
-    AttendPlan plan;
-    tq_status s = plan_attend(a, &plan);
-    if (s != TQ_OK) return s;
-    if (a->head_dim != c->d) return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: head_dim=%d but the codec has d=%d", a->head_dim, c->d);
-    if (!a->q || !a->k_packed || !a->k_norms || !a->v_data || !a->v_scales || !a->v_zeros || !a->out)
-        return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: NULL pointer in args");
-    if (!a->workspace || a->workspace_bytes < plan.workspace_bytes)
-        return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: workspace of %zu bytes required (got %zu)",
-                    plan.workspace_bytes, a->workspace ? a->workspace_bytes : static_cast<size_t>(0));
-    if (!aligned(a->q, 16) || !aligned(a->k_packed, 16) || !aligned(a->k_norms, 16) || !aligned(a->v_data, 16) ||
-        !aligned(a->v_scales, 16) || !aligned(a->v_zeros, 16) || !aligned(a->out, 16) || !aligned(a->workspace, 16))
-        return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode: every pointer must be 16-byte aligned");
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (c->d * 10 + c->bits) {
-        case 641: return attend_v<64, 1>(c, a, plan, st);
-        case 642: return attend_v<64, 2>(c, a, plan, st);
-        case 643: return attend_v<64, 3>(c, a, plan, st);
-        case 644: return attend_v<64, 4>(c, a, plan, st);
-        case 1281: return attend_v<128, 1>(c, a, plan, st);
-        case 1282: return attend_v<128, 2>(c, a, plan, st);
-        case 1283: return attend_v<128, 3>(c, a, plan, st);
-        case 1284: return attend_v<128, 4>(c, a, plan, st);
-        case 2561: return attend_v<256, 1>(c, a, plan, st);
-        case 2562: return attend_v<256, 2>(c, a, plan, st);
-        case 2563: return attend_v<256, 3>(c, a, plan, st);
-        case 2564: return attend_v<256, 4>(c, a, plan, st);
-        default: return fail(TQ_ERR_UNSUPPORTED, "tq_attend_decode: d=%d bits=%d", c->d, c->bits);
-    }
+    return attend_decode_impl("tq_attend_decode", c, a, nullptr, stream);
+}
+
+extern "C" tq_status tq_attend_decode_window(const tq_codec* c, const tq_attend_args* a, const tq_attend_window* w,
+                                             void* stream) {
+    clear_error();
+    if (!w) return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode_window: window is NULL");
+    return attend_decode_impl("tq_attend_decode_window", c, a, w, stream);
 }
 
 // ---------------------------------------------------------------------- attention without allocation

@@ -39,6 +39,11 @@ class AttendArgs(ctypes.Structure):
 
 
 # name -> (restype, argtypes)
+class AttendWindow(ctypes.Structure):
+    """Mirror of tq_attend_window."""
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("lens", ctypes.c_void_p), ("max_len", ctypes.c_int)]
+
+
 SIGNATURES = {
     "tq_last_error": (ctypes.c_char_p, []),
     "tq_version": (ctypes.c_int, []),
@@ -65,6 +70,10 @@ SIGNATURES = {
     "tq_attend_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(AttendArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "tq_attend_decode": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs), ctypes.c_void_p]),
     "tq_attend_decode_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs), ctypes.c_void_p]),
+    "tq_attend_window_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(AttendArgs), ctypes.POINTER(AttendWindow),
+                                                        ctypes.POINTER(ctypes.c_size_t)]),
+    "tq_attend_decode_window": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs),
+                                               ctypes.POINTER(AttendWindow), ctypes.c_void_p]),
     "tq_read_device_flag": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), ctypes.c_int]),
 }
 
@@ -245,6 +254,25 @@ class Cache:
     v_zeros: torch.Tensor
 
 
+ATTEND_WINDOW_MAX = 256
+
+
+def _window(win_k: torch.Tensor, win_v: torch.Tensor, win_lens: torch.Tensor | None, q) -> AttendWindow:
+    _need_cuda(win_k, "win_k", torch.float16)
+    _need_cuda(win_v, "win_v", torch.float16)
+    if win_k.dim() != 4 or win_k.shape != win_v.shape or not win_k.is_contiguous() or not win_v.is_contiguous():
+        raise ValueError("win_k and win_v must be contiguous [B, H_kv, W, d] fp16 tensors of one shape")
+    if win_k.shape[0] != q.shape[0] or win_k.shape[3] != q.shape[2]:
+        raise ValueError("the window's batch and head_dim must match q")
+    w = AttendWindow()
+    w.k, w.v = win_k.data_ptr(), win_v.data_ptr()
+    if win_lens is not None:
+        _need_cuda(win_lens, "win_lens", torch.int32)
+    w.lens = win_lens.data_ptr() if win_lens is not None else None
+    w.max_len = win_k.shape[2]
+    return w
+
+
 def _attend_args(codec: Codec, q, cache: Cache, *, num_kv_heads, v_bits, v_group, max_seq_len, block_table,
                  seq_lens, scale, out, workspace):
     b, hq, d = q.shape
@@ -277,20 +305,40 @@ def attend_workspace(codec: Codec, q, cache: Cache, **kw) -> torch.Tensor:
     return torch.empty(max(16, attend_workspace_bytes(codec, q, cache, **kw)), dtype=torch.uint8, device=q.device)
 
 
+def attend_window_workspace(codec: Codec, q, cache: Cache, win_k, win_v, win_lens=None, **kw) -> torch.Tensor:
+    """A workspace of the size tq_attend_window_workspace_bytes asks for."""
+    a = _attend_args(codec, q, cache, out=None, workspace=None, **kw)
+    w = _window(win_k, win_v, win_lens, q)
+    nb = ctypes.c_size_t()
+    _check("tq_attend_window_workspace_bytes",
+           LIB.tq_attend_window_workspace_bytes(ctypes.byref(a), ctypes.byref(w), ctypes.byref(nb)))
+    return torch.empty(max(16, nb.value), dtype=torch.uint8, device=q.device)
+
+
 def attend_decode(codec: Codec, q: torch.Tensor, cache: Cache, *, num_kv_heads: int, v_bits: int, v_group: int = 32,
                   max_seq_len: int | None = None, block_table: torch.Tensor | None = None,
                   seq_lens: torch.Tensor | None = None, scale: float = 0.0, out: torch.Tensor | None = None,
-                  workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """One decode step: q [B, H_q, d] fp16 against the compressed cache.  Returns out [B, H_q, d] f32."""
+                  workspace: torch.Tensor | None = None, win_k: torch.Tensor | None = None,
+                  win_v: torch.Tensor | None = None, win_lens: torch.Tensor | None = None) -> torch.Tensor:
+    """One decode step: q [B, H_q, d] fp16 against the compressed cache, plus (win_k, win_v: [B, H_kv, W, d]
+    fp16, win_lens: [B] int32 or None) a window of recent uncompressed tokens.  Returns out [B, H_q, d] f32."""
     _need_cuda(q, "q", torch.float16)
     kw = dict(num_kv_heads=num_kv_heads, v_bits=v_bits, v_group=v_group, max_seq_len=max_seq_len,
               block_table=block_table, seq_lens=seq_lens, scale=scale)
     if out is None:
         out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    if win_k is None:
+        if workspace is None:
+            workspace = attend_workspace(codec, q, cache, **kw)
+        a = _attend_args(codec, q, cache, out=out, workspace=workspace, **kw)
+        _check("tq_attend_decode", LIB.tq_attend_decode(codec.handle, ctypes.byref(a), _stream(q.device)))
+        return out
     if workspace is None:
-        workspace = attend_workspace(codec, q, cache, **kw)
+        workspace = attend_window_workspace(codec, q, cache, win_k, win_v, win_lens, **kw)
     a = _attend_args(codec, q, cache, out=out, workspace=workspace, **kw)
-    _check("tq_attend_decode", LIB.tq_attend_decode(codec.handle, ctypes.byref(a), _stream(q.device)))
+    w = _window(win_k, win_v, win_lens, q)
+    _check("tq_attend_decode_window", LIB.tq_attend_decode_window(codec.handle, ctypes.byref(a), ctypes.byref(w),
+                                                                  _stream(q.device)))
     return out
 
 

@@ -48,6 +48,25 @@ def test_hadamard_rotation_matches_oracle(d):
     assert np.array_equal(pi16.astype(np.float64), o.operational_rotation(d, 17, "hadamard"))
 
 
+def test_window_argument_errors():
+    a = tq.AttendArgs()
+    a.batch, a.num_q_heads, a.num_kv_heads, a.head_dim, a.v_bits, a.v_group = 1, 8, 1, 128, 2, 32
+    a.max_seq_len = 64
+    nb = ctypes.c_size_t(7)
+    assert tq.LIB.tq_attend_window_workspace_bytes(ctypes.byref(a), None, ctypes.byref(nb)) == tq.TQ_ERR_INVALID_ARG
+    w = tq.AttendWindow()
+    for bad in (0, tq.ATTEND_WINDOW_MAX + 1):
+        w.max_len = bad
+        assert tq.LIB.tq_attend_window_workspace_bytes(ctypes.byref(a), ctypes.byref(w), ctypes.byref(nb)) == \
+            tq.TQ_ERR_INVALID_ARG
+        assert b"max_len" in tq.LIB.tq_last_error()
+    w.max_len = 128
+    assert tq.LIB.tq_attend_window_workspace_bytes(ctypes.byref(a), ctypes.byref(w), ctypes.byref(nb)) == tq.TQ_OK
+    # one split plus the window's partial, after the prepared query
+    assert nb.value == (128 // 16 * 32 + 2) * 16 + 2 * (16 + 8 * 128) * 4
+    assert tq.LIB.tq_attend_decode_window(None, ctypes.byref(a), ctypes.byref(w), None) == tq.TQ_ERR_INVALID_ARG
+
+
 def test_rotation_kind_errors():
     out = np.empty(96 * 96)
     assert tq.LIB.tq_make_rotation_ex(96, 0, tq.TQ_ROT_HADAMARD, out.ctypes.data, None) == tq.TQ_ERR_INVALID_ARG
