@@ -294,8 +294,15 @@ def gpu_arm(args, w, rank, world, local_rank):
     qfrag_bytes = b * hkv * ((d // 16) * 32 + 2) * 16
     per_call = {"attend": 3 if ws.numel() > qfrag_bytes else 2}
     launches = sum(per_call.get(name, 1) for name, _, _ in events)
+    fid = None
+    if args.fidelity:
+        # logits of the compressed path vs the exact fp16 ones, over every (sequence, query head) of the step
+        from kv_cache_vector_norm_b200 import fidelity
+        codec.encode_k(k, packed=kp, norms=kn)
+        approx = tq.attend_scores(codec, q, cache, **{kk: vv for kk, vv in akw.items() if not kk.startswith("win_")})
+        fid = fidelity.score_fidelity(approx, fidelity.exact_scores(q, k.view(b, hkv, t, d)))
     return dict(per=per, ms_per_step=ms_per_step, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, n=n,
-                clocks=sampler.summary(), launches=launches)
+                clocks=sampler.summary(), launches=launches, fidelity=fid)
 
 
 # ------------------------------------------------------------------------------------- CPU (oracle)
@@ -363,6 +370,8 @@ def main():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--workload", default="70b_decode_128k", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fidelity", action="store_true",
+                    help="also report the attention-score fidelity (cosine, top-1, top-5) of the workload's cache")
     ap.add_argument("--window", type=int, default=0,
                     help="recent uncompressed tokens per (sequence, kv head) attended beside the compressed cache")
     ap.add_argument("--rotation", default="haar", choices=["haar", "hadamard"],
@@ -452,6 +461,8 @@ def main():
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"], "clocks": r["clocks"],
     }
+    if r.get("fidelity") is not None:
+        line["fidelity"] = r["fidelity"]
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line))

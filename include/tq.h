@@ -258,6 +258,19 @@ tq_status tq_attend_workspace_bytes(const tq_attend_args* args, size_t* bytes);
  */
 tq_status tq_attend_decode(const tq_codec* codec, const tq_attend_args* args, void* stream);
 
+/*
+ * tq_attend_scores -- the attention logits of the compressed path, for score-fidelity measurements
+ * ("turboquant-pytorch", V3: Attention Score Accuracy -- cosine similarity and top-1 / top-5 matches of the
+ * scores against the uncompressed ones): s[b][hq][t] = scale * n_t * <Pi_op q, c_op[idx_t]> in fp32, the
+ * same scores tq_attend_decode softmaxes.
+ *   scores  out, device float [batch][num_q_heads][L], L = max_seq_len (contiguous) or max_blocks * 16
+ *           (paged); positions at or past a sequence's length are -inf.
+ * args->out and the value pool are not used; args->workspace needs at least tq_attend_workspace_bytes bytes
+ * (only its prepared-query part is written).
+ * Errors: as tq_attend_decode.
+ */
+tq_status tq_attend_scores(const tq_codec* codec, const tq_attend_args* args, float* scores, void* stream);
+
 /* --------------------------------------------------------------------------------------------------
  * Attention with a window of recent uncompressed tokens.
  * ------------------------------------------------------------------------------------------------ */

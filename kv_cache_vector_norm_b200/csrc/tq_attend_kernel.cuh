@@ -747,6 +747,91 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
     }
 }
 
+// Attention logits of the compressed path, for score-fidelity measurements: s[b][hq][t] = scale * n_t *
+// <Pi_op q, c_op[idx_t]> (natural-log units) for t < len, -inf for len <= t < score_len.  Grid
+// (ceil(chunks / 4), H_kv, B), 4 warps, one 16-token chunk each; the score contraction is the split kernel's
+// (query fragments from attend_prep_kernel, code pairs from a per-bank replicated table, mma.sync).
+template <int D, int KB>
+__global__ void __launch_bounds__(128) attend_scores_kernel(const AttendParams p, float* __restrict__ scores,
+                                                            int64_t score_len) {
+    constexpr int KS = D / 16;
+    constexpr int kKRow = D * KB / 8;
+    constexpr int kQuarterHalves = D * KB / 4 / 16;
+    constexpr int kQuarterWords = (kQuarterHalves + 1) / 2 + 1;
+    constexpr int kPairs = 1 << (2 * KB);
+    extern __shared__ __align__(16) uint8_t smem[];
+    const uint32_t lut_addr = (smem_u32(smem) + kPairs * 128 - 1) & ~static_cast<uint32_t>(kPairs * 128 - 1);
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + (lut_addr - smem_u32(smem)));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int G = p.group;
+    for (int i = threadIdx.x; i < kPairs * 32; i += blockDim.x) lut[i] = __ldg(p.pair_lut + (i >> 5));
+    __syncthreads();
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();
+    const float unpre = __ldcg(reinterpret_cast<const float*>(qf + KS * 32) + gid);
+    const int64_t T = p.seq_lens ? static_cast<int64_t>(p.seq_lens[b]) : p.max_seq_len;
+    const int64_t chunk = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+    if (chunk * 16 >= score_len) return;
+    // this lane's quarter of the key rows of tokens 8 nt + gid (zero past the sequence)
+    uint32_t w[2][kQuarterWords];
+    float nrm[2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int64_t tk = chunk * 16 + 8 * nt + gid;
+#pragma unroll
+        for (int i = 0; i < kQuarterWords; ++i) w[nt][i] = 0u;
+        nrm[nt] = 0.f;
+        if (tk < T) {
+            const int64_t row = p.block_table
+                ? (static_cast<int64_t>(p.block_table[static_cast<int64_t>(b) * p.max_blocks + tk / 16]) * p.num_kv_heads + h) * 16 + tk % 16
+                : (static_cast<int64_t>(b) * p.num_kv_heads + h) * p.max_seq_len + tk;
+            const uint16_t* k16 = reinterpret_cast<const uint16_t*>(p.k_packed + row * kKRow) + tig * kQuarterHalves;
+#pragma unroll
+            for (int i = 0; i < kQuarterWords; ++i) {
+                const uint32_t lo16 = (2 * i < kQuarterHalves) ? k16[2 * i] : 0u;
+                const uint32_t hi16 = (2 * i + 1 < kQuarterHalves) ? k16[2 * i + 1] : 0u;
+                w[nt][i] = lo16 | (hi16 << 16);
+            }
+            nrm[nt] = p.k_norms[row];
+        }
+    }
+    const uint32_t lane_addr = lut_addr + 4u * lane;
+    constexpr uint32_t kFieldMask = static_cast<uint32_t>(kPairs - 1) << 7;
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+        const uint4 a = __ldcg(qf + ks * 32 + lane);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t e0 = window_shr(w[nt], 4 * ks * KB - 7) & kFieldMask;
+            const uint32_t e1 = window_shr(w[nt], (4 * ks + 2) * KB - 7) & kFieldMask;
+            mma_f16(sc[nt], a, lds_u32(lane_addr | e0), lds_u32(lane_addr | e1));
+        }
+    }
+    // C columns 2 tig, 2 tig + 1 of n-tile nt are tokens 8 nt + 2 tig (+1), whose norms sit in lanes 4 (2 tig + k)
+    float tn[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) tn[nt][k] = __shfl_sync(0xffffffffu, nrm[nt], 4 * (2 * tig + k));
+    }
+    if (gid < G) {
+        float* srow = scores + (static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * G + gid) * score_len;
+        constexpr float kLn2 = 0.69314718055994530942f;   // the fragments carry scale * log2(e)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int64_t t = chunk * 16 + 8 * nt + 2 * tig + k;
+                if (t < score_len)
+                    srow[t] = (t < T) ? (sc[nt][k] + sc[nt][k + 2]) * unpre * tn[nt][k] * kLn2 : -INFINITY;
+            }
+        }
+    }
+}
+
 // Split-K merge: out[b][h*G+g][:] = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M), M = max_s m_s.
 // One CTA per (g, h, b).  Slice k of the CTA's threads (D threads, one per column) folds splits k, k + kSlices,
 // ... with every load issued before the first is used, so the partials cost one round trip; the slices are

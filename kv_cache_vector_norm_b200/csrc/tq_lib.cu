@@ -615,6 +615,71 @@ tq_status attend_decode_impl(const char* fn, const tq_codec* c, const tq_attend_
 
 }  // namespace
 
+namespace {
+
+template <int D, int KB>
+tq_status launch_scores(const tq_codec* c, const tq_attend_args* a, const AttendPlan& plan, float* scores,
+                        int64_t score_len, cudaStream_t st) {
+    static std::atomic<uint64_t> mask{0};
+    auto kern = attend_scores_kernel<D, KB>;
+    const uint32_t smem = 2u * (1u << (2 * KB)) * 128u;
+    TQ_CUDA(allow_smem(kern, smem, mask), "tq_attend_scores: cudaFuncSetAttribute");
+    AttendParams p = {};
+    p.batch = a->batch;
+    p.num_q_heads = a->num_q_heads;
+    p.num_kv_heads = a->num_kv_heads;
+    p.group = a->num_q_heads / a->num_kv_heads;
+    const float scale = (a->scale == 0.f) ? 1.0f / std::sqrt(static_cast<float>(D)) : a->scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.max_seq_len = a->max_seq_len;
+    p.block_table = a->block_table;
+    p.max_blocks = a->max_blocks;
+    p.seq_lens = a->seq_lens;
+    p.q = static_cast<const __half*>(a->q);
+    p.pi_op = c->pi_op;
+    p.pair_lut = c->pair_lut;
+    p.k_packed = a->k_packed;
+    p.k_norms = a->k_norms;
+    p.qfrag = static_cast<uint4*>(a->workspace);
+    p.num_splits = p.num_parts = 1;
+    attend_prep_kernel<D><<<dim3(D / 32, a->num_kv_heads, a->batch), kPrepThreads, 0, st>>>(p);
+    TQ_CUDA(cudaGetLastError(), "tq_attend_scores: query preparation launch");
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((score_len + 63) / 64), a->num_kv_heads, a->batch);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    TQ_CUDA(cudaLaunchKernelEx(&cfg, kern, p, scores, score_len), "tq_attend_scores: launch");
+    return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" tq_status tq_attend_scores(const tq_codec* c, const tq_attend_args* a, float* scores, void* stream) {
+    clear_error();
+    if (!c) return fail(TQ_ERR_INVALID_ARG, "tq_attend_scores: codec is NULL");
+    AttendPlan plan;
+    tq_status s = plan_attend(a, &plan);
+    if (s != TQ_OK) return s;
+    if (a->head_dim != c->d) return fail(TQ_ERR_INVALID_ARG, "tq_attend_scores: head_dim=%d but the codec has d=%d", a->head_dim, c->d);
+    if (!a->q || !a->k_packed || !a->k_norms || !scores)
+        return fail(TQ_ERR_INVALID_ARG, "tq_attend_scores: q, k_packed, k_norms and scores must be non-NULL");
+    if (!a->workspace || a->workspace_bytes < plan.qfrag_bytes)
+        return fail(TQ_ERR_INVALID_ARG, "tq_attend_scores: workspace of %zu bytes required (got %zu)", plan.qfrag_bytes,
+                    a->workspace ? a->workspace_bytes : static_cast<size_t>(0));
+    if (!aligned(a->q, 16) || !aligned(a->k_norms, 4) || !aligned(a->workspace, 16) || !aligned(scores, 4))
+        return fail(TQ_ERR_INVALID_ARG, "tq_attend_scores: q and workspace must be 16-byte aligned");
+    const int64_t score_len = a->block_table ? static_cast<int64_t>(a->max_blocks) * 16 : a->max_seq_len;
+    if (score_len == 0) return TQ_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TQ_DISPATCH_DB(c->d, c->bits, launch_scores, c, a, plan, scores, score_len, st);
+}
+
 extern "C" tq_status tq_attend_workspace_bytes(const tq_attend_args* a, size_t* bytes) {
     clear_error();
     if (!bytes) return fail(TQ_ERR_INVALID_ARG, "tq_attend_workspace_bytes: bytes is NULL");

@@ -70,6 +70,7 @@ SIGNATURES = {
     "tq_attend_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(AttendArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "tq_attend_decode": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs), ctypes.c_void_p]),
     "tq_attend_decode_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs), ctypes.c_void_p]),
+    "tq_attend_scores": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs), ctypes.c_void_p, ctypes.c_void_p]),
     "tq_attend_window_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(AttendArgs), ctypes.POINTER(AttendWindow),
                                                         ctypes.POINTER(ctypes.c_size_t)]),
     "tq_attend_decode_window": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs),
@@ -340,6 +341,24 @@ def attend_decode(codec: Codec, q: torch.Tensor, cache: Cache, *, num_kv_heads: 
     _check("tq_attend_decode_window", LIB.tq_attend_decode_window(codec.handle, ctypes.byref(a), ctypes.byref(w),
                                                                   _stream(q.device)))
     return out
+
+
+def attend_scores(codec: Codec, q: torch.Tensor, cache: Cache, *, num_kv_heads: int, v_bits: int, v_group: int = 32,
+                  max_seq_len: int | None = None, block_table: torch.Tensor | None = None,
+                  seq_lens: torch.Tensor | None = None, scale: float = 0.0,
+                  workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """The compressed path's attention logits [B, H_q, L] f32 (L = max_seq_len, or max_blocks * 16 when paged);
+    -inf past each sequence's length."""
+    _need_cuda(q, "q", torch.float16)
+    kw = dict(num_kv_heads=num_kv_heads, v_bits=v_bits, v_group=v_group, max_seq_len=max_seq_len,
+              block_table=block_table, seq_lens=seq_lens, scale=scale)
+    length = block_table.shape[1] * 16 if block_table is not None else int(max_seq_len)
+    scores = torch.empty((q.shape[0], q.shape[1], length), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = attend_workspace(codec, q, cache, **kw)
+    a = _attend_args(codec, q, cache, out=None, workspace=workspace, **kw)
+    _check("tq_attend_scores", LIB.tq_attend_scores(codec.handle, ctypes.byref(a), scores.data_ptr(), _stream(q.device)))
+    return scores
 
 
 ATTEND_SCRATCH_BYTES = 4 << 20

@@ -43,3 +43,17 @@ def test_channel_scales_and_block_table():
     assert torch.all((sc > 20 * torch.exp(torch.tensor(-3.0))).sum(1) >= 1)
     bt = synth.block_table(0, 4, 8, 40)
     assert bt.shape == (4, 8) and len(set(bt.flatten().tolist())) == 32 and int(bt.max()) < 40
+
+
+def test_score_fidelity_metrics_on_known_cases():
+    from kv_cache_vector_norm_b200 import fidelity
+    e = torch.tensor([[[1.0, 5.0, 2.0, 0.5, 0.1, 3.0]]])
+    m = fidelity.score_fidelity(e.clone(), e)
+    assert abs(m["cosine"] - 1.0) < 1e-12 and m["top1"] == 1.0 and m["top5"] == 1.0
+    a = torch.tensor([[[1.0, 2.9, 2.0, 0.5, 0.1, 3.0]]])          # argmax moves to the last token
+    m = fidelity.score_fidelity(a, e)
+    ev, av = e.double().numpy().ravel(), a.double().numpy().ravel()
+    assert abs(m["cosine"] - ev @ av / (np.linalg.norm(ev) * np.linalg.norm(av))) < 1e-12
+    assert m["top1"] == 0.0 and m["top5"] == 1.0
+    assert fidelity.score_fidelity(a, e, k=1)["top1"] == 0.0
+    assert fidelity.score_fidelity(a, e, seq_lens=[0])["pairs"] == 0
