@@ -160,6 +160,22 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------------------ GPU arm
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest of every rank's x (the job's time is its slowest rank's); x itself with one rank."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, units_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput in M units/s: every rank processes units_per_rank per step (weak scaling)."""
+    return world * units_per_rank / (ms_per_step / 1000.0) / 1e6
+
+
 def gpu_arm(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -243,11 +259,7 @@ def gpu_arm(args, w, rank, world, local_rank):
         per[name] += e0.elapsed_time(e1)
     if args.only:
         return dict(per=per, launch_ms=[e0.elapsed_time(e1) for _, e0, e1 in events], n=n)
-    total_ms = sum(per.values())
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(per.values()), world, dev)
     ms_per_step = total_ms / args.steps
 
     # ---------------------------------------------------------------- end to end through host buffers
@@ -280,11 +292,7 @@ def gpu_arm(args, w, rank, world, local_rank):
         e2e_step()
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
     h2d = (k_host.numel() + v_host.numel() + q_host.numel()) * 2
     d2h = (kdec_host.numel() + vdec_host.numel()) * 2 + out_host.numel() * 4
     if tq.read_device_flag() != 0:
@@ -446,7 +454,7 @@ def main():
         kern[name] = {"ms": ms, "Mvectors_s": units / (ms / 1000.0) / 1e6, "GBps": gbps, "frac_of_hbm": gbps / hbm,
                       "bytes_per_vector": bpv[name]}
     dom = max(kern, key=lambda x: kern[x]["ms"])
-    value = world * n / (r["ms_per_step"] / 1000.0) / 1e6
+    value = job_value(world, n, r["ms_per_step"])
     line = {
         "metric": METRIC, "value": value, "unit": "Mvectors/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
@@ -457,7 +465,7 @@ def main():
                      "frac": kern[dom]["GBps"] / hbm, "peak_source": peak_src,
                      "traffic": traffic_record(dom, args.workload),
                      "algorithmic_bytes_per_launch": bpv[dom] * n},
-        "e2e": {"value": world * n / (r["e2e_ms"] / 1000.0) / 1e6, "unit": "Mvectors/s",
+        "e2e": {"value": job_value(world, n, r["e2e_ms"]), "unit": "Mvectors/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"], "clocks": r["clocks"],
     }
