@@ -606,3 +606,105 @@ def paged_rows(block_table: np.ndarray, b: int, h: int, length: int, num_kv_head
     p = np.arange(length)
     blocks = np.asarray(block_table)[b, p // block_size].astype(np.int64)
     return (blocks * num_kv_heads + h) * block_size + (p % block_size)
+
+
+# ----------------------------------------------------------------------------------------------
+# QJL residual keys  ([P3] compressors.py, TurboQuantCompressorV2: __init__, compress and
+# asymmetric_attention_scores; store.py TurboQuantKVCache.attention_scores uses that estimator for
+# the quantized part).  Stage 1 is the MSE key codec at bits - 1 (at least 1); stage 2 keeps one sign
+# bit per coordinate of S r, r the residual in the original space, and ||r||.
+# Readings: S is a d x d matrix of standard normal draws taken from this build's generator with seed
+# + 10000 (the page's offset; its torch stream is not reproduced); the multiply uses S_op = fp16(S),
+# as the rotation uses Pi_op; a sign bit is 1 for +1 (S r >= 0, zero included, as the page's
+# ``projected >= 0``); ||r|| is stored in f32 like the key norm (the page keeps both in fp16).
+# ----------------------------------------------------------------------------------------------
+
+QJL_SEED_OFFSET = 10000
+
+
+def qjl_mse_bits(bits: int) -> int:
+    """Bits of the MSE stage of a ``bits``-bit QJL key: max(bits - 1, 1)."""
+    return max(bits - 1, 1)
+
+
+def qjl_matrix(d: int, seed: int) -> np.ndarray:
+    """S (d x d, fp64): Gaussian draws i*d + j of the generator seeded with seed + 10000."""
+    return gaussian_stream(seed + QJL_SEED_OFFSET, d * d).reshape(d, d)
+
+
+def operational_qjl_matrix(d: int, seed: int) -> np.ndarray:
+    """S_op = fp16(S) as fp64 values: the projection the tensor-core path multiplies by."""
+    return to_fp16_values(qjl_matrix(d, seed))
+
+
+def encode_k_qjl(x16: np.ndarray, pi_op: np.ndarray, c_op: np.ndarray, t: np.ndarray, s_op: np.ndarray,
+                 idx: np.ndarray | None = None):
+    """QJL key encode of fp16 rows x [N][d], in the page's order.
+
+    n = ||x||; y = Pi_op x / (n + 1e-8); idx = nearest level of the (bits-1)-bit codebook (c_op, t);
+    k_mse = n * Pi_op^T c_op[idx] (the reconstruction in the original space); r = x - k_mse;
+    rho = ||r||; proj = S_op r; sign bit = (proj >= 0).
+    ``idx`` may be given (e.g. another implementation's indices) to take r from those.
+    Returns (idx [N][d], n [N], y [N][d], bits [N][d] bool, rho [N], proj [N][d]).
+    """
+    x = np.asarray(x16).astype(np.float64)
+    n = np.sqrt(np.sum(x * x, axis=-1))
+    y = (x @ pi_op.T) / (n + 1e-8)[:, None]
+    if idx is None:
+        idx = nearest_index(y, t)
+    k_mse = n[:, None] * (c_op[np.asarray(idx)] @ pi_op)
+    r = x - k_mse
+    rho = np.sqrt(np.sum(r * r, axis=-1))
+    proj = r @ s_op.T
+    return np.asarray(idx), n, y, proj >= 0, rho, proj
+
+
+def qjl_inner_products(q: np.ndarray, idx: np.ndarray, norms: np.ndarray, sign_bits: np.ndarray, rho: np.ndarray,
+                       pi_op: np.ndarray, c_op: np.ndarray, s_op: np.ndarray) -> np.ndarray:
+    """The asymmetric estimate of <q, k_t> for one query q [d] and T keys:
+    <q, k_mse_t> + rho_t * sqrt(pi / 2) / m * <S_op q, signs_t>, signs in {-1, +1}, m = rows of S."""
+    q = np.asarray(q, dtype=np.float64)
+    term1 = decode_k(idx, norms, pi_op, c_op) @ q
+    pm = np.where(np.asarray(sign_bits, dtype=bool), 1.0, -1.0)
+    term2 = math.sqrt(math.pi / 2.0) / s_op.shape[0] * np.asarray(rho, dtype=np.float64) * (pm @ (s_op @ q))
+    return term1 + term2
+
+
+def attend_qjl(q16: np.ndarray, k_idx: np.ndarray, k_norms: np.ndarray, k_bits: np.ndarray, k_rho: np.ndarray,
+               v_hat: np.ndarray, pi_op: np.ndarray, c_op: np.ndarray, s_op: np.ndarray,
+               scale: float | None = None, seq_lens: np.ndarray | None = None, win_k16: np.ndarray | None = None,
+               win_v16: np.ndarray | None = None, win_lens: np.ndarray | None = None) -> np.ndarray:
+    """Decode attention whose compressed part is scored by the QJL estimator ([P3] store.py
+    ``attention_scores``: scale * the asymmetric scores of the quantized part, then scale * q . key_buffer
+    for the recent uncompressed window when there is one; softmax over both; weights @ values).
+
+    q16 [B][H_q][d]; k_idx, k_bits [B][H_kv][T][d]; k_norms, k_rho [B][H_kv][T]; v_hat [B][H_kv][T][d];
+    optional window win_k16, win_v16 [B][H_kv][W][d] fp16 with win_lens [B].  Returns o [B][H_q][d] fp64.
+    """
+    bsz, hq, d = q16.shape
+    hkv = k_idx.shape[1]
+    grp = hq // hkv
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = np.zeros((bsz, hq, d), dtype=np.float64)
+    for b in range(bsz):
+        tl = k_idx.shape[2] if seq_lens is None else int(seq_lens[b])
+        wl = 0 if win_k16 is None else (win_k16.shape[2] if win_lens is None else int(win_lens[b]))
+        for h in range(hq):
+            kv = h // grp
+            q = np.asarray(q16[b, h]).astype(np.float64)
+            s = scale * qjl_inner_products(q, k_idx[b, kv, :tl], k_norms[b, kv, :tl], k_bits[b, kv, :tl],
+                                           k_rho[b, kv, :tl], pi_op, c_op, s_op)
+            v_all = np.asarray(v_hat[b, kv, :tl], dtype=np.float64)
+            if wl:
+                s = np.concatenate([s, scale * (np.asarray(win_k16[b, kv, :wl]).astype(np.float64) @ q)])
+                v_all = np.concatenate([v_all, np.asarray(win_v16[b, kv, :wl]).astype(np.float64)], axis=0)
+            if s.shape[0] == 0:
+                continue
+            p = np.exp(s - s.max())
+            out[b, h] = (p / p.sum()) @ v_all
+    return out
+
+
+def qjl_key_row_bytes(d: int, bits: int, norm_bytes: int = 4) -> int:
+    """Bytes of one QJL key: (bits-1)-bit codes + d sign bits + the norm and the residual norm."""
+    return k_row_bytes(d, qjl_mse_bits(bits)) + d // 8 + 2 * norm_bytes
