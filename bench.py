@@ -386,10 +386,16 @@ def main():
                     help="key rotation: seeded Haar (default) or randomized Walsh-Hadamard; same kernels")
     ap.add_argument("--only", choices=["encode_k", "encode_v", "decode_k", "decode_v", "attend"],
                     help="time one kernel of the path alone (profiling aid; prints its per-launch times)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's cache length (a multiple of 16; profiling aid for small captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    w = WORKLOADS[args.workload]
+    w = dict(WORKLOADS[args.workload])
+    if args.tokens > 0:
+        if args.tokens % 16:
+            ap.error("--tokens must be a multiple of 16")
+        w["tokens"] = args.tokens
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

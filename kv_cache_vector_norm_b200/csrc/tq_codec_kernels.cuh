@@ -332,12 +332,14 @@ constexpr float kGridScale = static_cast<float>(kGridRes);
 constexpr float kGridMagic = 12582912.0f + kGridOffset;   // 1.5 * 2^23 + 128
 
 
-// Encode CTA: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-3 compute the row norms of
-// each X stage ahead of the epilogue, warps 4.. are the epilogue (kEncEpiWarps: warp w reads TMEM lanes
-// 32*(w%4).. and owns kEncCols columns of them).
+
+// Encode CTA: warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2-5 compute the row norms of
+// each X stage ahead of the epilogue (one row per thread), warps 6.. are the epilogue (kEpiWarps: warp w
+// reads TMEM lanes 32*(w%4).. and owns kCols columns of them).
 template <int D>
 struct EncCfg {
-    static constexpr int kNormWarps = 2;
+    static constexpr int kNormWarps = 4;                     // one row per norm thread: the norms keep ahead
+    static constexpr int kNormRows = 128 / (32 * kNormWarps);   // rows per norm thread per tile
     static constexpr int kEpiWarps = (D == 64) ? 8 : 16;
     static constexpr int kFirstEpi = 2 + kNormWarps;
     static constexpr int kThreads = 32 * (kFirstEpi + kEpiWarps);
@@ -469,7 +471,7 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         }
     } else if (warp < E::kFirstEpi) {
         // -------------------------------------------------------------------- row norms, ahead of the epilogue
-        const int t = (warp - 2) * 32 + lane;                 // rows t and t + 64 of each tile
+        const int t = (warp - 2) * 32 + lane;                 // rows t, t + 32 kNormWarps, ... of each tile
         int li = 0;
         for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
             const int s = li % S;
@@ -477,8 +479,8 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
             if (!mbar_wait(b_nfree + 8 * s, ((li / S) & 1) ^ 1, abort_flag)) break;
             const uint8_t* xs = s_x + s * C::kTileBytes;
 #pragma unroll
-            for (int hrow = 0; hrow < 2; ++hrow) {
-                const int r = t + 64 * hrow;
+            for (int hrow = 0; hrow < E::kNormRows; ++hrow) {
+                const int r = t + 32 * E::kNormWarps * hrow;
                 float acc[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -555,11 +557,13 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                     const uint32_t cell[2] = {__float_as_uint(g2.x), __float_as_uint(g2.y)};
 #pragma unroll
                     for (int e2 = 0; e2 < 2; ++e2) {
-                        const uint32_t e = lds_u32(lut_lane + (cell[e2] & (C::kLutEntries - 1)) * 128u);
+                        const uint32_t e = lds_u32(lut_lane + ((cell[e2] & (C::kLutEntries - 1)) << 7));
                         // the entry read as a float is the cell's boundary moved by at most 15 ulps (its low 4 bits
-                        // hold the count; the boundary's own low bits are zero), or a NaN / +inf when it has none
-                        const uint32_t idx = (e & 15u) + (yv[e2] > __uint_as_float(e) ? 1u : 0u);
-                        add_field<BITS>(w, 2 * j2 + e2, idx);
+                        // hold the count; the boundary's own low bits are zero), or +inf / a NaN when it has none.
+                        // The sign of (boundary - y) is set exactly when y lies above the boundary (ties stay below);
+                        // +inf - y is +inf and NaN - y the canonical, positive NaN.
+                        const uint32_t above = __float_as_uint(__fsub_rn(__uint_as_float(e), yv[e2])) >> 31;
+                        add_field<BITS>(w, 2 * j2 + e2, (e & 15u) + above);
                     }
                 }
                 const int boff = (c0 + k * 32) * BITS / 8;
@@ -627,12 +631,18 @@ struct DecLayout {
     static constexpr uint32_t kA = kPit + C::kPiBytes;
     static constexpr uint32_t kIn = kA + C::kDecBufs * C::kTileBytes;
     static constexpr uint32_t kPair = kIn + kInBufs * kInBytes;
-    // per-warp output patches: 32 rows x 64 bytes, 64B-swizzled, the source of one tensor store each
+    // where the slack fits, the replicated table is placed on a multiple of its size, so a lookup address is
+    // (pair bits << 7) | lane bits: one funnel shift and one LOP3 per lookup
     static constexpr int kPatchBufs = (D <= 128) ? 2 : 1;
     static constexpr uint32_t kPatchBytes = 32 * 64;
-    static constexpr uint32_t kPatch = (kPair + kPairBytes + 511) & ~511u;     // 64B swizzle repeats every 512 bytes
-    static constexpr uint32_t kBar = kPatch + E::kEpiWarps * kPatchBufs * kPatchBytes;
     static constexpr int kBars = 2 * C::kDecBufs + 2 * kInBufs + 8;
+    static constexpr uint32_t kTailBytes = E::kEpiWarps * kPatchBufs * kPatchBytes + 8 * kBars + 16 + 1024;
+    static constexpr bool kAlignPairs = kReplPairs &&
+        (((kPair + 2 * kPairBytes + 511) & ~511u) + kTailBytes <= 227 * 1024);
+    static constexpr uint32_t kPairRegion = kAlignPairs ? 2 * kPairBytes : kPairBytes;
+    // per-warp output patches: 32 rows x 64 bytes, 64B-swizzled, the source of one tensor store each
+    static constexpr uint32_t kPatch = (kPair + kPairRegion + 511) & ~511u;    // 64B swizzle repeats every 512 bytes
+    static constexpr uint32_t kBar = kPatch + E::kEpiWarps * kPatchBufs * kPatchBytes;
     static constexpr uint32_t kMisc = kBar + 8 * kBars;
     static constexpr uint32_t kBytes = kMisc + 16 + 1024;
     static_assert(kBytes <= 227 * 1024, "decode layout exceeds the shared memory of one CTA");
@@ -663,7 +673,10 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
     uint8_t* s_pit = smem + Lo::kPit;
     uint8_t* s_a = smem + Lo::kA;
     uint8_t* s_in = smem + Lo::kIn;
-    uint32_t* s_pair = reinterpret_cast<uint32_t*>(smem + Lo::kPair);
+    const uint32_t pair_base = Lo::kAlignPairs
+        ? (smem_u32(smem + Lo::kPair) + Lo::kPairBytes - 1) & ~static_cast<uint32_t>(Lo::kPairBytes - 1)
+        : smem_u32(smem + Lo::kPair);
+    uint32_t* s_pair = reinterpret_cast<uint32_t*>(smem + (pair_base - smem_u32(smem)));
     const uint32_t bar0 = smem_u32(smem + Lo::kBar);
     const uint32_t b_afull = bar0, b_aempty = b_afull + 8 * NB, b_infull = b_aempty + 8 * NB,
                    b_inempty = b_infull + 8 * NI, b_accfull = b_inempty + 8 * NI, b_accempty = b_accfull + 16,
@@ -764,7 +777,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
         const int c0 = (ew >> 2) * E::kCols;               // first column of this warp
         const int r = quarter * 32 + lane;
         uint8_t* patches = smem + Lo::kPatch + ew * Lo::kPatchBufs * Lo::kPatchBytes;
-        const uint32_t pair_lane = smem_u32(s_pair) + 4u * lane;   // this lane's copy of the pair table
+        const uint32_t pair_lane = pair_base + 4u * lane;          // this lane's copy of the pair table
         int pcount = 0;                                    // tensor stores issued by this warp
         float nrm_next = 0.f;
 
@@ -775,7 +788,8 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
             if (!mbar_wait(b_infull + 8 * ib, (lt / NI) & 1, abort_flag)) return false;
             const int64_t rows = tile_rows(tile);
             const int64_t row = tile * 128 + r;
-            uint32_t w[kPartWords];
+            uint32_t w[kPartWords + 1];
+            w[kPartWords] = 0u;
             if (r < rows) {
                 if (bulk_ok(rows)) {
                     const uint8_t* src = s_in + ib * Lo::kInBytes + r * kRowBytes + c0 * BITS / 8;
@@ -783,7 +797,8 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
                     for (int i = 0; i < kPartWords; ++i) w[i] = reinterpret_cast<const uint32_t*>(src)[i];
                     nrm_next = reinterpret_cast<const float*>(s_in + ib * Lo::kInBytes + 128 * kRowBytes)[r];
                 } else {
-                    load_words<kPartWords>(packed + row * kRowBytes + c0 * BITS / 8, w);
+                    load_words<kPartWords>(packed + row * kRowBytes + c0 * BITS / 8,
+                                           *reinterpret_cast<uint32_t(*)[kPartWords]>(w));
                     nrm_next = norms[row];
                 }
             } else {
@@ -799,8 +814,13 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
                 uint32_t h[4];
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    const uint32_t key = get_bits<2 * BITS>(w, (c * 8 + 2 * p) * BITS);
-                    h[p] = Lo::kReplPairs ? lds_u32(pair_lane + key * 128u) : s_pair[key];
+                    if constexpr (Lo::kAlignPairs) {
+                        const uint32_t x = bits_shr(w, (c * 8 + 2 * p) * BITS - 7);
+                        h[p] = lds_u32((x & (static_cast<uint32_t>(kPairs - 1) << 7)) | pair_lane);
+                    } else {
+                        const uint32_t key = get_bits<2 * BITS>(w, (c * 8 + 2 * p) * BITS);
+                        h[p] = Lo::kReplPairs ? lds_u32(pair_lane + key * 128u) : s_pair[key];
+                    }
                 }
                 const int col = c0 + c * 8;
                 *reinterpret_cast<uint4*>(as + (col >> 6) * C::kTileBlockBytes + sw128_offset(r, (col & 63) >> 3)) =

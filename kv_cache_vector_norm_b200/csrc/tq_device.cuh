@@ -245,6 +245,15 @@ __device__ __forceinline__ uint32_t get_bits(const uint32_t (&w)[NW], int bit) {
     return (W == 32) ? v : (v & ((1u << W) - 1u));
 }
 
+// The little-endian bitstream `w` shifted right by `bit` (-31 <= bit; bit + 32 <= 32 NW), low 32 bits.
+template <int NW>
+__device__ __forceinline__ uint32_t bits_shr(const uint32_t (&w)[NW], int bit) {
+    if (bit < 0) return w[0] << (-bit);
+    const int wi = bit >> 5, sh = bit & 31;
+    if (sh == 0) return w[wi];
+    return (wi + 1 < NW) ? __funnelshift_r(w[wi], w[wi + 1], sh) : (w[wi] >> sh);
+}
+
 // Store NW words (4-byte aligned destination; wider vectors where NW allows and `dst` is aligned to them).
 template <int NW>
 __device__ __forceinline__ void store_words(uint8_t* dst, const uint32_t (&w)[NW]) {
