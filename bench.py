@@ -223,6 +223,10 @@ def gpu_arm(args, w, rank, world, local_rank):
     ]
 
     if args.only:
+        if args.only in ("decode_k", "decode_v", "attend"):
+            # the compressed cache these kernels read is written once, outside the timed launches
+            kernels[0][1]()
+            kernels[1][1]()
         kernels = [kv for kv in kernels if kv[0] == args.only]
 
     def one_step(record):
