@@ -627,9 +627,15 @@ struct DecLayout {
     // code-pair table: one copy per shared-memory bank (entry e of lane l at 128 e + 4 l) where it fits
     static constexpr bool kReplPairs = (D <= 128);
     static constexpr int kPairBytes = (1 << (2 * BITS)) * (kReplPairs ? 128 : 4);
+    // d <= 128: the A tile (the looked-up codebook values) is built in tensor memory with tcgen05.st and the MMA
+    // reads it from there, which takes its writes and the tensor core's reads off shared memory; d = 256 keeps
+    // it in shared memory (its two accumulators fill the 512 TMEM columns)
+    static constexpr bool kTmemA = (D <= 128);
+    static constexpr uint32_t kTmemCols = kTmemA ? (D == 128 ? 512 : 256) : C::kTmemCols;
+    static constexpr uint32_t kTmemACol = 2 * D;                              // A buffer b at 2 D + b D / 2
     static constexpr uint32_t kPit = 0;
     static constexpr uint32_t kA = kPit + C::kPiBytes;
-    static constexpr uint32_t kIn = kA + C::kDecBufs * C::kTileBytes;
+    static constexpr uint32_t kIn = kA + (kTmemA ? 0 : C::kDecBufs * C::kTileBytes);
     static constexpr uint32_t kPair = kIn + kInBufs * kInBytes;
     // where the slack fits, the replicated table is placed on a multiple of its size, so a lookup address is
     // (pair bits << 7) | lane bits: one funnel shift and one LOP3 per lookup
@@ -706,7 +712,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+        tmem_alloc(smem_u32(tmem_slot), Lo::kTmemCols);
         tmem_relinquish();
     }
     if constexpr (Lo::kReplPairs) {
@@ -757,13 +763,18 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
                 if (!mbar_wait(b_accempty + 8 * a, ((li >> 1) & 1) ^ 1, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + a * D;
-                const uint32_t aa = smem_u32(s_a + b * C::kTileBytes), pa = smem_u32(s_pit);
+                const uint32_t pa = smem_u32(s_pit);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k & 3) * 32;
-                    const uint64_t ad = desc_kmajor_sw128(aa + (k >> 2) * C::kTileBlockBytes + off);
                     const uint64_t bd = desc_kmajor_sw128(pa + (k >> 2) * C::kPiBlockBytes + off);
-                    umma_f16_ss(d_tmem, ad, bd, C::kIdesc, k > 0 ? 1u : 0u);
+                    if constexpr (Lo::kTmemA) {
+                        umma_f16_ts(d_tmem, tmem_base + Lo::kTmemACol + b * (D / 2) + 8 * k, bd, C::kIdesc, k > 0 ? 1u : 0u);
+                    } else {
+                        const uint32_t aa = smem_u32(s_a + b * C::kTileBytes);
+                        const uint64_t ad = desc_kmajor_sw128(aa + (k >> 2) * C::kTileBlockBytes + off);
+                        umma_f16_ss(d_tmem, ad, bd, C::kIdesc, k > 0 ? 1u : 0u);
+                    }
                 }
                 umma_commit(b_accfull + 8 * a);
                 umma_commit(b_aempty + 8 * b);
@@ -781,7 +792,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
         int pcount = 0;                                    // tensor stores issued by this warp
         float nrm_next = 0.f;
 
-        // build the A tile (c_op[idx] as fp16, 128B-swizzled K-major) for local tile index lt
+        // build the A tile (c_op[idx] as fp16: TMEM rows, or 128B-swizzled K-major smem) for local tile index lt
         auto build = [&](int lt, int64_t tile) -> bool {
             const int b = lt % NB, ib = lt % NI;
             if (!mbar_wait(b_aempty + 8 * b, ((lt / NB) & 1) ^ 1, abort_flag)) return false;
@@ -808,25 +819,44 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(b_inempty + 8 * ib);
-            uint8_t* as = s_a + b * C::kTileBytes;
-#pragma unroll
-            for (int c = 0; c < E::kCols / 8; ++c) {
-                uint32_t h[4];
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    if constexpr (Lo::kAlignPairs) {
-                        const uint32_t x = bits_shr(w, (c * 8 + 2 * p) * BITS - 7);
-                        h[p] = lds_u32((x & (static_cast<uint32_t>(kPairs - 1) << 7)) | pair_lane);
-                    } else {
-                        const uint32_t key = get_bits<2 * BITS>(w, (c * 8 + 2 * p) * BITS);
-                        h[p] = Lo::kReplPairs ? lds_u32(pair_lane + key * 128u) : s_pair[key];
-                    }
+            // one half2 of codebook values per code pair (two consecutive columns of the row)
+            auto pair_value = [&](int c, int p) -> uint32_t {
+                if constexpr (Lo::kAlignPairs) {
+                    const uint32_t x = bits_shr(w, (c * 8 + 2 * p) * BITS - 7);
+                    return lds_u32((x & (static_cast<uint32_t>(kPairs - 1) << 7)) | pair_lane);
+                } else {
+                    const uint32_t key = get_bits<2 * BITS>(w, (c * 8 + 2 * p) * BITS);
+                    return Lo::kReplPairs ? lds_u32(pair_lane + key * 128u) : s_pair[key];
                 }
-                const int col = c0 + c * 8;
-                *reinterpret_cast<uint4*>(as + (col >> 6) * C::kTileBlockBytes + sw128_offset(r, (col & 63) >> 3)) =
-                    make_uint4(h[0], h[1], h[2], h[3]);
+            };
+            if constexpr (Lo::kTmemA) {
+                static_assert(E::kCols == 32, "one 16-column TMEM store per warp and tile");
+                // the MMA that last read this A buffer has completed (aempty): order the stores after it
+                tc_fence_after();
+                uint32_t hc[16];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) hc[4 * c + p] = pair_value(c, p);
+                }
+                tmem_st_32x32b_x16(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + Lo::kTmemACol +
+                                       b * (D / 2) + c0 / 2,
+                                   hc);
+                tmem_st_wait();
+                tc_fence_before();
+            } else {
+                uint8_t* as = s_a + b * C::kTileBytes;
+#pragma unroll
+                for (int c = 0; c < E::kCols / 8; ++c) {
+                    uint32_t h[4];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) h[p] = pair_value(c, p);
+                    const int col = c0 + c * 8;
+                    *reinterpret_cast<uint4*>(as + (col >> 6) * C::kTileBlockBytes + sw128_offset(r, (col & 63) >> 3)) =
+                        make_uint4(h[0], h[1], h[2], h[3]);
+                }
+                fence_proxy_async_smem();
             }
-            fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(b_afull + 8 * b);
             return true;
@@ -909,7 +939,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::kTmemCols);
+        tmem_dealloc(tmem_base, Lo::kTmemCols);
     }
 }
 
