@@ -233,56 +233,87 @@ __global__ void __launch_bounds__(256) decode_v_kernel(const uint8_t* __restrict
     const int64_t step = warps_total * L::kRowsPerWarp;
     int64_t wrow = (static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + warp) * L::kRowsPerWarp;
     const int rl = lane / L::kRowLanes;
-    uint32_t c[4] = {0u, 0u, 0u, 0u};
-    __half s16 = __float2half_rn(0.f), z16 = s16;
-    if (wrow + rl < n) {
-        load_vchunk16<D, BITS>(data + (wrow + rl) * kRowBytes, j, c);
-        s16 = __ldg(scales + (wrow + rl) * kGroups + gi);
-        z16 = __ldg(zeros + (wrow + rl) * kGroups + gi);
+    // codes, scale and zero of the rows kPf iterations ahead are in flight while the current rows convert
+    // (one iteration: two measured slower with the permute path, the extra registers cost occupancy)
+    constexpr int kPf = 1;
+    uint32_t c[kPf + 1][4];
+    __half s16[kPf + 1], z16[kPf + 1];
+#pragma unroll
+    for (int f = 0; f <= kPf; ++f) {
+        const int64_t frow = wrow + f * step + rl;
+        c[f][0] = c[f][1] = c[f][2] = c[f][3] = 0u;
+        s16[f] = z16[f] = __float2half_rn(0.f);
+        if (f < kPf && frow < n) {
+            load_vchunk16<D, BITS>(data + frow * kRowBytes, j, c[f]);
+            s16[f] = __ldg(scales + frow * kGroups + gi);
+            z16[f] = __ldg(zeros + frow * kGroups + gi);
+        }
     }
     for (int it = 0; wrow < n; wrow += step, ++it) {
-        const int64_t nrow = wrow + step + rl;
-        uint32_t cn[4] = {0u, 0u, 0u, 0u};
-        __half sn = s16, zn = z16;
+        const int64_t nrow = wrow + kPf * step + rl;
         if (nrow < n) {
-            load_vchunk16<D, BITS>(data + nrow * kRowBytes, j, cn);
-            sn = __ldg(scales + nrow * kGroups + gi);
-            zn = __ldg(zeros + nrow * kGroups + gi);
+            load_vchunk16<D, BITS>(data + nrow * kRowBytes, j, c[kPf]);
+            s16[kPf] = __ldg(scales + nrow * kGroups + gi);
+            z16[kPf] = __ldg(zeros + nrow * kGroups + gi);
         }
-        const float s = __half2float(s16), z = __half2float(z16);
-        // q * s is exact in fp32 (q < 2^8, s an fp16), so (2^23 + q) s - 2^23 s in one FMA is exactly q s and the
-        // page's two roundings reduce to the one of the final addition: y = RN(RN(q s) + z) = RN(q s + z)
-        const float2 s2 = make_float2(s, s), z2 = make_float2(z, z);
-        const float2 off2 = make_float2(-8388608.0f * s, -8388608.0f * s);
-        float y[16];
-#pragma unroll
-        for (int k2 = 0; k2 < 8; ++k2) {
-            const float2 qm = make_float2(__uint_as_float(0x4B000000u | get_bits<BITS>(c, 2 * k2 * BITS)),
-                                          __uint_as_float(0x4B000000u | get_bits<BITS>(c, (2 * k2 + 1) * BITS)));
-            const float2 yy = __fadd2_rn(__ffma2_rn(qm, s2, off2), z2);
-            y[2 * k2] = yy.x;
-            y[2 * k2 + 1] = yy.y;
-        }
+        const float s = __half2float(s16[0]), z = __half2float(z16[0]);
         const int buf = it & 1;
         if (it >= 2) {
             if (lane == 0) bulk_wait_read<1>();                      // the copy that last read this buffer is done
             __syncwarp();
         }
         uint8_t* sb = &s_out[warp][buf][0];
-        if constexpr (OUT_F32) {
-            float4* o = reinterpret_cast<float4*>(sb) + 4 * lane;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) o[k] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
-        } else {
+        // q * s is exact in fp32 (q < 2^8, s an fp16), so (2^23 + q) s - 2^23 s in one FMA is exactly q s and the
+        // page's two roundings reduce to the one of the final addition: y = RN(RN(q s) + z) = RN(q s + z)
+        const float2 s2 = make_float2(s, s), z2 = make_float2(z, z);
+        const float2 off2 = make_float2(-8388608.0f * s, -8388608.0f * s);
+        if constexpr (BITS == 2 && !OUT_F32) {
+            // the four possible outputs of the lane's group, fp16(RN(q s + z)) for q = 0..3, by the same
+            // operations, as two half2 registers; each output pair is one byte permute of them, its selector
+            // (2 qa, 2 qa + 1, 2 qb, 2 qb + 1) one multiply-add of the codes spread to bytes 0 and 1
+            const float2 y01 = __fadd2_rn(__ffma2_rn(make_float2(__uint_as_float(0x4B000000u), __uint_as_float(0x4B000001u)),
+                                                     s2, off2), z2);
+            const float2 y23 = __fadd2_rn(__ffma2_rn(make_float2(__uint_as_float(0x4B000002u), __uint_as_float(0x4B000003u)),
+                                                     s2, off2), z2);
+            __half2 h01 = __floats2half2_rn(y01.x, y01.y), h23 = __floats2half2_rn(y23.x, y23.y);
+            const uint32_t t0 = *reinterpret_cast<uint32_t*>(&h01), t1 = *reinterpret_cast<uint32_t*>(&h23);
+            const uint32_t ev = c[0][0] & 0x33333333u, od = (c[0][0] >> 2) & 0x33333333u;  // codes 2k, 2k + 1 in nibble k
             uint32_t pk[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                __half2 hh = __floats2half2_rn(y[2 * k], y[2 * k + 1]);
-                pk[k] = *reinterpret_cast<uint32_t*>(&hh);
+            for (int m = 0; m < 4; ++m) {
+                const uint32_t wm = __byte_perm(ev, od, 0x40u + m + (m << 4));   // byte 0: ev.m, byte 1: od.m
+                const uint32_t lo = wm & 0x0303u, hi = (wm >> 4) & 0x0303u;
+                pk[2 * m] = __byte_perm(t0, t1, lo * 0x22u + 0x1010u);
+                pk[2 * m + 1] = __byte_perm(t0, t1, hi * 0x22u + 0x1010u);
             }
             uint4* o = reinterpret_cast<uint4*>(sb) + 2 * lane;
             o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else {
+            float y[16];
+#pragma unroll
+            for (int k2 = 0; k2 < 8; ++k2) {
+                const float2 qm = make_float2(__uint_as_float(0x4B000000u | get_bits<BITS>(c[0], 2 * k2 * BITS)),
+                                              __uint_as_float(0x4B000000u | get_bits<BITS>(c[0], (2 * k2 + 1) * BITS)));
+                const float2 yy = __fadd2_rn(__ffma2_rn(qm, s2, off2), z2);
+                y[2 * k2] = yy.x;
+                y[2 * k2 + 1] = yy.y;
+            }
+            if constexpr (OUT_F32) {
+                float4* o = reinterpret_cast<float4*>(sb) + 4 * lane;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) o[k] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+            } else {
+                uint32_t pk[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    __half2 hh = __floats2half2_rn(y[2 * k], y[2 * k + 1]);
+                    pk[k] = *reinterpret_cast<uint32_t*>(&hh);
+                }
+                uint4* o = reinterpret_cast<uint4*>(sb) + 2 * lane;
+                o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -292,9 +323,12 @@ __global__ void __launch_bounds__(256) decode_v_kernel(const uint8_t* __restrict
             bulk_commit();
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) c[k] = cn[k];
-        s16 = sn;
-        z16 = zn;
+        for (int f = 0; f < kPf; ++f) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) c[f][k] = c[f + 1][k];
+            s16[f] = s16[f + 1];
+            z16[f] = z16[f + 1];
+        }
     }
     if (lane == 0) bulk_wait_all();
 }
