@@ -65,7 +65,9 @@ struct AttCfg {
     static constexpr int kThreads = 32 * (kWarps + 1);
     static constexpr int kChunkTok = 16;             // tokens per chunk (= one paged block)
     static constexpr int kTileTok = kWarps * kChunkTok;
-    static constexpr int kStages = 4;               // a power of two
+    // stages of the copy ring (a power of two): 4; 2 with the 32 KB table of 4-bit keys, which keeps four CTAs
+    // per SM resident (two 64-token stages of four CTAs still hold ~60 KB per SM in flight)
+    static constexpr int kStages = ((1 << (2 * KB)) * 128 > 8192) ? 2 : 4;
     static constexpr int kKRow = D * KB / 8;
     static constexpr int kVRow = D * VB / 8;
     static constexpr int kVGroups = D / VG;
@@ -95,7 +97,11 @@ struct AttCfg {
         (kStages * kStageBytes > kCombineFloats * 4) ? kStages * kStageBytes : kCombineFloats * 4;
     static constexpr int kQfOff = kRingBytes;
     static constexpr int kLutOff = kQfOff + (kQInRegs ? 0 : (D / 16) * 32 * 16);
-    static constexpr int kZsOff = kLutOff + 2 * kLutBytes;
+    // tables up to 8 KB (key widths 1..3) start on a multiple of their size (slack reserved), so an entry's
+    // address is (pair bits << 7) | lane bits; the 32 KB table of 4-bit keys would need 32 KB of slack and cost
+    // resident CTAs, so it sits unaligned and its addresses are base + (pair bits << 7) + lane bits
+    static constexpr bool kLutAligned = (kLutBytes <= 8192);
+    static constexpr int kZsOff = kLutOff + (kLutAligned ? 2 : 1) * kLutBytes;
     static constexpr int kBarOff = (kZsOff + kWarps * 8 * kVGroups * 4 + 15) & ~15;
     static constexpr int kSmemMain = kBarOff + 8 * (2 * kStages) + 16;
     // the window CTA reuses the same allocation
@@ -422,8 +428,10 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
     const uint32_t b_full = smem_u32(bars), b_empty = b_full + 8 * S;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S);
-    // the key table starts on a multiple of its size, so an entry's address is (entry << 7) | lane bits
-    const uint32_t lut_addr = (smem_u32(smem + C::kLutOff) + C::kLutBytes - 1) & ~static_cast<uint32_t>(C::kLutBytes - 1);
+    // small key tables start on a multiple of their size, so an entry's address is (entry << 7) | lane bits
+    const uint32_t lut_addr = C::kLutAligned
+        ? (smem_u32(smem + C::kLutOff) + C::kLutBytes - 1) & ~static_cast<uint32_t>(C::kLutBytes - 1)
+        : smem_u32(smem + C::kLutOff);
     uint32_t* lut = reinterpret_cast<uint32_t*>(smem + (lut_addr - smem_u32(smem)));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -564,7 +572,11 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                         // code pairs (4ks, 4ks+1) and (4ks+2, 4ks+3) of the lane's quarter
                         const uint32_t e0 = window_shr(w[nt], 4 * ks * KB - 7) & kFieldMask;
                         const uint32_t e1 = window_shr(w[nt], (4 * ks + 2) * KB - 7) & kFieldMask;
-                        mma_f16(sc[nt], a, lds_u32(lane_addr | e0), lds_u32(lane_addr | e1));
+                        if constexpr (C::kLutAligned) {
+                            mma_f16(sc[nt], a, lds_u32(lane_addr | e0), lds_u32(lane_addr | e1));
+                        } else {
+                            mma_f16(sc[nt], a, lds_u32(lane_addr + e0), lds_u32(lane_addr + e1));
+                        }
                     }
                 }
                 // ---- logits (log2 domain) of head gid for tokens 2tig, 2tig+1, 8+2tig, 9+2tig

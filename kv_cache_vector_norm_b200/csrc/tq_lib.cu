@@ -441,7 +441,10 @@ struct AttendPlan {
     size_t workspace_bytes;    // qfrag_bytes + partial_bytes
 };
 
-tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan, bool window = false) {
+// ctas_per_sm: attention CTAs resident per SM.  Workspace sizes are planned with the largest (4); a launch
+// re-plans with its kernel's measured occupancy, which never needs more splits, so the workspace suffices.
+tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan, bool window = false,
+                      int ctas_per_sm = kAttendCtasPerSm) {
     if (!a) return fail(TQ_ERR_INVALID_ARG, "tq_attend: args is NULL");
     if (a->batch < 1 || a->num_kv_heads < 1 || a->num_q_heads < 1)
         return fail(TQ_ERR_INVALID_ARG, "tq_attend: batch, num_q_heads, num_kv_heads must be >= 1");
@@ -466,8 +469,9 @@ tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan, bool window = f
         max_chunks = a->max_seq_len / 16;
     }
     const int64_t bh = static_cast<int64_t>(a->batch) * a->num_kv_heads;
-    // fill every SM's resident CTAs once; a window's extra CTA per (sequence, kv head) takes one of them
-    int64_t splits = (static_cast<int64_t>(sm_count()) * kAttendCtasPerSm - (window ? bh : 0) + bh - 1) / bh;
+    // fill every SM's resident CTAs at most once (a grid one CTA past the resident slots runs a second, mostly
+    // empty wave that costs a whole CTA duration); a window's extra CTA per (sequence, kv head) takes one slot
+    int64_t splits = (static_cast<int64_t>(sm_count()) * ctas_per_sm - (window ? bh : 0)) / bh;
     const int64_t by_len = (max_chunks + 7) / 8;            // at least ~8 chunks (128 tokens) per split
     if (splits > by_len) splits = by_len;
     if (splits > kMaxSplits) splits = kMaxSplits;
@@ -482,12 +486,28 @@ tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan, bool window = f
 }
 
 template <int D, int KB, int VB, int VG>
-tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const tq_attend_window* win, const AttendPlan& plan,
-                        cudaStream_t st) {
+tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const tq_attend_window* win,
+                        const AttendPlan& plan_max, cudaStream_t st) {
     using Cfg = AttCfg<D, KB, VB, VG>;
     static std::atomic<uint64_t> mask{0};
+    static std::atomic<int> occupancy[64];                // resident CTAs per SM, per device (0: not yet queried)
     auto kern = attend_kernel<D, KB, VB, VG>;
     TQ_CUDA(allow_smem(kern, Cfg::kSmem, mask), "tq_attend_decode: cudaFuncSetAttribute");
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int occ = occupancy[dev & 63].load();
+    if (occ == 0) {
+        TQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, Cfg::kThreads, Cfg::kSmem),
+                "tq_attend_decode: cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+        occ = occ < 1 ? 1 : (occ > kAttendCtasPerSm ? kAttendCtasPerSm : occ);
+        occupancy[dev & 63].store(occ);
+    }
+    // split the sequences so that the grid fills the resident CTAs once
+    AttendPlan plan = plan_max;
+    if (occ < kAttendCtasPerSm) {
+        tq_status s = plan_attend(a, &plan, win != nullptr, occ);
+        if (s != TQ_OK) return s;
+    }
     AttendParams p;
     p.batch = a->batch;
     p.num_q_heads = a->num_q_heads;
