@@ -364,6 +364,78 @@ def gpu_arm(args, w, rank, world, local_rank):
                 clocks=sampler.summary(), launches=launches, fidelity=fid)
 
 
+# ----------------------------------------------------------------------------- bit-width sweep
+
+def sweep_arm(args):
+    """Encode and decode throughput of every key width (1..4 bits) and value width (2/3/4/8 bits, group 32
+    and one group per token) on 2^24 fp16 N(0,1) vectors of d = 128, each launch with a cold L2, plus the
+    measured key distortion mean ||x_hat - x||^2 / ||x||^2 against the codebook's D(b, d)."""
+    import torch
+    from kv_cache_vector_norm_b200 import synth, tq
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    n, d = args.sweep_rows, 128
+    x = synth.normal_fp16(0, synth.STREAM_K, (n, d), device=dev)
+    out = torch.empty(n, d, dtype=torch.float16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    hbm, peak_src = peaks()
+
+    def timeit(fn):
+        ms = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            if i >= args.warmup:
+                ms.append((e0, e1))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ms)
+
+    def entry(kind, bits, layout, bpv, ms):
+        gbps = bpv * n / (ms / 1e3) / 1e9
+        return {"kernel": kind, "bits": bits, "layout": layout, "us": ms * 1e3, "Mvectors_s": n / (ms / 1e3) / 1e6,
+                "GBps": gbps, "frac_of_hbm": gbps / hbm, "bytes_per_vector": bpv}
+
+    rows = []
+    for kb in (1, 2, 3, 4):
+        codec = tq.Codec(d, kb, 0)
+        kp = torch.empty(n, d * kb // 8, dtype=torch.uint8, device=dev)
+        kn = torch.empty(n, dtype=torch.float32, device=dev)
+        bpv = 2 * d + d * kb // 8 + 4
+        rows.append(entry("encode_k", kb, "-", bpv, timeit(lambda: codec.encode_k(x, packed=kp, norms=kn))))
+        rows.append(entry("decode_k", kb, "-", bpv, timeit(lambda: codec.decode_k(kp, kn, out=out))))
+        # evaluation of the round trip (not part of the timed path): mean relative squared error
+        acc, cnt = 0.0, 0
+        for r0 in range(0, n, 1 << 20):
+            xf = x[r0:r0 + (1 << 20)].float()
+            e = (out[r0:r0 + (1 << 20)].float() - xf).pow(2).sum(1) / xf.pow(2).sum(1).clamp_min(1e-30)
+            acc += float(e.double().sum())
+            cnt += e.numel()
+        rows[-1]["mse_rel"] = acc / cnt
+        rows[-1]["distortion_D_b_d"] = tq.build_codebook(d, kb)["distortion"]
+        del codec, kp, kn
+    for vb in (2, 3, 4, 8):
+        for g in (32, d):
+            vd = torch.empty(n, (d * vb + 7) // 8, dtype=torch.uint8, device=dev)
+            vs = torch.empty(n, d // g, dtype=torch.float16, device=dev)
+            vz = torch.empty(n, d // g, dtype=torch.float16, device=dev)
+            bpv = 2 * d + (d * vb + 7) // 8 + 4 * (d // g)
+            lay = "group32" if g == 32 else "token"
+            rows.append(entry("encode_v", vb, lay, bpv,
+                              timeit(lambda: tq.encode_v(x, vb, g, data=vd, scales=vs, zeros=vz))))
+            rows.append(entry("decode_v", vb, lay, bpv,
+                              timeit(lambda: tq.decode_v(vd, vs, vz, d, vb, g, out=out))))
+            del vd, vs, vz
+    if tq.read_device_flag() != 0:
+        raise RuntimeError("a kernel raised the device error flag during the sweep")
+    print(json.dumps({"mode": "bit-width sweep", "vectors": n, "head_dim": d, "data": "synthetic fp16 N(0,1), seed 0",
+                      "l2": "flushed by a 256 MiB write before every launch", "steps": args.steps,
+                      "hbm_peak_GBps": hbm, "peak_source": peak_src, "rows": rows}))
+
+
 # ------------------------------------------------------------------------------------- CPU (oracle)
 
 def oracle_sample(w, tokens, seed=0):
@@ -437,6 +509,10 @@ def main():
                     help="key rotation: seeded Haar (default) or randomized Walsh-Hadamard; same kernels")
     ap.add_argument("--only", choices=["encode_k", "encode_v", "decode_k", "decode_v", "attend"],
                     help="time one kernel of the path alone (profiling aid; prints its per-launch times)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="bit-width sweep instead of the step: encode/decode of every key and value width on "
+                         "--sweep-rows vectors (one JSON line of per-kernel rows)")
+    ap.add_argument("--sweep-rows", type=int, default=1 << 24)
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="row chunks of the end-to-end pass (host copies overlap the kernels across chunks)")
     ap.add_argument("--tokens", type=int, default=0,
@@ -485,6 +561,9 @@ def main():
         print(json.dumps(line))
         return
 
+    if args.sweep:
+        sweep_arm(args)
+        return
     import torch
     if world > 1:
         import datetime
