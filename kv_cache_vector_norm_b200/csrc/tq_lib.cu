@@ -341,16 +341,28 @@ extern "C" tq_status tq_decode_k(const tq_codec* c, const uint8_t* packed, const
 
 namespace {
 
+// Grid of the value kernels (256 threads, grid-stride over 16-element lane chunks): enough CTAs for the work,
+// at most one wave of the kernel's resident CTAs (queried once per device), so the grid never ends in a partial
+// wave that leaves the SMs nearly idle (a fixed 16 CTAs per SM ran 3.2 waves: value decode 61.4 -> 59.4 us).
+template <auto Kernel>
 int grid_for(int64_t units) {
+    static std::atomic<int> occupancy[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int occ = occupancy[dev & 63].load();
+    if (occ == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, Kernel, 256, 0) != cudaSuccess || occ < 1) occ = 1;
+        occupancy[dev & 63].store(occ);
+    }
     const int64_t blocks = (units + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 16;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * occ;
     return static_cast<int>(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
 }
 
 template <int D, int BITS, int GROUP>
 tq_status launch_encode_v(const void* x, int64_t n, int64_t stride, const int64_t* slots, uint8_t* data, void* scales,
                           void* zeros, cudaStream_t st) {
-    encode_v_kernel<D, BITS, GROUP><<<grid_for(n * (D / 16)), 256, 0, st>>>(
+    encode_v_kernel<D, BITS, GROUP><<<grid_for<encode_v_kernel<D, BITS, GROUP>>(n * (D / 16)), 256, 0, st>>>(
         static_cast<const __half*>(x), n, stride, slots, data, static_cast<__half*>(scales), static_cast<__half*>(zeros));
     TQ_CUDA(cudaGetLastError(), "tq_encode_v: launch");
     return TQ_OK;
@@ -359,7 +371,8 @@ tq_status launch_encode_v(const void* x, int64_t n, int64_t stride, const int64_
 template <int D, int BITS, int GROUP>
 tq_status launch_decode_v(const uint8_t* data, const void* scales, const void* zeros, int64_t n, void* out, int dtype,
                           cudaStream_t st) {
-    const int grid = grid_for(n * (D / 16));
+    const int grid = (dtype == TQ_F32) ? grid_for<decode_v_kernel<D, BITS, GROUP, true>>(n * (D / 16))
+                                       : grid_for<decode_v_kernel<D, BITS, GROUP, false>>(n * (D / 16));
     if (dtype == TQ_F32)
         decode_v_kernel<D, BITS, GROUP, true><<<grid, 256, 0, st>>>(data, static_cast<const __half*>(scales),
                                                                     static_cast<const __half*>(zeros), n, out);
