@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         *abort_flag = 0;
         fence_mbar_init();
     }
-    for (int i = threadIdx.x; i < C::kPairs * 32; i += blockDim.x) lut[i] = __ldg(p.pair_lut + (i >> 5));
+    fill_replicated(lut, p.pair_lut, C::kPairs);
     __syncthreads();
 
     if (warp == C::kWarps) {
@@ -778,7 +778,7 @@ __global__ void __launch_bounds__(128) attend_scores_kernel(const AttendParams p
     const int gid = lane >> 2, tig = lane & 3;
     const int h = blockIdx.y, b = blockIdx.z;
     const int G = p.group;
-    for (int i = threadIdx.x; i < kPairs * 32; i += blockDim.x) lut[i] = __ldg(p.pair_lut + (i >> 5));
+    fill_replicated(lut, p.pair_lut, kPairs);
     __syncthreads();
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();

@@ -453,8 +453,7 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
-    for (int i = threadIdx.x; i < C::kLutEntries * 32; i += blockDim.x)
-        reinterpret_cast<uint32_t*>(smem + Lo::kLut)[i] = lut_g[i >> 5];
+    fill_replicated(reinterpret_cast<uint32_t*>(smem + Lo::kLut), lut_g, C::kLutEntries);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -750,7 +749,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
         tmem_relinquish();
     }
     if constexpr (Lo::kReplPairs) {
-        for (int i = threadIdx.x; i < kPairs * 32; i += blockDim.x) s_pair[i] = pair_lut_g[i >> 5];
+        fill_replicated(s_pair, pair_lut_g, kPairs);
     } else {
         for (int i = threadIdx.x; i < kPairs; i += blockDim.x) s_pair[i] = pair_lut_g[i];
     }
