@@ -171,6 +171,13 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def chunk_bounds(n: int, chunks: int) -> list:
+    """Row boundaries of the end-to-end pass's chunks: nondecreasing, from 0 to n, every inner boundary a
+    multiple of 128 rows (whole key-codec tiles; every pool array then starts each chunk 16-byte aligned)."""
+    chunks = max(1, chunks)
+    return [((n * j // chunks) // 128) * 128 for j in range(chunks)] + [n]
+
+
 def job_value(world: int, units_per_rank: int, ms_per_step: float) -> float:
     """Whole-job throughput in M units/s: every rank processes units_per_rank per step (weak scaling)."""
     return world * units_per_rank / (ms_per_step / 1000.0) / 1e6
@@ -279,7 +286,7 @@ def gpu_arm(args, w, rank, world, local_rank):
     # device-to-host copies, so both PCIe directions and the kernels overlap; attention runs once every
     # chunk is encoded.  Events order each chunk's buffers between consecutive steps.
     nch = max(1, args.e2e_chunks)
-    bounds = [((n * j // nch) // 128) * 128 for j in range(nch)] + [n]
+    bounds = chunk_bounds(n, nch)
     s_cmp = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     ev_in = [torch.cuda.Event() for _ in range(nch)]
