@@ -239,7 +239,9 @@ typedef struct tq_attend_args {
 /*
  * tq_attend_workspace_bytes -- bytes of workspace tq_attend_decode needs for these arguments on the current
  * device: (head_dim / 16 * 32 + 2) * 16 bytes per (sequence, kv head) for the prepared query, plus the split-K
- * partials when the sequence axis is split.  Only the shape fields of args are read.
+ * partials when the sequence axis is split.  Only the shape fields of args are read.  The size assumes the
+ * most splits any key width can use (four attention CTAs per SM); a launch whose kernel keeps fewer CTAs
+ * resident splits less and uses a prefix of the same workspace.
  * Errors: the same argument checks as tq_attend_decode (TQ_ERR_INVALID_ARG / TQ_ERR_UNSUPPORTED).
  */
 tq_status tq_attend_workspace_bytes(const tq_attend_args* args, size_t* bytes);
