@@ -41,15 +41,34 @@ WORKLOADS = {
                             desc="Llama-3-8B-shaped layer: batch 8, 8 KV heads, 32 query heads, 8192 tokens, "
                                  "head_dim 128, K 4-bit, V 2-bit group 32, lognormal channel scales, 1% outlier "
                                  "channels x20"),
+    "paged_64x4096_d64": dict(kind="paged", batch=64, kv_heads=8, q_heads=32, tokens=4096, d=64, k_bits=4, v_bits=4,
+                              v_group=32, outliers=0.0,
+                              desc="high-concurrency paged cache: 64 sequences x 4096 tokens, 8 KV heads, head_dim 64, "
+                                   "16-token blocks of a seeded permuted block table; K 4-bit / V 4-bit group 32 bulk "
+                                   "encode through slots, decode of the pool, then one appended token per sequence "
+                                   "and a decode-step attend of 32 query heads over 4097 tokens"),
+    "paged_64x4096_d256": dict(kind="paged", batch=64, kv_heads=8, q_heads=32, tokens=4096, d=256, k_bits=4,
+                               v_bits=4, v_group=32, outliers=0.0,
+                               desc="high-concurrency paged cache: 64 sequences x 4096 tokens, 8 KV heads, head_dim "
+                                    "256, 16-token blocks of a seeded permuted block table; K 4-bit / V 4-bit group 32 "
+                                    "bulk encode through slots, decode of the pool, then one appended token per "
+                                    "sequence and a decode-step attend of 32 query heads over 4097 tokens"),
+    "k_roundtrip_4096": dict(kind="k_only", batch=1, kv_heads=1, q_heads=1, tokens=4096, d=128, k_bits=4, v_bits=2,
+                             v_group=32, outliers=0.0, scaled=False,
+                             desc="K-only round trip: 4096 key vectors, head_dim 128, fp16 N(0,1) iid, 4-bit codebook, "
+                                  "one seeded 128x128 Haar rotation; encode to 64 B + f32 norm per vector, then "
+                                  "decode"),
 }
 
 
 def algorithmic_bytes(w):
+    """Bytes per unit of each launch: per vector for the codec calls (the appended token counts its key and
+    value), per (token, kv head) for attention."""
     d, kb, vb, g = w["d"], w["k_bits"], w["v_bits"], w["v_group"]
     k = 2 * d + d * kb // 8 + 4
     v = 2 * d + (d * vb + 7) // 8 + 4 * (d // g)
     att = (d * kb // 8 + 4) + ((d * vb + 7) // 8 + 4 * (d // g))
-    return {"encode_k": k, "decode_k": k, "encode_v": v, "decode_v": v, "attend": att}
+    return {"encode_k": k, "decode_k": k, "encode_v": v, "decode_v": v, "append": k + v, "attend": att}
 
 
 def peaks():
@@ -69,6 +88,7 @@ KERNEL_SOURCES = {
     "decode_k": ("tq_device.cuh", "tq_codec_kernels.cuh", "tq_lib.cu"),
     "encode_v": ("tq_device.cuh", "tq_codec_kernels.cuh", "tq_lib.cu"),
     "decode_v": ("tq_device.cuh", "tq_codec_kernels.cuh", "tq_lib.cu"),
+    "append": ("tq_device.cuh", "tq_codec_kernels.cuh", "tq_lib.cu"),
     "attend": ("tq_device.cuh", "tq_attend_kernel.cuh", "tq_lib.cu"),
 }
 
@@ -127,17 +147,16 @@ class ClockSampler:
     def _run(self):
         while not self._stop.is_set():
             try:
+                # the sampler runs only while the timed launches are in flight: every sample counts
                 mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
-                util = self.nv.nvmlDeviceGetUtilizationRates(self.h).gpu
                 r = self._reasons_fn(self.h) if self._reasons_fn else 0
-                if util > 0:
-                    self.samples.append(mhz)
-                    for bit, name in self.REASONS.items():
-                        if r & bit and name != "gpu_idle":
-                            self.reasons.add(name)
+                self.samples.append(mhz)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.02)
+            time.sleep(0.005)
 
     def __enter__(self):
         if self.ok:
@@ -183,58 +202,158 @@ def job_value(world: int, units_per_rank: int, ms_per_step: float) -> float:
     return world * units_per_rank / (ms_per_step / 1000.0) / 1e6
 
 
+def paged_slots(table, hkv: int, t: int):
+    """Pool rows of a paged cache with 16-token blocks: (slots of tokens 0..t-1 in (sequence, kv head, token)
+    order, slots of the appended token t in (sequence, kv head) order); row = (block * H_kv + h) * 16 + t % 16
+    with block = table[sequence][t / 16]."""
+    import torch
+    dev = table.device
+    tt = torch.arange(t, device=dev)
+    hh = torch.arange(hkv, device=dev)
+    blk = table[:, tt // 16].to(torch.int64)                                          # [b][t]
+    slots = ((blk[:, None, :] * hkv + hh[None, :, None]) * 16 + (tt % 16)[None, None, :]).reshape(-1)
+    nb = table[:, t // 16].to(torch.int64)                                            # [b]
+    new_slots = ((nb[:, None] * hkv + hh[None, :]) * 16 + t % 16).reshape(-1)
+    return slots, new_slots
+
+
+def build_workload(w, dev, seed, rotation):
+    """Device buffers and the calls of one step of the workload: the codec launches over row ranges (so the
+    end-to-end pass can pipeline them in chunks) and the attention launch.
+
+    kind "contiguous": the cache rows are (b * H_kv + h) * T + t; encode writes them in place.
+    kind "paged": 16-token blocks; the block table is a seeded permutation of B * (T/16 + 1) physical blocks;
+    encode scatters every token through its slot, decode reads the whole pool, and the attention step first
+    appends one token per (sequence, kv head) through its slot, then attends over T + 1 tokens.
+    kind "k_only": the key round trip (encode, decode) with no values and no attention.
+    """
+    import torch
+    from kv_cache_vector_norm_b200 import synth, tq
+
+    kind = w.get("kind", "contiguous")
+    b, hkv, hq, t, d = w["batch"], w["kv_heads"], w["q_heads"], w["tokens"], w["d"]
+    kb, vb, vg = w["k_bits"], w["v_bits"], w["v_group"]
+    n_in = b * hkv * t
+    has_v = kind != "k_only"
+    scaled = w.get("scaled", True)
+    ks = synth.channel_scales(seed, hkv, d, "k", outlier_frac=w["outliers"]) if scaled else None
+    vs = synth.channel_scales(seed, hkv, d, "v", outlier_frac=w["outliers"]) if scaled else None
+    k = synth.kv_tensor(seed, synth.STREAM_K, b, hkv, t, d, device=dev, scales=ks).view(n_in, d)
+    v = synth.kv_tensor(seed, synth.STREAM_V, b, hkv, t, d, device=dev, scales=vs).view(n_in, d) if has_v else None
+    q = synth.normal_fp16(seed, synth.STREAM_Q, (b, hq, d), device=dev) if has_v else None
+    codec = tq.Codec(d, kb, 0, rotation=rotation)
+    slots = table = lens = k_new = v_new = new_slots = None
+    if kind == "paged":
+        per_seq = t // 16 + 1                             # room for the appended token
+        table = synth.block_table(seed, b, per_seq, b * per_seq).to(dev)
+        n_pool = b * per_seq * hkv * 16
+        slots, new_slots = paged_slots(table, hkv, t)
+        k_new = synth.normal_fp16(seed, 23, (b * hkv, d), device=dev)
+        v_new = synth.normal_fp16(seed, 24, (b * hkv, d), device=dev)
+        lens = torch.full((b,), t + 1, dtype=torch.int32, device=dev)
+    else:
+        n_pool = n_in
+    kp = torch.zeros(n_pool, d * kb // 8, dtype=torch.uint8, device=dev)
+    kn = torch.zeros(n_pool, dtype=torch.float32, device=dev)
+    kdec = torch.empty(n_pool, d, dtype=torch.float16, device=dev)
+    vd = vsc = vz = vdec = out = cache = ws = akw = None
+    if has_v:
+        vd = torch.zeros(n_pool, (d * vb + 7) // 8, dtype=torch.uint8, device=dev)
+        vsc = torch.zeros(n_pool, d // vg, dtype=torch.float16, device=dev)
+        vz = torch.zeros(n_pool, d // vg, dtype=torch.float16, device=dev)
+        vdec = torch.empty(n_pool, d, dtype=torch.float16, device=dev)
+        out = torch.empty(b, hq, d, dtype=torch.float32, device=dev)
+        cache = tq.Cache(kp, kn, vd, vsc, vz)
+        if kind == "paged":
+            akw = dict(num_kv_heads=hkv, v_bits=vb, v_group=vg, max_seq_len=None, block_table=table, seq_lens=lens,
+                       scale=0.0)
+        else:
+            akw = dict(num_kv_heads=hkv, v_bits=vb, v_group=vg, max_seq_len=t, block_table=None, seq_lens=None,
+                       scale=0.0)
+        ws = tq.attend_workspace(codec, q, cache, **akw)
+
+    def enc_k(r0, r1):
+        if slots is None:
+            codec.encode_k(k[r0:r1], packed=kp[r0:r1], norms=kn[r0:r1])
+        else:
+            codec.encode_k(k[r0:r1], slot_mapping=slots[r0:r1], packed=kp, norms=kn)
+
+    def enc_v(r0, r1):
+        if slots is None:
+            tq.encode_v(v[r0:r1], vb, vg, data=vd[r0:r1], scales=vsc[r0:r1], zeros=vz[r0:r1])
+        else:
+            tq.encode_v(v[r0:r1], vb, vg, slot_mapping=slots[r0:r1], data=vd, scales=vsc, zeros=vz)
+
+    def dec_k(r0, r1):
+        codec.decode_k(kp[r0:r1], kn[r0:r1], out=kdec[r0:r1])
+
+    def dec_v(r0, r1):
+        tq.decode_v(vd[r0:r1], vsc[r0:r1], vz[r0:r1], d, vb, vg, out=vdec[r0:r1])
+
+    def append():
+        codec.encode_k(k_new, slot_mapping=new_slots, packed=kp, norms=kn)
+        tq.encode_v(v_new, vb, vg, slot_mapping=new_slots, data=vd, scales=vsc, zeros=vz)
+
+    def attend():
+        tq.attend_decode(codec, q, cache, out=out, workspace=ws, **akw)
+
+    kernels = [("encode_k", lambda: enc_k(0, n_in))]
+    if has_v:
+        kernels.append(("encode_v", lambda: enc_v(0, n_in)))
+    kernels.append(("decode_k", lambda: dec_k(0, n_pool)))
+    if has_v:
+        kernels.append(("decode_v", lambda: dec_v(0, n_pool)))
+    if kind == "paged":
+        kernels.append(("append", append))
+    if has_v:
+        kernels.append(("attend", attend))
+    att_tokens = (t + 1) if kind == "paged" else t
+    # launches per call: one for each codec call; attention = query preparation + split kernel (+ the split
+    # merge when the workspace holds split-K partials beyond the query fragments)
+    qfrag_bytes = b * hkv * ((d // 16) * 32 + 2) * 16
+    per_call = {"append": 2, "attend": (3 if ws.numel() > qfrag_bytes else 2) if has_v else 0}
+    return dict(kind=kind, n_in=n_in, n_pool=n_pool, att_units=b * hkv * att_tokens, kernels=kernels,
+                per_call=per_call, enc_k=enc_k, enc_v=enc_v, dec_k=dec_k, dec_v=dec_v, append=append, attend=attend,
+                k=k, v=v, q=q, k_new=k_new, v_new=v_new, kdec=kdec, vdec=vdec, out=out, has_v=has_v,
+                codec=codec, cache=cache, akw=akw, kp=kp, kn=kn)
+
+
+def kernel_units(wl, w):
+    """Units each timed call processes: vectors for the codec calls, (token, kv head) pairs for attention."""
+    return {"encode_k": wl["n_in"], "encode_v": wl["n_in"], "decode_k": wl["n_pool"], "decode_v": wl["n_pool"],
+            "append": w["batch"] * w["kv_heads"], "attend": wl["att_units"]}
+
+
 def gpu_arm(args, w, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
-    from kv_cache_vector_norm_b200 import synth, tq
+    from kv_cache_vector_norm_b200 import tq
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    b, hkv, hq, t, d = w["batch"], w["kv_heads"], w["q_heads"], w["tokens"], w["d"]
-    kb, vb, vg = w["k_bits"], w["v_bits"], w["v_group"]
-    n = b * hkv * t
-    seed = rank
-    ks = synth.channel_scales(seed, hkv, d, "k", outlier_frac=w["outliers"])
-    vs = synth.channel_scales(seed, hkv, d, "v", outlier_frac=w["outliers"])
-    k = synth.kv_tensor(seed, synth.STREAM_K, b, hkv, t, d, device=dev, scales=ks).view(n, d)
-    v = synth.kv_tensor(seed, synth.STREAM_V, b, hkv, t, d, device=dev, scales=vs).view(n, d)
-    q = synth.normal_fp16(seed, synth.STREAM_Q, (b, hq, d), device=dev)
-    codec = tq.Codec(d, kb, 0, rotation=args.rotation)
-    kp = torch.empty(n, d * kb // 8, dtype=torch.uint8, device=dev)
-    kn = torch.empty(n, dtype=torch.float32, device=dev)
-    vd = torch.empty(n, (d * vb + 7) // 8, dtype=torch.uint8, device=dev)
-    vsc = torch.empty(n, d // vg, dtype=torch.float16, device=dev)
-    vz = torch.empty(n, d // vg, dtype=torch.float16, device=dev)
-    kdec = torch.empty(n, d, dtype=torch.float16, device=dev)
-    vdec = torch.empty(n, d, dtype=torch.float16, device=dev)
-    out = torch.empty(b, hq, d, dtype=torch.float32, device=dev)
-    cache = tq.Cache(kp, kn, vd, vsc, vz)
-    akw = dict(num_kv_heads=hkv, v_bits=vb, v_group=vg, max_seq_len=t, block_table=None, seq_lens=None, scale=0.0)
-    if args.window > 0:
+    wl = build_workload(w, dev, rank, args.rotation)
+    if args.window > 0 and wl["kind"] == "contiguous":
         # recent uncompressed tokens beside the compressed cache ("KV Cache API" store.py buffer)
+        from kv_cache_vector_norm_b200 import synth
+        b, hkv, d = w["batch"], w["kv_heads"], w["d"]
         win_k = synth.normal_fp16(0, 21, (b, hkv, args.window, d), device=dev)
         win_v = synth.normal_fp16(0, 22, (b, hkv, args.window, d), device=dev)
-        akw.update(win_k=win_k, win_v=win_v)
-        ws = tq.attend_window_workspace(codec, q, cache, win_k, win_v, None,
-                                        **{k: v for k, v in akw.items() if not k.startswith("win_")})
-    else:
-        ws = tq.attend_workspace(codec, q, cache, **akw)
+        akw = wl["akw"]
+        ws = tq.attend_window_workspace(wl["codec"], wl["q"], wl["cache"], win_k, win_v, None, **akw)
+        out, codec, q, cache = wl["out"], wl["codec"], wl["q"], wl["cache"]
+        wl["attend"] = lambda: tq.attend_decode(codec, q, cache, out=out, workspace=ws, win_k=win_k, win_v=win_v,
+                                                **akw)
+        wl["kernels"][-1] = ("attend", wl["attend"])
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-
-    kernels = [
-        ("encode_k", lambda: codec.encode_k(k, packed=kp, norms=kn)),
-        ("encode_v", lambda: tq.encode_v(v, vb, vg, data=vd, scales=vsc, zeros=vz)),
-        ("decode_k", lambda: codec.decode_k(kp, kn, out=kdec)),
-        ("decode_v", lambda: tq.decode_v(vd, vsc, vz, d, vb, vg, out=vdec)),
-        ("attend", lambda: tq.attend_decode(codec, q, cache, out=out, workspace=ws, **akw)),
-    ]
-
+    kernels = wl["kernels"]
     if args.only:
-        if args.only in ("decode_k", "decode_v", "attend"):
+        if args.only in ("decode_k", "decode_v", "attend", "append"):
             # the compressed cache these kernels read is written once, outside the timed launches
-            kernels[0][1]()
-            kernels[1][1]()
+            for name, fn in kernels:
+                if name.startswith("encode"):
+                    fn()
         kernels = [kv for kv in kernels if kv[0] == args.only]
+        if not kernels:
+            raise SystemExit(f"--only {args.only}: the workload has no such kernel")
 
     def one_step(record):
         for name, fn in kernels:
@@ -255,6 +374,7 @@ def gpu_arm(args, w, rank, world, local_rank):
         raise RuntimeError("a kernel raised the device error flag during warm-up")
 
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     events = []
@@ -269,106 +389,130 @@ def gpu_arm(args, w, rank, world, local_rank):
     for name, e0, e1 in events:
         per[name] += e0.elapsed_time(e1)
     if args.only:
-        return dict(per=per, launch_ms=[e0.elapsed_time(e1) for _, e0, e1 in events], n=n)
+        return dict(per=per, launch_ms=[e0.elapsed_time(e1) for _, e0, e1 in events], wl=wl)
     total_ms = max_over_ranks(sum(per.values()), world, dev)
     ms_per_step = total_ms / args.steps
+    e2e_ms, h2d, d2h = e2e_pass(args, wl, world, dev)
+    if tq.read_device_flag() != 0:
+        raise RuntimeError("a kernel raised the device error flag during timing")
+    launches = sum(wl["per_call"].get(name, 1) for name, _, _ in events)
+    fid = None
+    if args.fidelity and wl["has_v"] and wl["kind"] == "contiguous":
+        # logits of the compressed path vs the exact fp16 ones, over every (sequence, query head) of the step
+        from kv_cache_vector_norm_b200 import fidelity
+        b, hkv, t, d = w["batch"], w["kv_heads"], w["tokens"], w["d"]
+        wl["enc_k"](0, wl["n_in"])
+        approx = tq.attend_scores(wl["codec"], wl["q"], wl["cache"], **wl["akw"])
+        fid = fidelity.score_fidelity(approx, fidelity.exact_scores(wl["q"], wl["k"].view(b, hkv, t, d)))
+    return dict(per=per, ms_per_step=ms_per_step, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, wl=wl,
+                clocks=sampler.summary(), launches=launches, fidelity=fid)
 
-    # ---------------------------------------------------------------- end to end through host buffers
-    k_host = k.cpu().pin_memory()
-    v_host = v.cpu().pin_memory()
-    q_host = q.cpu().pin_memory()
-    kdec_host = torch.empty_like(kdec, device="cpu").pin_memory()
-    vdec_host = torch.empty_like(vdec, device="cpu").pin_memory()
-    out_host = torch.empty_like(out, device="cpu").pin_memory()
+
+def e2e_pass(args, wl, world, dev):
+    """The same step through host buffers: every step copies the inputs (keys, values, query, appended token)
+    from pinned host memory and the results (decoded keys and values, attention output) back, inside the timed
+    interval.  The cache moves in row chunks on three streams -- host-to-device copies, the codec kernels and
+    device-to-host copies -- so both PCIe directions overlap the kernels; attention runs once every chunk is
+    encoded.  Events order each chunk's buffers between consecutive steps.  Returns (ms per step, H2D bytes,
+    D2H bytes per step)."""
+    import torch
+
+    has_v = wl["has_v"]
+    ins = [x for x in (wl["k"], wl["v"]) if x is not None]
+    small_in = [x for x in (wl["q"], wl["k_new"], wl["v_new"]) if x is not None]
+    outs = [x for x in (wl["kdec"], wl["vdec"]) if x is not None]
+    ins_h = [x.cpu().pin_memory() for x in ins]
+    small_h = [x.cpu().pin_memory() for x in small_in]
+    outs_h = [torch.empty_like(x, device="cpu").pin_memory() for x in outs]
+    out_h = torch.empty_like(wl["out"], device="cpu").pin_memory() if has_v else None
     e2e_steps = max(3, min(args.steps, 20))
-
-    # The cache moves in row chunks on three streams: host-to-device copies, the codec kernels, and
-    # device-to-host copies, so both PCIe directions and the kernels overlap; attention runs once every
-    # chunk is encoded.  Events order each chunk's buffers between consecutive steps.
     nch = max(1, args.e2e_chunks)
-    bounds = chunk_bounds(n, nch)
+    bin_, bpool = chunk_bounds(wl["n_in"], nch), chunk_bounds(wl["n_pool"], nch)
     s_cmp = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     ev_in = [torch.cuda.Event() for _ in range(nch)]
-    ev_enc = [torch.cuda.Event() for _ in range(nch)]
     ev_dec = [torch.cuda.Event() for _ in range(nch)]
     ev_out = [torch.cuda.Event() for _ in range(nch)]
-    ev_att, ev_q = torch.cuda.Event(), torch.cuda.Event()
+    ev_enc_all, ev_att, ev_small = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
+    ev_enc_all.record(s_cmp)
+    ev_att.record(s_cmp)
 
-    def e2e_step():
+    def step():
+        s_in.wait_event(ev_enc_all)                       # the previous step's encoders are done with the inputs
         for j in range(nch):
-            r0, r1 = bounds[j], bounds[j + 1]
-            s_in.wait_event(ev_enc[j])                    # the previous step's encoders are done with chunk j
+            r0, r1 = bin_[j], bin_[j + 1]
             with torch.cuda.stream(s_in):
-                k[r0:r1].copy_(k_host[r0:r1], non_blocking=True)
-                v[r0:r1].copy_(v_host[r0:r1], non_blocking=True)
+                for x, xh in zip(ins, ins_h):
+                    x[r0:r1].copy_(xh[r0:r1], non_blocking=True)
             ev_in[j].record(s_in)
         s_in.wait_event(ev_att)                           # the previous step's attention is done with q
         with torch.cuda.stream(s_in):
-            q.copy_(q_host, non_blocking=True)
-        ev_q.record(s_in)
-        for j in range(nch):
-            r0, r1 = bounds[j], bounds[j + 1]
-            s_cmp.wait_event(ev_in[j])
-            codec.encode_k(k[r0:r1], packed=kp[r0:r1], norms=kn[r0:r1])
-            tq.encode_v(v[r0:r1], vb, vg, data=vd[r0:r1], scales=vsc[r0:r1], zeros=vz[r0:r1])
-            ev_enc[j].record(s_cmp)
+            for x, xh in zip(small_in, small_h):
+                x.copy_(xh, non_blocking=True)
+        ev_small.record(s_in)
+        def decode(j):
+            r0, r1 = bpool[j], bpool[j + 1]
             s_cmp.wait_event(ev_out[j])                   # the previous step's copies of chunk j have left
-            codec.decode_k(kp[r0:r1], kn[r0:r1], out=kdec[r0:r1])
-            tq.decode_v(vd[r0:r1], vsc[r0:r1], vz[r0:r1], d, vb, vg, out=vdec[r0:r1])
+            wl["dec_k"](r0, r1)
+            if has_v:
+                wl["dec_v"](r0, r1)
             ev_dec[j].record(s_cmp)
-        s_cmp.wait_event(ev_q)
-        kernels[-1][1]()                                  # attention over the whole compressed cache
+
+        # contiguous rows: chunk j decodes as soon as it is encoded; a scatter through slots can write any pool
+        # row, so the paged pool is decoded after every chunk is encoded
+        interleave = wl["kind"] != "paged"
+        for j in range(nch):
+            r0, r1 = bin_[j], bin_[j + 1]
+            s_cmp.wait_event(ev_in[j])
+            wl["enc_k"](r0, r1)
+            if has_v:
+                wl["enc_v"](r0, r1)
+            if interleave:
+                decode(j)
+        ev_enc_all.record(s_cmp)
+        if not interleave:
+            for j in range(nch):
+                decode(j)
+        if has_v:
+            s_cmp.wait_event(ev_small)
+            if wl["kind"] == "paged":
+                wl["append"]()
+            wl["attend"]()
         ev_att.record(s_cmp)
         for j in range(nch):
-            r0, r1 = bounds[j], bounds[j + 1]
+            r0, r1 = bpool[j], bpool[j + 1]
             s_out.wait_event(ev_dec[j])
             with torch.cuda.stream(s_out):
-                kdec_host[r0:r1].copy_(kdec[r0:r1], non_blocking=True)
-                vdec_host[r0:r1].copy_(vdec[r0:r1], non_blocking=True)
+                for x, xh in zip(outs, outs_h):
+                    xh[r0:r1].copy_(x[r0:r1], non_blocking=True)
             ev_out[j].record(s_out)
-        s_out.wait_event(ev_att)
-        with torch.cuda.stream(s_out):
-            out_host.copy_(out, non_blocking=True)
+        if has_v:
+            s_out.wait_event(ev_att)
+            with torch.cuda.stream(s_out):
+                out_h.copy_(wl["out"], non_blocking=True)
 
     for _ in range(2):
-        e2e_step()
+        step()
     torch.cuda.synchronize()
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(s_cmp)
     s_in.wait_event(e0)
     s_out.wait_event(e0)
     for _ in range(e2e_steps):
-        e2e_step()
-    done = torch.cuda.Event()
-    done.record(s_out)
-    s_cmp.wait_event(done)
-    s_in_done = torch.cuda.Event()
-    s_in_done.record(s_in)
-    s_cmp.wait_event(s_in_done)
+        step()
+    for s in (s_in, s_out):
+        ev = torch.cuda.Event()
+        ev.record(s)
+        s_cmp.wait_event(ev)
     e1.record(s_cmp)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
-    h2d = (k_host.numel() + v_host.numel() + q_host.numel()) * 2
-    d2h = (kdec_host.numel() + vdec_host.numel()) * 2 + out_host.numel() * 4
-    if tq.read_device_flag() != 0:
-        raise RuntimeError("a kernel raised the device error flag during timing")
-    # kernels per call: one each for the codec calls; attention = query preparation + split kernel
-    # (+ the split merge when the workspace holds split-K partials beyond the query fragments)
-    qfrag_bytes = b * hkv * ((d // 16) * 32 + 2) * 16
-    per_call = {"attend": 3 if ws.numel() > qfrag_bytes else 2}
-    launches = sum(per_call.get(name, 1) for name, _, _ in events)
-    fid = None
-    if args.fidelity:
-        # logits of the compressed path vs the exact fp16 ones, over every (sequence, query head) of the step
-        from kv_cache_vector_norm_b200 import fidelity
-        codec.encode_k(k, packed=kp, norms=kn)
-        approx = tq.attend_scores(codec, q, cache, **{kk: vv for kk, vv in akw.items() if not kk.startswith("win_")})
-        fid = fidelity.score_fidelity(approx, fidelity.exact_scores(q, k.view(b, hkv, t, d)))
-    return dict(per=per, ms_per_step=ms_per_step, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, n=n,
-                clocks=sampler.summary(), launches=launches, fidelity=fid)
+    ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    h2d = sum(x.numel() * x.element_size() for x in ins_h + small_h)
+    d2h = sum(x.numel() * x.element_size() for x in outs_h) + (out_h.numel() * 4 if has_v else 0)
+    return ms, h2d, d2h
 
 
 # ----------------------------------------------------------------------------- bit-width sweep
@@ -445,10 +589,11 @@ def sweep_arm(args):
 
 # ------------------------------------------------------------------------------------- CPU (oracle)
 
-def oracle_sample(w, tokens, seed=0):
-    """The oracle on one kv head's first `tokens` tokens of the workload: key and value encode and
-    decode of those vectors, then attention of that kv head's query heads over them.  Returns
-    seconds."""
+def oracle_sample(w, tokens, seed=0, head=0):
+    """The oracle on kv head `head`'s first `tokens` tokens of the workload: key (and value) encode and decode
+    of those vectors, then attention of that kv head's query heads over them (the key round trip only for the
+    K-only workload; the paged layout permutes rows, not arithmetic, so contiguous rows stand in for it).
+    Returns seconds."""
     import numpy as np
     import torch
     from kv_cache_vector_norm_b200 import synth
@@ -456,12 +601,15 @@ def oracle_sample(w, tokens, seed=0):
 
     d, kb, vb, vg = w["d"], w["k_bits"], w["v_bits"], w["v_group"]
     g = w["q_heads"] // w["kv_heads"]
+    has_v = w.get("kind", "contiguous") != "k_only"
     shape = (w["batch"], w["kv_heads"], w["tokens"], d)
-    rows = torch.arange(tokens, dtype=torch.int64)
-    ks = synth.channel_scales(seed, w["kv_heads"], d, "k", outlier_frac=w["outliers"])
-    vs = synth.channel_scales(seed, w["kv_heads"], d, "v", outlier_frac=w["outliers"])
+    head = head % (w["batch"] * w["kv_heads"])
+    rows = head * w["tokens"] + torch.arange(tokens, dtype=torch.int64)
+    scaled = w.get("scaled", True)
+    ks = synth.channel_scales(seed, w["kv_heads"], d, "k", outlier_frac=w["outliers"]) if scaled else None
+    vs = synth.channel_scales(seed, w["kv_heads"], d, "v", outlier_frac=w["outliers"]) if scaled else None
     k = synth.kv_rows(seed, synth.STREAM_K, shape, rows, scales=ks).numpy()
-    v = synth.kv_rows(seed, synth.STREAM_V, shape, rows, scales=vs).numpy()
+    v = synth.kv_rows(seed, synth.STREAM_V, shape, rows, scales=vs).numpy() if has_v else None
     q = synth.normal_fp16(seed, synth.STREAM_Q, (1, g, d)).numpy()
     pi = o.operational_rotation(d, 0)
     c, t = o.operational_codebook(d, kb)
@@ -470,32 +618,115 @@ def oracle_sample(w, tokens, seed=0):
     idx, nrm, _ = o.encode_k(k, pi, t)
     packed = o.pack_lsb(idx, kb)
     nrm32 = nrm.astype(np.float32)
-    data, s16, z16, _ = o.encode_v(v, vb, 32, layout)
     kidx = o.unpack_lsb(packed, kb, d)
     o.decode_k(kidx, nrm32.astype(np.float64), pi, c)
-    vhat = o.decode_v(data, s16, z16, vb, d, 32, layout)
-    o.attend(q, kidx[None, None], nrm32.astype(np.float64)[None, None], vhat[None, None], pi, c)
+    if has_v:
+        data, s16, z16, _ = o.encode_v(v, vb, 32, layout)
+        vhat = o.decode_v(data, s16, z16, vb, d, 32, layout)
+        o.attend(q, kidx[None, None], nrm32.astype(np.float64)[None, None], vhat[None, None], pi, c)
     return time.perf_counter() - t0
 
 
-def cpu_threads():
+def _limit_blas_threads(n=1):
+    """Keep numpy's BLAS pool at n threads in this process (so one process is one busy core)."""
     try:
-        from threadpoolctl import threadpool_info
-        return max(int(i.get("num_threads", 1)) for i in threadpool_info()) or 1
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=n)
     except Exception:
-        return os.cpu_count() or 1
+        return None
 
 
-def cpu_baseline(w, budget_s=15.0):
-    probe = 2048
+def _oracle_worker(w, tokens, head, barrier):
+    """One process of the multi-process CPU baseline: a warm-up sample, then a timed one started together
+    with the other processes.  Returns (start, end) wall-clock seconds of the timed sample."""
+    _limit_blas_threads(1)
+    oracle_sample(w, min(tokens, 256), head=head)
+    barrier.wait()
+    t0 = time.time()
+    oracle_sample(w, tokens, head=head)
+    return t0, time.time()
+
+
+def cpu_baseline(w, budget_s=10.0):
+    """The oracle as it stands, timed on the host cores: one process on one core (BLAS limited to one thread),
+    then one process per core each on its own kv head's slice, started together; the rate of the second is the
+    reported value.  Both are extrapolated from the bounded samples they time (Mvectors/s of the sample)."""
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+
+    lim = _limit_blas_threads(1)
+    probe = 1024
     dt = oracle_sample(w, probe)
     tokens = int(min(w["tokens"], max(probe, probe * budget_s / max(dt, 1e-3))))
     tokens = max(16, (tokens // 16) * 16)
-    dt = oracle_sample(w, tokens)
-    return {"value": tokens / dt / 1e6, "unit": "Mvectors/s", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"one kv head x {tokens} tokens of the workload: key+value encode and decode of {tokens} "
-                      f"vectors each and attention of {w['q_heads'] // w['kv_heads']} query heads over them "
-                      f"(fp64 numpy oracle, {dt:.1f} s)"}
+    dt1 = oracle_sample(w, tokens)
+    if lim is not None:
+        lim.restore_original_limits()
+    single = tokens / dt1 / 1e6
+    procs = max(1, os.cpu_count() or 1)
+    ctx = mp.get_context("spawn")                     # after CUDA work a forked child would hang
+    multi, span = None, None
+    try:
+        with ctx.Manager() as mgr:
+            barrier = mgr.Barrier(procs)
+            with ProcessPoolExecutor(max_workers=procs, mp_context=ctx) as ex:
+                futs = [ex.submit(_oracle_worker, w, tokens, i, barrier) for i in range(procs)]
+                spans = [f.result(timeout=600) for f in futs]
+        span = max(e for _, e in spans) - min(s for s, _ in spans)
+        multi = procs * tokens / span / 1e6
+    except Exception as exc:                          # report the single-core figure if the pool cannot run
+        sys.stderr.write(f"multi-process CPU baseline skipped: {exc}\n")
+    what = ("key encode and decode" if w.get("kind") == "k_only" else
+            f"key+value encode and decode and attention of {w['q_heads'] // w['kv_heads']} query heads")
+    out = {"value": multi if multi is not None else single, "unit": "Mvectors/s",
+           "cores": procs if multi is not None else 1, "kind": "oracle",
+           "sample": (f"{procs if multi is not None else 1} process(es), one core each (BLAS limited to one thread), "
+                      f"each on one kv head x {tokens} tokens of the workload ({what}); rate extrapolated from "
+                      f"that bounded sample, fp64 numpy oracle"),
+           "single_core": {"value": single, "seconds": dt1, "tokens": tokens}}
+    if multi is not None:
+        out["multi_process"] = {"value": multi, "processes": procs, "seconds": span}
+    return out
+
+
+def _oracle_step(w, tokens, head):
+    _limit_blas_threads(1)
+    t0 = time.time()
+    oracle_sample(w, tokens, head=head)
+    return t0, time.time()
+
+
+def reference_arm(args, w, config):
+    """The oracle as the reference arm: each step runs one bounded sample per host core (one process per core,
+    BLAS limited to one thread, each on its own kv head's slice), sized so the whole run ends in a few minutes;
+    the step's time is the wall-clock span of its processes."""
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+
+    total = args.steps + args.warmup
+    per_step_budget = max(0.05, 150.0 / total)
+    _limit_blas_threads(1)
+    probe = 1024
+    dt = oracle_sample(w, probe)
+    tokens = int(max(16, min(w["tokens"], probe * per_step_budget / max(dt, 1e-4))) // 16 * 16)
+    procs = max(1, os.cpu_count() or 1)
+    ctx = mp.get_context("spawn")
+    spans = []
+    with ProcessPoolExecutor(max_workers=procs, mp_context=ctx) as ex:
+        for i in range(total):
+            res = [f.result() for f in [ex.submit(_oracle_step, w, tokens, j) for j in range(procs)]]
+            if i >= args.warmup:
+                spans.append(max(e for _, e in res) - min(s for s, _ in res))
+    ms = 1000.0 * sum(spans) / len(spans)
+    value = procs * tokens / (ms / 1000.0) / 1e6
+    sample = (f"{procs} processes, one core each (BLAS limited to one thread), each on one kv head x {tokens} "
+              f"tokens of the workload per step; fp64 numpy oracle")
+    return {"metric": METRIC, "value": value, "unit": "Mvectors/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (f32 for the value format)",
+            "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": value, "unit": "Mvectors/s", "cores": procs, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "Mvectors/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 # --------------------------------------------------------------------------------------------- main
@@ -548,24 +779,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        total = args.steps + args.warmup
-        per_step_budget = max(0.05, 150.0 / total)
-        probe = 1024
-        dt = oracle_sample(w, probe)
-        tokens = int(max(16, min(w["tokens"], probe * per_step_budget / max(dt, 1e-4))) // 16 * 16)
-        for _ in range(args.warmup):
-            oracle_sample(w, tokens)
-        times = [oracle_sample(w, tokens) for _ in range(args.steps)]
-        ms = 1000.0 * sum(times) / len(times)
-        value = tokens / (ms / 1000.0) / 1e6
-        line = {"metric": METRIC, "value": value, "unit": "Mvectors/s", "impl": "reference", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64 (f32 for the value format)",
-                "data": "synthetic", "config": config,
-                "cpu_baseline": {"value": value, "unit": "Mvectors/s", "cores": cpu_threads(), "kind": "oracle",
-                                 "sample": f"one kv head x {tokens} tokens per step"},
-                "e2e": {"value": value, "unit": "Mvectors/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(line))
+        print(json.dumps(reference_arm(args, w, config)))
         return
 
     if args.sweep:
@@ -582,8 +796,9 @@ def main():
         if rank == 0:
             bpv_k = algorithmic_bytes(w)[args.only]
             ms = [round(x, 5) for x in r["launch_ms"]]
+            units = kernel_units(r["wl"], w)[args.only]
             print(json.dumps({"mode": "single-kernel", "kernel": args.only, "workload": args.workload,
-                              "launch_ms": ms, "GBps_median": bpv_k * r["n"] / (statistics.median(ms) / 1e3) / 1e9}))
+                              "launch_ms": ms, "GBps_median": bpv_k * units / (statistics.median(ms) / 1e3) / 1e9}))
         return
     if world > 1:
         import torch.distributed as dist
@@ -592,11 +807,12 @@ def main():
     if rank != 0:
         return
     hbm, peak_src = peaks()
-    n = r["n"]
+    n = r["wl"]["n_in"]
+    units_of = kernel_units(r["wl"], w)
     kern = {}
     for name, tot in r["per"].items():
         ms = tot / args.steps
-        units = n if name != "attend" else n
+        units = units_of[name]
         gbps = bpv[name] * units / (ms / 1000.0) / 1e9
         kern[name] = {"ms": ms, "Mvectors_s": units / (ms / 1000.0) / 1e6, "GBps": gbps, "frac_of_hbm": gbps / hbm,
                       "bytes_per_vector": bpv[name]}
@@ -607,15 +823,17 @@ def main():
         "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16 in, f32 accumulate, u8 codes", "data": "synthetic (seeded, counter-based)",
         "config": config, "kernels": kern,
-        "attend_GBps": kern["attend"]["GBps"], "attend_frac_of_hbm": kern["attend"]["frac_of_hbm"],
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": kern[dom]["GBps"], "peak": hbm, "unit": "GB/s",
                      "frac": kern[dom]["GBps"] / hbm, "peak_source": peak_src,
                      "traffic": traffic_record(dom, args.workload),
-                     "algorithmic_bytes_per_launch": bpv[dom] * n},
+                     "algorithmic_bytes_per_launch": bpv[dom] * units_of[dom]},
         "e2e": {"value": job_value(world, n, r["e2e_ms"]), "unit": "Mvectors/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"], "clocks": r["clocks"],
     }
+    if "attend" in kern:
+        line["attend_GBps"] = kern["attend"]["GBps"]
+        line["attend_frac_of_hbm"] = kern["attend"]["frac_of_hbm"]
     if r.get("fidelity") is not None:
         line["fidelity"] = r["fidelity"]
     if not args.no_cpu_baseline:

@@ -206,7 +206,10 @@ tq_status tq_decode_v(int d, int bits, int group, const uint8_t* data, const voi
  *   paged:      row = (block_table[b * max_blocks + t / block_size] * num_kv_heads + h) * block_size
  *                     + t % block_size.
  * Sequence b attends to tokens 0 .. seq_lens[b]-1 (all max_seq_len tokens if seq_lens is NULL in the
- * contiguous layout; seq_lens is required for the paged layout).  Query head hq reads kv head
+ * contiguous layout; seq_lens is required for the paged layout).  The kernels clamp seq_lens[b] to
+ * [0, max_seq_len] in the contiguous layout and to [0, max_blocks * block_size] in the paged one, so a length
+ * past the cache attends to the whole addressable sequence and never reads beyond its rows or its
+ * block-table row.  Every block_table entry below the (clamped) length must name a block of the pools.  Query head hq reads kv head
  * hq / (num_q_heads / num_kv_heads).
  */
 typedef struct tq_attend_args {
@@ -326,11 +329,14 @@ tq_status tq_attend_decode_window(const tq_codec* codec, const tq_attend_args* a
  * declares at file scope in device memory; args->workspace and args->workspace_bytes are ignored.  The
  * entry point calls no allocator (no cudaMalloc, no cudaFree, nothing that allocates).
  *   - Set-up: the first call on each device looks up the scratch array's device address with
- *     cudaGetSymbolAddress (with that device current) and caches it; make that first call outside any
- *     stream capture.
- *   - Limit: a launch whose workspace (query fragments and split-K partials) needs more than
- *     TQ_ATTEND_SCRATCH_BYTES (see tq_attend_workspace_bytes) is rejected with TQ_ERR_INVALID_ARG and a message giving both sizes;
- *     use tq_attend_decode with a caller workspace for such shapes.
+ *     cudaGetSymbolAddress (with that device current) and caches it for the life of the process; make that
+ *     first call outside any stream capture.  The cached address belongs to the device's primary context:
+ *     after cudaDeviceReset (or any reset of that context) it is stale, so do not call this entry point
+ *     again in a process that has reset the device.
+ *   - Limit: the check uses the size tq_attend_workspace_bytes reports for the same arguments (planned for
+ *     the most splits any key width can use); when that exceeds TQ_ATTEND_SCRATCH_BYTES the call is
+ *     rejected with TQ_ERR_INVALID_ARG and a message giving both sizes, even if this codec's key width
+ *     would launch fewer splits.  Use tq_attend_decode with a caller workspace for such shapes.
  *   - Sharing: all calls on a device share the one array and it keeps the last call's contents; nothing
  *     in it needs to start at zero, since every launch overwrites the part it reads.  Calls that can
  *     overlap on the GPU (different streams without ordering, or different threads) race on it and must

@@ -224,6 +224,16 @@ __device__ __forceinline__ uint32_t vfield(const uint8_t* row, int sl, int gid) 
     }
 }
 
+// Tokens of sequence b that the compressed part attends to: seq_lens[b] (all max_seq_len tokens when seq_lens
+// is NULL), clamped to [0, the tokens the layout can address] -- max_seq_len rows in the contiguous layout,
+// max_blocks * 16 in the paged one -- so a length past the cache never reads past a sequence's rows or its
+// block-table row.
+__device__ __forceinline__ int64_t attend_seq_len(const AttendParams& p, int b) {
+    const int64_t cap = p.block_table ? static_cast<int64_t>(p.max_blocks) * 16 : p.max_seq_len;
+    const int64_t t = p.seq_lens ? static_cast<int64_t>(p.seq_lens[b]) : cap;
+    return t < 0 ? 0 : (t > cap ? cap : t);
+}
+
 // Query preparation: the rotated query q_rot[g] = Pi_op q[g] of each of the group's heads, scaled by softmax
 // scale * log2(e) and a per-head power-of-two prescale, split into fp16 hi/lo halves and laid out as the score A
 // fragments (rows gid = hi, gid + 8 = lo); slots d/16 * 32 and + 1 hold 1 / prescale of heads 0..7.
@@ -448,7 +458,7 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
         return;
     }
-    const int64_t T = p.seq_lens ? static_cast<int64_t>(p.seq_lens[b]) : p.max_seq_len;
+    const int64_t T = attend_seq_len(p, b);
     const int64_t nchunks = (T + 15) / 16;
     const int64_t cps = (nchunks + p.num_splits - 1) / p.num_splits;
     const int64_t c_begin = split * cps;
@@ -783,7 +793,7 @@ __global__ void __launch_bounds__(128) attend_scores_kernel(const AttendParams p
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();
     const float unpre = __ldcg(reinterpret_cast<const float*>(qf + KS * 32) + gid);
-    const int64_t T = p.seq_lens ? static_cast<int64_t>(p.seq_lens[b]) : p.max_seq_len;
+    const int64_t T = attend_seq_len(p, b);
     const int64_t chunk = static_cast<int64_t>(blockIdx.x) * 4 + warp;
     if (chunk * 16 >= score_len) return;
     // this lane's quarter of the key rows of tokens 8 nt + gid (zero past the sequence)

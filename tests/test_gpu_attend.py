@@ -154,3 +154,47 @@ def test_attend_70b_class_full_size_sampled():
 def test_attend_llama8b_layer_sampled():
     # batch 8, 8 kv heads, 32 query heads, 8192 tokens, d = 128, K 4-bit, V 2-bit group 32
     _run_contiguous(8, 8, 32, 8192, 128, 4, 2, 32, check_bh=[(0, 0), (7, 7), (3, 2)])
+
+
+def test_attend_seq_lens_are_clamped_to_the_layout():
+    # contiguous: a length past max_seq_len attends to all max_seq_len tokens, a negative one to none
+    b, hkv, hq, t, d, kb, vb, vg = 3, 2, 8, 256, 128, 3, 2, 32
+    cd, cache = build_contiguous(b, hkv, t, d, kb, vb, vg)
+    q16 = synth.normal_fp16(4, synth.STREAM_Q, (b, hq, d))
+    lens = torch.tensor([t + 1000, -7, 100], dtype=torch.int32, device=DEV)
+    out = to_np(tq.attend_decode(cd, q16.to(DEV), cache, num_kv_heads=hkv, v_bits=vb, v_group=vg, max_seq_len=t,
+                                 seq_lens=lens))
+    g = hq // hkv
+    for bi, length in enumerate([t, 0, 100]):
+        for h in range(hkv):
+            rows = (bi * hkv + h) * t + np.arange(length)
+            ref = oracle_heads(cd, cache, q16.numpy(), bi, h, rows, vb, vg, g)
+            for gi in range(g):
+                got = out[bi, h * g + gi]
+                if length == 0:
+                    assert np.all(got == 0)
+                else:
+                    assert rel_l2(got, ref[gi]) <= L2_RTOL
+    # paged: a length past max_blocks * 16 attends to the table's max_blocks * 16 tokens; every pool row is filled
+    b, max_blocks = 2, 4
+    nblocks = b * max_blocks
+    table = synth.block_table(5, b, max_blocks, nblocks)
+    rows_total = nblocks * hkv * 16
+    k = synth.normal_fp16(21, synth.STREAM_K, (rows_total, d)).to(DEV)
+    v = synth.normal_fp16(21, synth.STREAM_V, (rows_total, d)).to(DEV)
+    kp, kn = cd.encode_k(k)
+    vd, vs, vz = tq.encode_v(v, vb, vg)
+    pcache = tq.Cache(kp, kn, vd, vs, vz)
+    plens = torch.tensor([10 ** 6, 17], dtype=torch.int32, device=DEV)
+    q16 = synth.normal_fp16(6, synth.STREAM_Q, (b, hq, d))
+    kw = dict(num_kv_heads=hkv, v_bits=vb, v_group=vg, block_table=table.to(DEV), seq_lens=plens)
+    out = to_np(tq.attend_decode(cd, q16.to(DEV), pcache, **kw))
+    scores = to_np(tq.attend_scores(cd, q16.to(DEV), pcache, **kw))
+    for bi, length in enumerate([16 * max_blocks, 17]):
+        assert np.all(np.isfinite(scores[bi, :, :length])) and np.all(scores[bi, :, length:] == -np.inf)
+        for h in range(hkv):
+            rows = o.paged_rows(table.numpy(), bi, h, length, hkv, 16)
+            ref = oracle_heads(cd, pcache, q16.numpy(), bi, h, rows, vb, vg, g)
+            for gi in range(g):
+                assert rel_l2(out[bi, h * g + gi], ref[gi]) <= L2_RTOL
+    assert tq.read_device_flag() == 0

@@ -42,15 +42,21 @@ def test_noalloc_matches_workspace_entry_point_twice():
 
 
 def test_noalloc_rejects_launches_beyond_its_scratch():
-    # find a head_dim-256 shape whose split-K partials do not fit in the fixed scratch
+    # A head_dim-256 shape whose split-K partials do not fit in the fixed scratch.  The cache is paged and every
+    # block-table entry names its one block, so every row such a launch could read exists: if the size check
+    # ever stopped refusing, the launch would read valid memory and the test would fail on the missing error.
     cd, cache = _cache(1, 1, 16, d=256, kb=4, vb=4)
+    max_blocks = 256                                   # 4096 tokens per sequence
     for bh in range(150, 1200, 10):
         q = torch.zeros(bh, 4, 256, dtype=torch.float16, device=DEV)
-        kw = dict(num_kv_heads=1, v_bits=4, v_group=32, max_seq_len=4096, block_table=None, seq_lens=None, scale=0.0)
-        need = tq.attend_workspace_bytes(cd, q, cache, **kw)
+        table = torch.zeros(bh, max_blocks, dtype=torch.int32, device=DEV)
+        lens = torch.full((bh,), 16 * max_blocks, dtype=torch.int32, device=DEV)
+        kw = dict(num_kv_heads=1, v_bits=4, v_group=32, block_table=table, seq_lens=lens, scale=0.0)
+        need = tq.attend_workspace_bytes(cd, q, cache, max_seq_len=None, **kw)
         if need > tq.ATTEND_SCRATCH_BYTES:
             break
     else:
         pytest.skip("no shape on this device needs more split-K scratch than the fixed array holds")
     with pytest.raises(tq.TQError, match="static scratch"):
         tq.attend_decode_noalloc(cd, q, cache, out=torch.empty(bh, 4, 256, device=DEV), **kw)
+    torch.cuda.synchronize()
