@@ -473,7 +473,8 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         *abort_flag = 0;
         fence_mbar_init();
     }
-    fill_replicated(lut, p.pair_lut, C::kPairs);
+    // the producer issues its first copies as soon as the barriers exist; the consumers fill the code-pair table
+    // (its global load overlaps those copies) and publish it with their own named barrier
     __syncthreads();
 
     if (warp == C::kWarps) {
@@ -517,13 +518,14 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
     } else {
         // ------------------------------------------------------------------ query fragments
         // written by attend_prep_kernel, the grid this one depends on programmatically
+        fill_replicated_by(lut, p.pair_lut, C::kPairs, threadIdx.x, 32 * C::kWarps);
         asm volatile("griddepcontrol.wait;" ::: "memory");
         const uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();
         const float unpre = __ldcg(reinterpret_cast<const float*>(qf + KS * 32) + gid);   // head gid's
         if constexpr (!C::kQInRegs) {
             for (int i = threadIdx.x; i < KS * 32; i += 32 * C::kWarps) s_qf[i] = __ldcg(qf + i);
-            named_bar_sync(1, 32 * C::kWarps);
         }
+        named_bar_sync(1, 32 * C::kWarps);              // the table and the query fragments are in place
 
         // ------------------------------------------------------------------ token loop
         uint4 qa[C::kQInRegs ? KS : 1];
@@ -539,31 +541,43 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         float zacc[G8];
 #pragma unroll
         for (int g = 0; g < G8; ++g) zacc[g] = 0.f;
-        float m_run = -INFINITY, l_run = 0.f;
-        const int tok[4] = {2 * tig, 2 * tig + 1, 8 + 2 * tig, 9 + 2 * tig};
+        // Lazy running maximum: the probabilities are 2^(logit - m_off) with m_off = m_run - kPExp, and m_run moves
+        // only when a logit exceeds m_run + kSlack (then every accumulator is rescaled once); in between, p may
+        // reach 2^(kSlack + kPExp), which fp32 and the bf16 operands hold with ample room.
+        constexpr float kSlack = 8.f;
+        float m_run = -INFINITY, m_thr = -INFINITY, m_off = 0.f, l_run = 0.f;
+        // this lane's byte offsets inside one stage: its quarter of key rows gid and 8 + gid, its tokens' norms,
+        // scale / zero rows and value fields
+        const uint8_t* const st0 = smem + warp * 16 * C::kKRow + gid * C::kKRow + tig * (C::kQuarterBits / 8);
+        const int t0 = 2 * tig;                        // tokens t0, t0 + 1, t0 + 8, t0 + 9 of the chunk
+        const int o_nrm = C::kNOff + (warp * 16 + t0) * 4;
+        const int o_scl = C::kSOff + (warp * 16 + t0) * G8 * 2;
+        const int o_zer = C::kZOff + (warp * 16 + t0) * G8 * 2;
+        const int o_val = C::kVOff + (warp * 16 + t0) * C::kVRow;
 
         // 32-bit loop state: a split holds fewer than 2^31 chunks
         const int ntiles32 = static_cast<int>(ntiles);
         const int nrel = static_cast<int>(c_end - c_begin);
+        // tokens of the split's last chunk that belong to the sequence (16 for every other chunk)
+        const int last_valid = static_cast<int>(T - (c_end - 1) * 16);
         for (int ti = 0; ti < ntiles32; ++ti) {
-            const int s = ti % S;
+            const int s = ti & (S - 1);
             if (!mbar_wait(b_full + 8 * s, static_cast<uint32_t>((ti / S) & 1), abort_flag)) break;
             const int rel = ti * C::kWarps + warp;        // chunk index within the split
             if (rel < nrel) {
-                const uint8_t* st = smem + s * C::kStageBytes;
-                const uint8_t* kch = st + C::kKOff + warp * 16 * C::kKRow;
+                const uint8_t* const stg = smem + s * C::kStageBytes;
+                const uint8_t* const kch = st0 + s * C::kStageBytes;
                 // ---- scores: S'[16 x 8 tokens] per n-tile, rows gid (hi part) and gid+8 (lo part)
                 uint32_t w[2][C::kQuarterWords];
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
-                    // this lane's quarter of the key row of token 8nt + gid
-                    const uint8_t* krow = kch + (8 * nt + gid) * C::kKRow;
+                    const uint8_t* krow = kch + 8 * nt * C::kKRow;
                     if constexpr (C::kQuarterHalves % 2 == 0) {
-                        const uint32_t* k32 = reinterpret_cast<const uint32_t*>(krow) + tig * (C::kQuarterHalves / 2);
+                        const uint32_t* k32 = reinterpret_cast<const uint32_t*>(krow);
 #pragma unroll
                         for (int i = 0; i < C::kQuarterWords; ++i) w[nt][i] = (2 * i < C::kQuarterHalves) ? k32[i] : 0u;
                     } else {
-                        const uint16_t* k16 = reinterpret_cast<const uint16_t*>(krow) + tig * C::kQuarterHalves;
+                        const uint16_t* k16 = reinterpret_cast<const uint16_t*>(krow);
 #pragma unroll
                         for (int i = 0; i < C::kQuarterWords; ++i) {
                             const uint32_t lo16 = (2 * i < C::kQuarterHalves) ? k16[2 * i] : 0u;
@@ -579,7 +593,6 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                     if constexpr (C::kQInRegs) a = qa[ks]; else a = s_qf[ks * 32 + lane];
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
-                        // code pairs (4ks, 4ks+1) and (4ks+2, 4ks+3) of the lane's quarter
                         const uint32_t e0 = window_shr(w[nt], 4 * ks * KB - 7) & kFieldMask;
                         const uint32_t e1 = window_shr(w[nt], (4 * ks + 2) * KB - 7) & kFieldMask;
                         if constexpr (C::kLutAligned) {
@@ -589,95 +602,101 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                         }
                     }
                 }
-                // ---- logits (log2 domain) of head gid for tokens 2tig, 2tig+1, 8+2tig, 9+2tig
-                const float* nrm = reinterpret_cast<const float*>(st + C::kNOff) + warp * 16;
-                const int64_t rem = T - (c_begin + rel) * 16;
-                const int valid = (rem < 16) ? static_cast<int>(rem) : 16;
+                // ---- logits (log2 domain) of head gid for tokens t0, t0+1, t0+8, t0+9
+                const float2 n01 = *reinterpret_cast<const float2*>(stg + o_nrm);
+                const float2 n89 = *reinterpret_cast<const float2*>(stg + o_nrm + 32);
                 float lg[4];
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    // tokens 8 nt + 2 tig, + 1: (hi row + lo row) * unpre * n_t, two per packed f32x2 operation
-                    const float2 sum = __fadd2_rn(make_float2(sc[nt][0], sc[nt][1]), make_float2(sc[nt][2], sc[nt][3]));
-                    const float2 nn = __fmul2_rn(make_float2(nrm[tok[2 * nt]], nrm[tok[2 * nt + 1]]), make_float2(unpre, unpre));
-                    const float2 raw = __fmul2_rn(sum, nn);
-                    lg[2 * nt] = raw.x;
-                    lg[2 * nt + 1] = raw.y;
+                {
+                    const float2 u2 = make_float2(unpre, unpre);
+                    const float2 r0 = __fmul2_rn(__fadd2_rn(make_float2(sc[0][0], sc[0][1]), make_float2(sc[0][2], sc[0][3])),
+                                                 __fmul2_rn(n01, u2));
+                    const float2 r1 = __fmul2_rn(__fadd2_rn(make_float2(sc[1][0], sc[1][1]), make_float2(sc[1][2], sc[1][3])),
+                                                 __fmul2_rn(n89, u2));
+                    lg[0] = r0.x; lg[1] = r0.y; lg[2] = r1.x; lg[3] = r1.y;
                 }
-                if (valid < 16) {                                  // the sequence's last, partial chunk
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) lg[e] = (tok[e] < valid) ? lg[e] : -INFINITY;
+                if (rel == nrel - 1 && last_valid < 16) {          // the sequence's last, partial chunk
+                    lg[0] = (t0 < last_valid) ? lg[0] : -INFINITY;
+                    lg[1] = (t0 + 1 < last_valid) ? lg[1] : -INFINITY;
+                    lg[2] = (t0 + 8 < last_valid) ? lg[2] : -INFINITY;
+                    lg[3] = (t0 + 9 < last_valid) ? lg[3] : -INFINITY;
                 }
-                float mt = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-                const float m_new = fmaxf(m_run, mt);
-                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+                const float lm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
+                if (__any_sync(0xffffffffu, lm > m_thr)) {
+                    // a logit passed its head's threshold: move that head's maximum and rescale everything once
+                    float mq = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 1));
+                    mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, 2));
+                    if (mq > m_thr) {
+                        const float corr = ex2(m_run - mq);                  // 0 while m_run is -inf
+                        m_run = mq;
+                        m_thr = mq + kSlack;
+                        m_off = mq - static_cast<float>(kPExp);
+                        l_run *= corr;
+#pragma unroll
+                        for (int g = 0; g < G8; ++g) zacc[g] *= corr;
+                        // stash the factor for the lanes holding this head's accumulator columns
+                        mq = corr;
+                    } else {
+                        mq = 1.f;
+                    }
+                    // the accumulator columns are heads 2tig and 2tig+1: their factors sit in lanes 8tig, 8tig+4
+                    const float ca = __shfl_sync(0xffffffffu, mq, 8 * tig);
+                    const float cb = __shfl_sync(0xffffffffu, mq, 8 * tig + 4);
+#pragma unroll
+                    for (int m = 0; m < MT; ++m) {
+                        o[m][0] *= ca; o[m][1] *= cb; o[m][2] *= ca; o[m][3] *= cb;
+                    }
+                }
                 // probabilities carry the factor 2^kPExp (so do l_run and zacc; removed at the end)
-                const float m_off = m_use - static_cast<float>(kPExp);
                 float pr[4];
                 {
                     const float2 a01 = __fadd2_rn(make_float2(lg[0], lg[1]), make_float2(-m_off, -m_off));
                     const float2 a23 = __fadd2_rn(make_float2(lg[2], lg[3]), make_float2(-m_off, -m_off));
                     pr[0] = ex2(a01.x); pr[1] = ex2(a01.y); pr[2] = ex2(a23.x); pr[3] = ex2(a23.y);
                 }
-                if (__any_sync(0xffffffffu, m_new != m_run)) {     // some head's running max moved
-                    const float corr = ex2(m_run - m_use);
-                    // the accumulator columns are heads 2tig and 2tig+1: their factors sit in lanes 8tig, 8tig+4
-                    const float ca = __shfl_sync(0xffffffffu, corr, 8 * tig);
-                    const float cb = __shfl_sync(0xffffffffu, corr, 8 * tig + 4);
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        o[m][0] *= ca; o[m][1] *= cb; o[m][2] *= ca; o[m][3] *= cb;
-                    }
-#pragma unroll
-                    for (int g = 0; g < G8; ++g) zacc[g] *= corr;
-                    l_run *= corr;
-                }
                 l_run += (pr[0] + pr[1]) + (pr[2] + pr[3]);
-                m_run = m_new;
-                // ---- zero term on FMAs: zacc[g] += p * z
-                const __half* zch = reinterpret_cast<const __half*>(st + C::kZOff) + warp * 16 * G8;
-                const __half* sch = reinterpret_cast<const __half*>(st + C::kSOff) + warp * 16 * G8;
-                const uint8_t* vch = st + C::kVOff + warp * 16 * C::kVRow;
+                // ---- scale and zero rows of the lane's four tokens: one vector load per token and array
+                float sf[4][G8], zf[4][G8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    float zr[G8];
-                    load_halves<G8>(zch + tok[e] * G8, zr);
+                    const int toff = (e & 1) + 8 * (e >> 1);
+                    load_halves<G8>(reinterpret_cast<const __half*>(stg + o_scl + toff * G8 * 2), sf[e]);
+                    load_halves<G8>(reinterpret_cast<const __half*>(stg + o_zer + toff * G8 * 2), zf[e]);
+                }
+                // ---- zero term on FMAs: zacc[g] += p * z
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
                     if constexpr (G8 % 2 == 0) {
-                        // two groups per packed f32x2 FMA
 #pragma unroll
                         for (int g = 0; g < G8; g += 2) {
-                            const float2 t = __ffma2_rn(make_float2(pr[e], pr[e]), make_float2(zr[g], zr[g + 1]),
+                            const float2 t = __ffma2_rn(make_float2(pr[e], pr[e]), make_float2(zf[e][g], zf[e][g + 1]),
                                                         make_float2(zacc[g], zacc[g + 1]));
                             zacc[g] = t.x;
                             zacc[g + 1] = t.y;
                         }
                     } else {
 #pragma unroll
-                        for (int g = 0; g < G8; ++g) zacc[g] = fmaf(pr[e], zr[g], zacc[g]);
+                        for (int g = 0; g < G8; ++g) zacc[g] = fmaf(pr[e], zf[e][g], zacc[g]);
                     }
                 }
                 // ---- values: A = codes (exact bf16), B = hi/lo of p * scale; per 32-column slice
+                const uint8_t* vch = stg + o_val;
                 uint32_t bh0 = 0, bh1 = 0, bl0 = 0, bl1 = 0;
 #pragma unroll
                 for (int sl = 0; sl < NSL; ++sl) {
                     const int g = (32 * sl) / VG;
                     if (sl == 0 || (32 * sl) % VG == 0) {
-                        const float2 x01 = __fmul2_rn(make_float2(pr[0], pr[1]),
-                                                      make_float2(__half2float(sch[tok[0] * G8 + g]), __half2float(sch[tok[1] * G8 + g])));
-                        const float2 x23 = __fmul2_rn(make_float2(pr[2], pr[3]),
-                                                      make_float2(__half2float(sch[tok[2] * G8 + g]), __half2float(sch[tok[3] * G8 + g])));
+                        const float2 x01 = __fmul2_rn(make_float2(pr[0], pr[1]), make_float2(sf[0][g], sf[1][g]));
+                        const float2 x23 = __fmul2_rn(make_float2(pr[2], pr[3]), make_float2(sf[2][g], sf[3][g]));
                         split_bf16(x01, bh0, bl0);
                         split_bf16(x23, bh1, bl1);
                     }
                     uint32_t f[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) f[e] = vfield<VB>(vch + tok[e] * C::kVRow, sl, gid);
+                    for (int e = 0; e < 4; ++e) f[e] = vfield<VB>(vch + ((e & 1) + 8 * (e >> 1)) * C::kVRow, sl, gid);
 #pragma unroll
                     for (int hm = 0; hm < 2; ++hm) {
                         uint4 a;
                         if constexpr (VB == 8) {
-                            // bytes pos of both tokens into the low bytes of the 16-bit halves, pos = 2 hm (+1)
                             const uint32_t s0 = 0x4400u + 0x1111u * (2 * hm), s1 = s0 + 0x1111u;
                             a.x = __byte_perm(f[0], f[1], s0) & 0x00FF00FFu;
                             a.y = __byte_perm(f[0], f[1], s1) & 0x00FF00FFu;
@@ -855,22 +874,26 @@ __global__ void __launch_bounds__(128) attend_scores_kernel(const AttendParams p
 }
 
 // Split-K merge: out[b][h*G+g][:] = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M), M = max_s m_s.
-// One CTA per (g, h, b).  Slice k of the CTA's threads (D threads, one per column) folds splits k, k + kSlices,
-// ... with every load issued before the first is used, so the partials cost one round trip; the slices are
-// then combined in shared memory the same way.
-constexpr int kMergeThreads = 1024;
+// Grid (G * D/32, H_kv, B): each CTA merges 32 columns of one (query head, kv head, sequence), so the partials
+// are read by four times as many SMs as with one CTA per head.  Slice k of the CTA's threads folds splits
+// k, k + kSlices, ... with every load issued before the first is used (one round trip per batch); the slices
+// are then combined in shared memory the same way.
+constexpr int kMergeThreads = 256;
+constexpr int kMergeCols = 32;
 constexpr int kMaxSplits = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kMergeThreads) attend_merge_kernel(const AttendParams p) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     constexpr int kPart = 16 + 8 * D;
-    constexpr int kSlices = kMergeThreads / D;
+    constexpr int kCS = D / kMergeCols;
+    constexpr int kSlices = kMergeThreads / kMergeCols;
     constexpr int kBatch = 12;                           // splits per slice per round of loads
-    __shared__ float s_o[kSlices][D];
+    __shared__ float s_o[kSlices][kMergeCols];
     __shared__ float s_ml[kSlices][2];
-    const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-    const int col = tid % D, slice = tid / D;
+    const int g = blockIdx.x / kCS, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    const int lc = tid % kMergeCols, slice = tid / kMergeCols;
+    const int col = (blockIdx.x % kCS) * kMergeCols + lc;
     const int S = p.num_parts;
     const float* base = p.partials + (static_cast<int64_t>(b) * p.num_kv_heads + h) * S * kPart;
     float M = -INFINITY, L = 0.f, O = 0.f;
@@ -899,8 +922,8 @@ __global__ void __launch_bounds__(kMergeThreads) attend_merge_kernel(const Atten
         }
         M = Mn;
     }
-    s_o[slice][col] = O;
-    if (col == 0) {
+    s_o[slice][lc] = O;
+    if (lc == 0) {
         s_ml[slice][0] = M;
         s_ml[slice][1] = L;
     }
@@ -915,7 +938,7 @@ __global__ void __launch_bounds__(kMergeThreads) attend_merge_kernel(const Atten
         for (int k = 0; k < kSlices; ++k) {
             const float f = exp2f(s_ml[k][0] - Mu);
             Lt = fmaf(s_ml[k][1], f, Lt);
-            Ot = fmaf(s_o[k][col], f, Ot);
+            Ot = fmaf(s_o[k][lc], f, Ot);
         }
         p.out[(static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * p.group + g) * D + col] =
             (Lt > 0.f) ? Ot / Lt : 0.f;

@@ -262,6 +262,17 @@ __device__ __forceinline__ float fma_f16_f32(uint16_t h, float acc) {
 // A table replicated once per shared-memory bank (entry e of lane l at word 32 e + l) filled from `entries` words
 // of global memory by all threads of the block: each entry is read once and written as eight 16-byte stores, so
 // the fill costs one round trip to L2 per thread instead of one per word.
+__device__ __forceinline__ void fill_replicated_by(uint32_t* dst, const uint32_t* __restrict__ src, int entries,
+                                                   int tid, int nthreads) {
+    for (int e = tid; e < entries; e += nthreads) {
+        const uint32_t v = __ldg(src + e);
+        uint4* d = reinterpret_cast<uint4*>(dst + 32 * e);
+        const uint4 q = make_uint4(v, v, v, v);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) d[k] = q;
+    }
+}
+
 __device__ __forceinline__ void fill_replicated(uint32_t* dst, const uint32_t* __restrict__ src, int entries) {
     for (int e = threadIdx.x; e < entries; e += blockDim.x) {
         const uint32_t v = __ldg(src + e);

@@ -571,7 +571,7 @@ tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const tq_att
     cfg.numAttrs = 1;
     TQ_CUDA(cudaLaunchKernelEx(&cfg, kern, p), "tq_attend_decode: launch");
     if (plan.num_parts > 1) {
-        cfg.gridDim = dim3(p.group, a->num_kv_heads, a->batch);
+        cfg.gridDim = dim3(p.group * (D / kMergeCols), a->num_kv_heads, a->batch);
         cfg.blockDim = dim3(kMergeThreads);
         cfg.dynamicSmemBytes = 0;
         TQ_CUDA(cudaLaunchKernelEx(&cfg, attend_merge_kernel<D>, p), "tq_attend_decode: merge launch");
