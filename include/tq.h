@@ -346,6 +346,75 @@ tq_status tq_attend_decode_window(const tq_codec* codec, const tq_attend_args* a
 tq_status tq_attend_decode_noalloc(const tq_codec* codec, const tq_attend_args* args, void* stream);
 
 /* --------------------------------------------------------------------------------------------------
+ * QJL residual keys.
+ * ------------------------------------------------------------------------------------------------ */
+
+/*
+ * tq_codec_create_qjl -- a key codec for QJL residual keys ("KV Cache API", compressors.py
+ * TurboQuantCompressorV2: the MSE compressor at bits - 1, then one sign bit per row of a seeded Gaussian matrix S
+ * applied to the residual r of the MSE reconstruction, and ||r||).
+ *   bits      total bits per coordinate, 2..5; the MSE stage uses bits - 1 (tq_codec_info reports bits - 1, so
+ *             the codec also serves tq_encode_k / tq_decode_k / tq_attend_decode as an ordinary key codec).
+ *   S         d x d, entry (i, j) = Gaussian draw i * d + j of this library's generator (SplitMix64 and
+ *             Box-Muller) seeded with seed + 10000; the tensor cores multiply by S_op = fp16(S).
+ * Errors: as tq_codec_create_ex, TQ_ERR_UNSUPPORTED for bits outside 2..5.
+ */
+tq_status tq_codec_create_qjl(int d, int bits, uint64_t seed, int rotation, tq_codec** out);
+
+/*
+ * tq_make_qjl_matrix -- the sketch S of a QJL codec with this d and seed, on the host (row-major d*d): entry
+ * (i, j) is Gaussian draw i * d + j of the generator seeded with seed + 10000; s_f16 (nullable) receives
+ * fp16(S), the operand the kernels use.  Either output may be NULL, not both.
+ */
+tq_status tq_make_qjl_matrix(int d, uint64_t seed, double* s, uint16_t* s_f16);
+
+/* tq_codec_qjl_bits -- the total bits of a QJL codec; 0 for a codec made by tq_codec_create / _ex. */
+tq_status tq_codec_qjl_bits(const tq_codec* codec, int* bits);
+
+/*
+ * tq_encode_k_qjl -- QJL key encode ("KV Cache API", compressors.py TurboQuantCompressorV2.compress):
+ *   the MSE stage, exactly tq_encode_k with this codec at bits - 1, into packed and norms; then
+ *   k_mse = n * Pi_op^T c_op[idx];  r = x - k_mse (f32);  rho = ||r|| (f32);  sign_i = ((S_op r)_i >= 0).
+ *   signs     out, device: rows of d/8 bytes; coordinate i is bit i of the row's LSB-first bitstream, 1 for +1.
+ *   rho       out, device: float per row.
+ * Rows, strides, alignment and the slot mapping (which places packed, norms, signs and rho alike) are those of
+ * tq_encode_k.  k_mse multiplies fp16 codebook values by fp16 Pi_op and S_op r multiplies r, split into fp16
+ * hi + lo halves, by fp16 S_op, both with f32 accumulation: a sign can differ from an exact evaluation only
+ * where (S_op r)_i lies within about 1e-6 * ||S_op row i|| * ||x|| of zero.  Launches two kernels on `stream`.
+ * Errors: as tq_encode_k; TQ_ERR_INVALID_ARG for a codec not made by tq_codec_create_qjl or NULL signs / rho.
+ */
+tq_status tq_encode_k_qjl(const tq_codec* codec, const void* x, int64_t n, int64_t x_row_stride,
+                          const int64_t* slot_mapping, uint8_t* packed, float* norms, uint8_t* signs, float* rho,
+                          void* stream);
+
+/* QJL key pools beside the MSE-stage pools of tq_attend_args, indexed by the same rows. */
+typedef struct tq_qjl_keys {
+    const uint8_t* signs;      /* device pool of sign rows (tq_encode_k_qjl format: d/8 bytes per row) */
+    const float* rho;          /* device pool of residual norms */
+} tq_qjl_keys;
+
+/*
+ * tq_attend_qjl_workspace_bytes -- workspace bytes tq_attend_decode_qjl needs: as tq_attend_workspace_bytes, with
+ * a second block of prepared query fragments (the sketched query) per (sequence, kv head).
+ */
+tq_status tq_attend_qjl_workspace_bytes(const tq_attend_args* args, size_t* bytes);
+
+/*
+ * tq_attend_decode_qjl -- decode attention over QJL residual keys ("KV Cache API", store.py attention_scores
+ * with compressors.py asymmetric_attention_scores): for each (b, hq), kv head h = hq / G,
+ *   s_t = scale * ( n_t <Pi_op q, c_op[idx_t]> + rho_t sqrt(pi/2) / d <S_op q, sign_t> ),  sign_t in {-1, +1}^d,
+ *   p = softmax(s);  out = sum_t p_t * (q_t * scale16_t + zero16_t),
+ * i.e. tq_attend_decode with the estimator's second term in every logit.  args describes the MSE-stage pools
+ * (the codec's bits - 1 codes and norms) and the values exactly as for tq_attend_decode; keys adds the sign and
+ * rho pools.  The prepared query now has two halves (Pi_op q and S_op q, each fp16 hi + lo fragments); the sign
+ * pairs enter the tensor cores as fp16 +-1.  Values: 2 or 4 bits in groups of 32.
+ * Errors: as tq_attend_decode; TQ_ERR_INVALID_ARG for a codec not made by tq_codec_create_qjl, NULL or
+ * misaligned (16-byte) signs / rho; TQ_ERR_UNSUPPORTED for another value format.
+ */
+tq_status tq_attend_decode_qjl(const tq_codec* codec, const tq_attend_args* args, const tq_qjl_keys* keys,
+                               void* stream);
+
+/* --------------------------------------------------------------------------------------------------
  * Diagnostics.
  * ------------------------------------------------------------------------------------------------ */
 

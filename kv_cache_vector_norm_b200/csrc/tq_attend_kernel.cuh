@@ -44,6 +44,13 @@ struct AttendParams {
     const __half* win_v;
     const int32_t* win_lens;                         // nullable: win_max for every sequence
     int win_max;
+    int qfrag_stride;                                // uint4 slots per (sequence, kv head) of qfrag
+    // QJL residual keys (the kernels' QJL instantiations only)
+    const uint8_t* k_signs;                          // pool of sign rows, d/8 bytes, LSB-first (1 = +1)
+    const float* k_rho;                              // pool of residual norms
+    const __half* s_op;                              // d x d sketch, row-major
+    float s_scale_log2;                              // softmax scale * log2(e) * sqrt(pi/2) / d
+    float s_row_bound;                               // max over rows of ||S_op row||
 };
 
 constexpr int kWinMax = 256;                         // largest window per (sequence, kv head)
@@ -59,7 +66,7 @@ __host__ __device__ constexpr int window_smem_floats() {
 template <int D>
 __host__ __device__ constexpr int qfrag_slots() { return (D / 16) * 32 + 2; }
 
-template <int D, int KB, int VB, int VG>
+template <int D, int KB, int VB, int VG, bool QJL = false>
 struct AttCfg {
     static constexpr int kWarps = 4;                 // consumer warps
     static constexpr int kThreads = 32 * (kWarps + 1);
@@ -77,7 +84,11 @@ struct AttCfg {
     static constexpr int kVOff = kNOff + kTileTok * 4;
     static constexpr int kSOff = kVOff + kTileTok * kVRow;
     static constexpr int kZOff = kSOff + kTileTok * kVGroups * 2;
-    static constexpr int kStageBytes = kZOff + kTileTok * kVGroups * 2;
+    // QJL: the sign rows (d/8 bytes) and residual norms of the tile follow the value arrays
+    static constexpr int kSgRow = D / 8;
+    static constexpr int kSgOff = kZOff + kTileTok * kVGroups * 2;
+    static constexpr int kRhoOff = kSgOff + (QJL ? kTileTok * kSgRow : 0);
+    static constexpr int kStageBytes = kRhoOff + (QJL ? kTileTok * 4 : 0);
     static constexpr int kQuarterBits = D * KB / 4;  // one lane's quarter of a key row (16-bit multiple)
     static constexpr int kQuarterHalves = kQuarterBits / 16;
     static constexpr int kQuarterWords = (kQuarterHalves + 1) / 2 + 1;
@@ -96,17 +107,21 @@ struct AttCfg {
     static constexpr int kRingBytes =
         (kStages * kStageBytes > kCombineFloats * 4) ? kStages * kStageBytes : kCombineFloats * 4;
     static constexpr int kQfOff = kRingBytes;
-    static constexpr int kLutOff = kQfOff + (kQInRegs ? 0 : (D / 16) * 32 * 16);
+    static constexpr int kLutOff = kQfOff + (kQInRegs ? 0 : (QJL ? 2 : 1) * (D / 16) * 32 * 16);
     // tables up to 8 KB (key widths 1..3) start on a multiple of their size (slack reserved), so an entry's
     // address is (pair bits << 7) | lane bits; the 32 KB table of 4-bit keys would need 32 KB of slack and cost
     // resident CTAs, so it sits unaligned and its addresses are base + (pair bits << 7) + lane bits
     static constexpr bool kLutAligned = (kLutBytes <= 8192);
-    static constexpr int kZsOff = kLutOff + (kLutAligned ? 2 : 1) * kLutBytes;
+    // QJL: a table of the four sign pairs (two bits -> half2 of +-1), replicated per bank like the key table and
+    // aligned to its 512 bytes (slack reserved)
+    static constexpr int kSLutOff = kLutOff + (kLutAligned ? 2 : 1) * kLutBytes;
+    static constexpr int kZsOff = kSLutOff + (QJL ? 1024 : 0);
     static constexpr int kBarOff = (kZsOff + kWarps * 8 * kVGroups * 4 + 15) & ~15;
     static constexpr int kSmemMain = kBarOff + 8 * (2 * kStages) + 16;
     // the window CTA reuses the same allocation
     static constexpr int kSmem = (kSmemMain > window_smem_floats<D>() * 4) ? kSmemMain : window_smem_floats<D>() * 4;
-    static_assert(kNOff % 16 == 0 && kVOff % 16 == 0 && kSOff % 16 == 0 && kZOff % 16 == 0 && kStageBytes % 16 == 0,
+    static_assert(kNOff % 16 == 0 && kVOff % 16 == 0 && kSOff % 16 == 0 && kZOff % 16 == 0 && kSgOff % 16 == 0 &&
+                      kRhoOff % 16 == 0 && kStageBytes % 16 == 0,
                   "bulk copies need 16-byte multiples");
     static_assert(VG % 32 == 0, "a 32-column slice of the value row lies in one scale group");
 };
@@ -241,6 +256,9 @@ __device__ __forceinline__ int64_t attend_seq_len(const AttendParams& p, int b) 
 // no reduction over q_rot is needed: CTA x of grid (d / 32, H_kv, B) computes n-tiles 4x .. 4x + 3 (one per
 // warp) and writes their fragments straight from the MMA accumulators.  The attention grid is its
 // programmatic dependent.
+// With QJL residual keys the grid is (2 d / 32, H_kv, B): CTAs x >= d / 32 prepare, the same way, the sketched
+// query S_op q scaled by softmax scale * log2(e) * sqrt(pi/2) / d (the estimator's factor), whose bound is
+// ||S_op row||_max ||q||, into a second block of fragments.
 constexpr int kPrepThreads = 128;
 
 template <int D>
@@ -248,17 +266,23 @@ __global__ void __launch_bounds__(kPrepThreads) attend_prep_kernel(const AttendP
     constexpr int KS = D / 16;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;
-    const int nt = blockIdx.x * (kPrepThreads / 32) + warp;      // n-tile: columns 8 nt .. 8 nt + 7
+    const bool sketch = blockIdx.x >= D / 32;                   // the QJL block: S_op q
+    const int bx = sketch ? blockIdx.x - D / 32 : blockIdx.x;
+    const int nt = bx * (kPrepThreads / 32) + warp;             // n-tile: columns 8 nt .. 8 nt + 7
     const int h = blockIdx.y, b = blockIdx.z;
     const int G = p.group;
-    uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();
+    uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * p.qfrag_stride +
+                (sketch ? qfrag_slots<D>() : 0);
+    const __half* mat = sketch ? p.s_op : p.pi_op;
+    const float scale_log2 = sketch ? p.s_scale_log2 : p.scale_log2;
+    const float mat_bound = sketch ? p.s_row_bound : 1.0625f;
     // the attention grid may be scheduled at once and start streaming the cache; its consumers wait for this
     // grid's completion (griddepcontrol.wait) before they read the fragments
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const __half* qg = p.q + (static_cast<int64_t>(b) * p.num_q_heads + static_cast<int64_t>(h) * G) * D;
     // every fragment is loaded before the first MMA, so the loads overlap
     uint32_t bf[KS][2], af[KS][2];
-    const __half* prow = p.pi_op + (8 * nt + gid) * D + 2 * tig;
+    const __half* prow = mat + (8 * nt + gid) * D + 2 * tig;
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
         bf[ks][0] = __ldg(reinterpret_cast<const uint32_t*>(prow + 16 * ks));
@@ -278,7 +302,7 @@ __global__ void __launch_bounds__(kPrepThreads) attend_prep_kernel(const AttendP
     }
     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
     ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-    const float bound = sqrtf(ss) * fabsf(p.scale_log2) * 1.0625f;
+    const float bound = sqrtf(ss) * fabsf(scale_log2) * mat_bound;
     // bound = m 2^ex with m in [0.5, 1); pre = 2^(14 - ex), so |x| * pre < 2^15 (zero or tiny queries clamped)
     int ex = static_cast<int>((__float_as_uint(bound) >> 23) & 255u) - 126;
     ex = (bound > 0.f) ? max(ex, -100) : 14;
@@ -292,7 +316,7 @@ __global__ void __launch_bounds__(kPrepThreads) attend_prep_kernel(const AttendP
     float hi[2], lo[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-        const float x = c[e] * p.scale_log2 * pre;
+        const float x = c[e] * scale_log2 * pre;
         hi[e] = __half2float(__float2half_rn(x));
         lo[e] = x - hi[e];
     }
@@ -303,7 +327,7 @@ __global__ void __launch_bounds__(kPrepThreads) attend_prep_kernel(const AttendP
         const int tg = col / (D / 4), ks = (col % (D / 4)) / 4;
         qf[ks * 32 + gid * 4 + tg] = make_uint4(h01, l01, h23, l23);
     }
-    if (blockIdx.x == 0 && warp == 0 && tig == 0) reinterpret_cast<float*>(qf + KS * 32)[gid] = 1.0f / pre;
+    if (bx == 0 && warp == 0 && tig == 0) reinterpret_cast<float*>(qf + KS * 32)[gid] = 1.0f / pre;
 }
 
 // The window part of one (sequence, kv head): scores of the group's queries against the recent uncompressed
@@ -422,10 +446,12 @@ __device__ void attend_window_partial(const AttendParams& p, int b, int h, uint8
 //   values  O^T[col][head] += (value codes, bf16 A, exact) x (hi/lo of p * scale, bf16 B)
 // so each lane's probabilities (head gid, tokens 2tig, 2tig+1, 2tig+8, 2tig+9) are already the B fragment
 // of the value product, and the accumulator is D/16 x 4 registers.
-template <int D, int KB, int VB, int VG>
-__global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB, VB, VG>::kMinBlocks)
+// QJL: the keys are QJL residual keys; each chunk adds a second score contraction, the sketched query S_op q
+// against the keys' sign bits as +-1 pairs, weighted by the key's residual norm.
+template <int D, int KB, int VB, int VG, bool QJL = false>
+__global__ void __launch_bounds__(AttCfg<D, KB, VB, VG, QJL>::kThreads, AttCfg<D, KB, VB, VG, QJL>::kMinBlocks)
     attend_kernel(const AttendParams p) {
-    using C = AttCfg<D, KB, VB, VG>;
+    using C = AttCfg<D, KB, VB, VG, QJL>;
     constexpr int S = C::kStages;
     constexpr int KS = D / 16;                        // k-steps of the score contraction
     constexpr int MT = D / 16;                        // m-tiles (16 value columns) of the value contraction
@@ -443,6 +469,7 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         ? (smem_u32(smem + C::kLutOff) + C::kLutBytes - 1) & ~static_cast<uint32_t>(C::kLutBytes - 1)
         : smem_u32(smem + C::kLutOff);
     uint32_t* lut = reinterpret_cast<uint32_t*>(smem + (lut_addr - smem_u32(smem)));
+    const uint32_t slut_addr = (smem_u32(smem + C::kSLutOff) + 511u) & ~511u;    // QJL sign pairs
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tig = lane & 3;
@@ -497,6 +524,10 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                     bulk_load(smem_u32(st + C::kVOff), p.v_data + row0 * C::kVRow, rows * C::kVRow, bar);
                     bulk_load(smem_u32(st + C::kSOff), p.v_scales + row0 * G8, rows * G8 * 2, bar);
                     bulk_load(smem_u32(st + C::kZOff), p.v_zeros + row0 * G8, rows * G8 * 2, bar);
+                    if constexpr (QJL) {
+                        bulk_load(smem_u32(st + C::kSgOff), p.k_signs + row0 * C::kSgRow, rows * C::kSgRow, bar);
+                        bulk_load(smem_u32(st + C::kRhoOff), p.k_rho + row0, rows * 4, bar);
+                    }
                 } else {
                     for (int c = 0; c < nc; ++c) {
                         const int64_t blk = p.block_table[static_cast<int64_t>(b) * p.max_blocks + c0 + c];
@@ -508,6 +539,11 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                                   16 * C::kVRow, bar);
                         bulk_load(smem_u32(st + C::kSOff + c * 32 * G8), p.v_scales + row0 * G8, 32 * G8, bar);
                         bulk_load(smem_u32(st + C::kZOff + c * 32 * G8), p.v_zeros + row0 * G8, 32 * G8, bar);
+                        if constexpr (QJL) {
+                            bulk_load(smem_u32(st + C::kSgOff + c * 16 * C::kSgRow), p.k_signs + row0 * C::kSgRow,
+                                      16 * C::kSgRow, bar);
+                            bulk_load(smem_u32(st + C::kRhoOff + c * 64), p.k_rho + row0, 64, bar);
+                        }
                     }
                 }
             }
@@ -519,11 +555,24 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
         // ------------------------------------------------------------------ query fragments
         // written by attend_prep_kernel, the grid this one depends on programmatically
         fill_replicated_by(lut, p.pair_lut, C::kPairs, threadIdx.x, 32 * C::kWarps);
+        if constexpr (QJL) {
+            // entry e = two sign bits (first coordinate in bit 0) -> half2 of +-1 (1 = +1), per bank as above
+            if (threadIdx.x < 4 * 32) {
+                const uint32_t e = threadIdx.x >> 5;
+                const uint32_t v = ((e & 1u) ? 0x3C00u : 0xBC00u) | (((e & 2u) ? 0x3C00u : 0xBC00u) << 16);
+                reinterpret_cast<uint32_t*>(smem + (slut_addr - smem_u32(smem)))[threadIdx.x] = v;
+            }
+        }
         asm volatile("griddepcontrol.wait;" ::: "memory");
-        const uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();
+        const uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * p.qfrag_stride;
         const float unpre = __ldcg(reinterpret_cast<const float*>(qf + KS * 32) + gid);   // head gid's
+        float unpre2 = 0.f;
+        if constexpr (QJL) unpre2 = __ldcg(reinterpret_cast<const float*>(qf + qfrag_slots<D>() + KS * 32) + gid);
         if constexpr (!C::kQInRegs) {
             for (int i = threadIdx.x; i < KS * 32; i += 32 * C::kWarps) s_qf[i] = __ldcg(qf + i);
+            if constexpr (QJL)
+                for (int i = threadIdx.x; i < KS * 32; i += 32 * C::kWarps)
+                    s_qf[KS * 32 + i] = __ldcg(qf + qfrag_slots<D>() + i);
         }
         named_bar_sync(1, 32 * C::kWarps);              // the table and the query fragments are in place
 
@@ -613,6 +662,41 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG>::kThreads, AttCfg<D, KB,
                     const float2 r1 = __fmul2_rn(__fadd2_rn(make_float2(sc[1][0], sc[1][1]), make_float2(sc[1][2], sc[1][3])),
                                                  __fmul2_rn(n89, u2));
                     lg[0] = r0.x; lg[1] = r0.y; lg[2] = r1.x; lg[3] = r1.y;
+                }
+                if constexpr (QJL) {
+                    // QJL term: rho_t * <S_op q, signs_t> (the prepared fragments carry scale log2(e) sqrt(pi/2)/d);
+                    // this lane's quarter of the sign row of token 8 nt + gid holds coordinates tig d/4 ..
+                    constexpr int kSW = (D / 4 + 31) / 32;
+                    uint32_t sw[2][kSW + 1];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const uint8_t* srow = stg + C::kSgOff + (warp * 16 + 8 * nt + gid) * C::kSgRow + tig * (D / 32);
+                        if constexpr (D == 64) {
+                            sw[nt][0] = *reinterpret_cast<const uint16_t*>(srow);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < kSW; ++i) sw[nt][i] = reinterpret_cast<const uint32_t*>(srow)[i];
+                        }
+                        sw[nt][kSW] = 0u;
+                    }
+                    const uint32_t slane = slut_addr + 4u * lane;
+                    float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                    for (int ks = 0; ks < KS; ++ks) {
+                        const uint4 a = s_qf[KS * 32 + ks * 32 + lane];
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt) {
+                            const uint32_t e0 = window_shr(sw[nt], 4 * ks - 7) & (3u << 7);
+                            const uint32_t e1 = window_shr(sw[nt], 4 * ks + 2 - 7) & (3u << 7);
+                            mma_f16(s2[nt], a, lds_u32(slane | e0), lds_u32(slane | e1));
+                        }
+                    }
+                    const float2 rh01 = *reinterpret_cast<const float2*>(stg + C::kRhoOff + (warp * 16 + t0) * 4);
+                    const float2 rh89 = *reinterpret_cast<const float2*>(stg + C::kRhoOff + (warp * 16 + t0 + 8) * 4);
+                    lg[0] = fmaf((s2[0][0] + s2[0][2]) * unpre2, rh01.x, lg[0]);
+                    lg[1] = fmaf((s2[0][1] + s2[0][3]) * unpre2, rh01.y, lg[1]);
+                    lg[2] = fmaf((s2[1][0] + s2[1][2]) * unpre2, rh89.x, lg[2]);
+                    lg[3] = fmaf((s2[1][1] + s2[1][3]) * unpre2, rh89.y, lg[3]);
                 }
                 if (rel == nrel - 1 && last_valid < 16) {          // the sequence's last, partial chunk
                     lg[0] = (t0 < last_valid) ? lg[0] : -INFINITY;
@@ -810,7 +894,7 @@ __global__ void __launch_bounds__(128) attend_scores_kernel(const AttendParams p
     fill_replicated(lut, p.pair_lut, kPairs);
     __syncthreads();
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * qfrag_slots<D>();
+    const uint4* qf = p.qfrag + (static_cast<int64_t>(b) * p.num_kv_heads + h) * p.qfrag_stride;
     const float unpre = __ldcg(reinterpret_cast<const float*>(qf + KS * 32) + gid);
     const int64_t T = attend_seq_len(p, b);
     const int64_t chunk = static_cast<int64_t>(blockIdx.x) * 4 + warp;

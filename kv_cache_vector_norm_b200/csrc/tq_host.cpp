@@ -46,7 +46,7 @@ static inline uint64_t splitmix64_at(uint64_t seed, uint64_t i) {
     return z ^ (z >> 31);
 }
 
-static void gaussians(uint64_t seed, size_t count, double* out) {
+void host_gaussians(uint64_t seed, size_t count, double* out) {
     const double two_pi = 6.283185307179586476925286766559;
     for (size_t p = 0; 2 * p < count; ++p) {
         double u1 = (static_cast<double>(splitmix64_at(seed, 2 * p) >> 11) + 0.5) * 0x1.0p-53;
@@ -62,7 +62,7 @@ static void gaussians(uint64_t seed, size_t count, double* out) {
 void host_rotation(int d, uint64_t seed, double* pi) {
     const size_t n = static_cast<size_t>(d);
     std::vector<double> a(n * n), vs(n * n, 0.0);   // a: working matrix (row-major); vs: reflectors
-    gaussians(seed, n * n, a.data());
+    host_gaussians(seed, n * n, a.data());
     std::vector<double> rdiag(n);
     // Householder QR: for column k, reflect a[k:, k] onto a multiple of e_k.
     for (size_t k = 0; k < n; ++k) {
@@ -314,6 +314,20 @@ extern "C" tq_status tq_make_rotation_ex(int d, uint64_t seed, int rotation, dou
     if (pi) std::memcpy(pi, m.data(), m.size() * sizeof(double));
     if (pi_f16)
         for (size_t i = 0; i < m.size(); ++i) pi_f16[i] = tq::f64_to_f16(m[i]);
+    return TQ_OK;
+}
+
+extern "C" tq_status tq_make_qjl_matrix(int d, uint64_t seed, double* s, uint16_t* s_f16) {
+    tq::clear_error();
+    if (d < 1 || d > 4096) return tq::fail(TQ_ERR_INVALID_ARG, "tq_make_qjl_matrix: d=%d outside [1, 4096]", d);
+    if (!s && !s_f16) return tq::fail(TQ_ERR_INVALID_ARG, "tq_make_qjl_matrix: both outputs are NULL");
+    const size_t dd = static_cast<size_t>(d) * d;
+    std::vector<double> g(dd);
+    tq::host_gaussians(seed + 10000, dd, g.data());
+    for (size_t i = 0; i < dd; ++i) {
+        if (s) s[i] = g[i];
+        if (s_f16) s_f16[i] = tq::f64_to_f16(g[i]);
+    }
     return TQ_OK;
 }
 

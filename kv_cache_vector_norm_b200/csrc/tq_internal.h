@@ -11,6 +11,10 @@ namespace tq {
 tq_status fail(tq_status status, const char* fmt, ...);
 void clear_error();
 
+// count standard normal draws of the seeded generator: SplitMix64 outputs 2p and 2p+1 give draws 2p and 2p+1
+// through the Box-Muller transform.
+void host_gaussians(uint64_t seed, size_t count, double* out);
+
 // Seeded Haar rotation (row-major d*d doubles): QR of a SplitMix64/Box-Muller Gaussian matrix by
 // Householder reflections, Q's columns multiplied by sign(diag R) (zero taken as +1).
 void host_rotation(int d, uint64_t seed, double* pi);

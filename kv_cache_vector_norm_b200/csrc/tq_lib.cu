@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "tq_attend_kernel.cuh"
+#include "tq_qjl_kernel.cuh"
 #include "tq_codec_kernels.cuh"
 #include "tq_internal.h"
 
@@ -119,6 +120,9 @@ struct tq_codec {
     uint32_t* enc_lut = nullptr;    // kGridCells grid cells: boundary bits | count below (low 4 bits)
     uint32_t* pair_lut = nullptr;   // 2^(2 bits) half2 pairs
     CUtensorMap tmap_pi, tmap_pit;
+    int qjl_bits = 0;               // QJL codec: total bits per coordinate (bits + 1), else 0
+    __half* s_op = nullptr;         // QJL codec: the d x d Gaussian sketch S_op = fp16(S), row-major
+    float s_row_max = 0.f;          // QJL codec: max over rows of ||S_op row||
 };
 
 namespace {
@@ -218,8 +222,51 @@ extern "C" tq_status tq_codec_destroy(tq_codec* c) {
     cudaFree(c->pi_op_t);
     cudaFree(c->enc_lut);
     cudaFree(c->pair_lut);
+    cudaFree(c->s_op);
     cudaSetDevice(prev);
     delete c;
+    return TQ_OK;
+}
+
+extern "C" tq_status tq_codec_create_qjl(int d, int bits, uint64_t seed, int rotation, tq_codec** out) {
+    clear_error();
+    if (!out) return fail(TQ_ERR_INVALID_ARG, "tq_codec_create_qjl: out is NULL");
+    *out = nullptr;
+    if (bits < 2 || bits > 5)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_codec_create_qjl: bits=%d (supported: 2..5, an MSE stage of bits - 1)", bits);
+    tq_codec* c = nullptr;
+    tq_status st = tq_codec_create_ex(d, bits - 1, seed, rotation, &c);
+    if (st != TQ_OK) return st;
+    // S: Gaussian draws i * d + j of the generator seeded with seed + 10000; the tensor cores multiply by fp16(S)
+    const size_t dd = static_cast<size_t>(d) * d;
+    std::vector<double> sg(dd);
+    host_gaussians(seed + kQjlSeedOffset, dd, sg.data());
+    std::vector<uint16_t> s16(dd);
+    double row_max = 0.0;
+    for (int i = 0; i < d; ++i) {
+        double ss = 0.0;
+        for (int j = 0; j < d; ++j) {
+            s16[static_cast<size_t>(i) * d + j] = f64_to_f16(sg[static_cast<size_t>(i) * d + j]);
+            const double v = f16_to_f64(s16[static_cast<size_t>(i) * d + j]);
+            ss += v * v;
+        }
+        row_max = std::max(row_max, std::sqrt(ss));
+    }
+    c->s_row_max = static_cast<float>(row_max * (1.0 + 1e-6));
+    if (cudaMalloc(&c->s_op, dd * 2) != cudaSuccess ||
+        cudaMemcpy(c->s_op, s16.data(), dd * 2, cudaMemcpyHostToDevice) != cudaSuccess) {
+        tq_codec_destroy(c);
+        return fail(TQ_ERR_CUDA, "tq_codec_create_qjl: upload of the sketch failed");
+    }
+    c->qjl_bits = bits;
+    *out = c;
+    return TQ_OK;
+}
+
+extern "C" tq_status tq_codec_qjl_bits(const tq_codec* c, int* bits) {
+    clear_error();
+    if (!c || !bits) return fail(TQ_ERR_INVALID_ARG, "tq_codec_qjl_bits: codec and bits must be non-NULL");
+    *bits = c->qjl_bits;
     return TQ_OK;
 }
 
@@ -319,6 +366,42 @@ extern "C" tq_status tq_encode_k(const tq_codec* c, const void* x, int64_t n, in
     if (slot_mapping && !aligned(slot_mapping, 8)) return fail(TQ_ERR_INVALID_ARG, "tq_encode_k: slot_mapping misaligned");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     TQ_DISPATCH_DB(c->d, c->bits, launch_encode_k, c, x, n, x_row_stride, slot_mapping, packed, norms, st);
+}
+
+namespace {
+
+template <int D, int KB>
+tq_status launch_qjl_residual(const tq_codec* c, const void* x, int64_t n, int64_t stride, const int64_t* slots,
+                              const uint8_t* packed, const float* norms, uint8_t* signs, float* rho, cudaStream_t st) {
+    static std::atomic<uint64_t> mask{0};
+    constexpr uint32_t smem = qjl_smem_bytes<D, KB>();
+    auto kern = qjl_residual_kernel<D, KB>;
+    TQ_CUDA(allow_smem(kern, smem, mask), "tq_encode_k_qjl: cudaFuncSetAttribute");
+    const int64_t grid = (n + 16 * kQjlWarps - 1) / (16 * kQjlWarps);
+    kern<<<static_cast<unsigned>(grid), 32 * kQjlWarps, smem, st>>>(static_cast<const __half*>(x), n, stride, slots,
+                                                                     packed, norms, c->pair_lut, c->pi_op_t, c->s_op,
+                                                                     signs, rho);
+    TQ_CUDA(cudaGetLastError(), "tq_encode_k_qjl: residual launch");
+    return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" tq_status tq_encode_k_qjl(const tq_codec* c, const void* x, int64_t n, int64_t x_row_stride,
+                                     const int64_t* slot_mapping, uint8_t* packed, float* norms, uint8_t* signs,
+                                     float* rho, void* stream) {
+    clear_error();
+    if (!c) return fail(TQ_ERR_INVALID_ARG, "tq_encode_k_qjl: codec is NULL");
+    if (!c->qjl_bits) return fail(TQ_ERR_INVALID_ARG, "tq_encode_k_qjl: the codec was not made by tq_codec_create_qjl");
+    if (n == 0) return TQ_OK;
+    if (!signs || !rho) return fail(TQ_ERR_INVALID_ARG, "tq_encode_k_qjl: signs and rho must be non-NULL");
+    if (!aligned(rho, 4)) return fail(TQ_ERR_INVALID_ARG, "tq_encode_k_qjl: rho must be 4-byte aligned");
+    // the MSE stage: the codec's key encoder at bits - 1 (same checks and formats as tq_encode_k)
+    tq_status s = tq_encode_k(c, x, n, x_row_stride, slot_mapping, packed, norms, stream);
+    if (s != TQ_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TQ_DISPATCH_DB(c->d, c->bits, launch_qjl_residual, c, x, n, x_row_stride, slot_mapping, packed, norms, signs, rho,
+                   st);
 }
 
 extern "C" tq_status tq_decode_k(const tq_codec* c, const uint8_t* packed, const float* norms, int64_t n, void* out,
@@ -457,7 +540,7 @@ struct AttendPlan {
 // ctas_per_sm: attention CTAs resident per SM.  Workspace sizes are planned with the largest (4); a launch
 // re-plans with its kernel's measured occupancy, which never needs more splits, so the workspace suffices.
 tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan, bool window = false,
-                      int ctas_per_sm = kAttendCtasPerSm) {
+                      int ctas_per_sm = kAttendCtasPerSm, bool qjl = false) {
     if (!a) return fail(TQ_ERR_INVALID_ARG, "tq_attend: args is NULL");
     if (a->batch < 1 || a->num_kv_heads < 1 || a->num_q_heads < 1)
         return fail(TQ_ERR_INVALID_ARG, "tq_attend: batch, num_q_heads, num_kv_heads must be >= 1");
@@ -493,18 +576,19 @@ tq_status plan_attend(const tq_attend_args* a, AttendPlan* plan, bool window = f
     plan->num_parts = static_cast<int>(splits) + (window ? 1 : 0);
     plan->partial_bytes =
         (plan->num_parts > 1) ? static_cast<size_t>(bh) * plan->num_parts * (16 + 8 * a->head_dim) * 4 : 0;
-    plan->qfrag_bytes = static_cast<size_t>(bh) * ((a->head_dim / 16) * 32 + 2) * 16;
+    // prepared query fragments per (sequence, kv head): Pi_op q, and with QJL keys also S_op q
+    plan->qfrag_bytes = static_cast<size_t>(bh) * ((a->head_dim / 16) * 32 + 2) * 16 * (qjl ? 2 : 1);
     plan->workspace_bytes = plan->qfrag_bytes + plan->partial_bytes;
     return TQ_OK;
 }
 
-template <int D, int KB, int VB, int VG>
+template <int D, int KB, int VB, int VG, bool QJL = false>
 tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const tq_attend_window* win,
-                        const AttendPlan& plan_max, cudaStream_t st) {
-    using Cfg = AttCfg<D, KB, VB, VG>;
+                        const tq_qjl_keys* qjl, const AttendPlan& plan_max, cudaStream_t st) {
+    using Cfg = AttCfg<D, KB, VB, VG, QJL>;
     static std::atomic<uint64_t> mask{0};
     static std::atomic<int> occupancy[64];                // resident CTAs per SM, per device (0: not yet queried)
-    auto kern = attend_kernel<D, KB, VB, VG>;
+    auto kern = attend_kernel<D, KB, VB, VG, QJL>;
     TQ_CUDA(allow_smem(kern, Cfg::kSmem, mask), "tq_attend_decode: cudaFuncSetAttribute");
     int dev = 0;
     cudaGetDevice(&dev);
@@ -518,7 +602,7 @@ tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const tq_att
     // split the sequences so that the grid fills the resident CTAs once
     AttendPlan plan = plan_max;
     if (occ < kAttendCtasPerSm) {
-        tq_status s = plan_attend(a, &plan, win != nullptr, occ);
+        tq_status s = plan_attend(a, &plan, win != nullptr, occ, QJL);
         if (s != TQ_OK) return s;
     }
     AttendParams p;
@@ -549,13 +633,19 @@ tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const tq_att
     p.win_v = nullptr;
     p.win_lens = nullptr;
     p.win_max = 0;
+    p.qfrag_stride = qfrag_slots<D>() * (QJL ? 2 : 1);
+    p.k_signs = QJL ? qjl->signs : nullptr;
+    p.k_rho = QJL ? qjl->rho : nullptr;
+    p.s_op = c->s_op;
+    p.s_scale_log2 = p.scale_log2 * static_cast<float>(std::sqrt(std::acos(-1.0) / 2.0) / D);
+    p.s_row_bound = c->s_row_max;
     if (win) {
         p.win_k = static_cast<const __half*>(win->k);
         p.win_v = static_cast<const __half*>(win->v);
         p.win_lens = win->lens;
         p.win_max = win->max_len;
     }
-    attend_prep_kernel<D><<<dim3(D / 32, a->num_kv_heads, a->batch), kPrepThreads, 0, st>>>(p);
+    attend_prep_kernel<D><<<dim3((QJL ? 2 : 1) * D / 32, a->num_kv_heads, a->batch), kPrepThreads, 0, st>>>(p);
     TQ_CUDA(cudaGetLastError(), "tq_attend_decode: query preparation launch");
     // the attention grid and the split merge are programmatic dependents of the grid before them: each is
     // scheduled while its predecessor drains and waits for it (griddepcontrol.wait) before reading its output
@@ -580,18 +670,25 @@ tq_status launch_attend(const tq_codec* c, const tq_attend_args* a, const tq_att
 }
 
 template <int D, int KB>
-tq_status attend_v(const tq_codec* c, const tq_attend_args* a, const tq_attend_window* win, const AttendPlan& plan,
-                   cudaStream_t st) {
+tq_status attend_v(const tq_codec* c, const tq_attend_args* a, const tq_attend_window* win, const tq_qjl_keys* qjl,
+                   const AttendPlan& plan, cudaStream_t st) {
     const bool tok = a->v_group == D;
+    if (qjl) {
+        // QJL residual keys: values of 2 or 4 bits in groups of 32
+        if (!tok && a->v_bits == 2) return launch_attend<D, KB, 2, 32, true>(c, a, win, qjl, plan, st);
+        if (!tok && a->v_bits == 4) return launch_attend<D, KB, 4, 32, true>(c, a, win, qjl, plan, st);
+        return fail(TQ_ERR_UNSUPPORTED, "tq_attend_decode_qjl: v_bits=%d v_group=%d (supported: 2 or 4 bits, group 32)",
+                    a->v_bits, a->v_group);
+    }
     switch (a->v_bits * 2 + (tok ? 1 : 0)) {
-        case 4: return launch_attend<D, KB, 2, 32>(c, a, win, plan, st);
-        case 5: return launch_attend<D, KB, 2, D>(c, a, win, plan, st);
-        case 6: return launch_attend<D, KB, 3, 32>(c, a, win, plan, st);
-        case 7: return launch_attend<D, KB, 3, D>(c, a, win, plan, st);
-        case 8: return launch_attend<D, KB, 4, 32>(c, a, win, plan, st);
-        case 9: return launch_attend<D, KB, 4, D>(c, a, win, plan, st);
-        case 16: return launch_attend<D, KB, 8, 32>(c, a, win, plan, st);
-        case 17: return launch_attend<D, KB, 8, D>(c, a, win, plan, st);
+        case 4: return launch_attend<D, KB, 2, 32>(c, a, win, qjl, plan, st);
+        case 5: return launch_attend<D, KB, 2, D>(c, a, win, qjl, plan, st);
+        case 6: return launch_attend<D, KB, 3, 32>(c, a, win, qjl, plan, st);
+        case 7: return launch_attend<D, KB, 3, D>(c, a, win, qjl, plan, st);
+        case 8: return launch_attend<D, KB, 4, 32>(c, a, win, qjl, plan, st);
+        case 9: return launch_attend<D, KB, 4, D>(c, a, win, qjl, plan, st);
+        case 16: return launch_attend<D, KB, 8, 32>(c, a, win, qjl, plan, st);
+        case 17: return launch_attend<D, KB, 8, D>(c, a, win, qjl, plan, st);
         default: return fail(TQ_ERR_UNSUPPORTED, "tq_attend_decode: v_bits=%d", a->v_bits);
     }
 }
@@ -608,10 +705,10 @@ tq_status check_window(const char* fn, const tq_attend_window* w) {
 }
 
 tq_status attend_decode_impl(const char* fn, const tq_codec* c, const tq_attend_args* a, const tq_attend_window* win,
-                             void* stream) {
+                             void* stream, const tq_qjl_keys* qjl = nullptr) {
     if (!c) return fail(TQ_ERR_INVALID_ARG, "%s: codec is NULL", fn);
     AttendPlan plan;
-    tq_status s = plan_attend(a, &plan, win != nullptr);
+    tq_status s = plan_attend(a, &plan, win != nullptr, kAttendCtasPerSm, qjl != nullptr);
     if (s != TQ_OK) return s;
     if (a->head_dim != c->d) return fail(TQ_ERR_INVALID_ARG, "%s: head_dim=%d but the codec has d=%d", fn, a->head_dim, c->d);
     if (!a->q || !a->k_packed || !a->k_norms || !a->v_data || !a->v_scales || !a->v_zeros || !a->out)
@@ -628,20 +725,26 @@ tq_status attend_decode_impl(const char* fn, const tq_codec* c, const tq_attend_
         if (!aligned(win->k, 16) || !aligned(win->v, 16) || (win->lens && !aligned(win->lens, 4)))
             return fail(TQ_ERR_INVALID_ARG, "%s: window k and v must be 16-byte aligned", fn);
     }
+    if (qjl) {
+        if (!c->qjl_bits) return fail(TQ_ERR_INVALID_ARG, "%s: the codec was not made by tq_codec_create_qjl", fn);
+        if (!qjl->signs || !qjl->rho) return fail(TQ_ERR_INVALID_ARG, "%s: signs and rho must be non-NULL", fn);
+        if (!aligned(qjl->signs, 16) || !aligned(qjl->rho, 16))
+            return fail(TQ_ERR_INVALID_ARG, "%s: signs and rho must be 16-byte aligned", fn);
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     switch (c->d * 10 + c->bits) {
-        case 641: return attend_v<64, 1>(c, a, win, plan, st);
-        case 642: return attend_v<64, 2>(c, a, win, plan, st);
-        case 643: return attend_v<64, 3>(c, a, win, plan, st);
-        case 644: return attend_v<64, 4>(c, a, win, plan, st);
-        case 1281: return attend_v<128, 1>(c, a, win, plan, st);
-        case 1282: return attend_v<128, 2>(c, a, win, plan, st);
-        case 1283: return attend_v<128, 3>(c, a, win, plan, st);
-        case 1284: return attend_v<128, 4>(c, a, win, plan, st);
-        case 2561: return attend_v<256, 1>(c, a, win, plan, st);
-        case 2562: return attend_v<256, 2>(c, a, win, plan, st);
-        case 2563: return attend_v<256, 3>(c, a, win, plan, st);
-        case 2564: return attend_v<256, 4>(c, a, win, plan, st);
+        case 641: return attend_v<64, 1>(c, a, win, qjl, plan, st);
+        case 642: return attend_v<64, 2>(c, a, win, qjl, plan, st);
+        case 643: return attend_v<64, 3>(c, a, win, qjl, plan, st);
+        case 644: return attend_v<64, 4>(c, a, win, qjl, plan, st);
+        case 1281: return attend_v<128, 1>(c, a, win, qjl, plan, st);
+        case 1282: return attend_v<128, 2>(c, a, win, qjl, plan, st);
+        case 1283: return attend_v<128, 3>(c, a, win, qjl, plan, st);
+        case 1284: return attend_v<128, 4>(c, a, win, qjl, plan, st);
+        case 2561: return attend_v<256, 1>(c, a, win, qjl, plan, st);
+        case 2562: return attend_v<256, 2>(c, a, win, qjl, plan, st);
+        case 2563: return attend_v<256, 3>(c, a, win, qjl, plan, st);
+        case 2564: return attend_v<256, 4>(c, a, win, qjl, plan, st);
         default: return fail(TQ_ERR_UNSUPPORTED, "%s: d=%d bits=%d", fn, c->d, c->bits);
     }
 }
@@ -675,6 +778,12 @@ tq_status launch_scores(const tq_codec* c, const tq_attend_args* a, const Attend
     p.k_norms = a->k_norms;
     p.qfrag = static_cast<uint4*>(a->workspace);
     p.num_splits = p.num_parts = 1;
+    p.qfrag_stride = qfrag_slots<D>();
+    p.k_signs = nullptr;
+    p.k_rho = nullptr;
+    p.s_op = nullptr;
+    p.s_scale_log2 = 0.f;
+    p.s_row_bound = 0.f;
     attend_prep_kernel<D><<<dim3(D / 32, a->num_kv_heads, a->batch), kPrepThreads, 0, st>>>(p);
     TQ_CUDA(cudaGetLastError(), "tq_attend_scores: query preparation launch");
     cudaLaunchAttribute attr[1];
@@ -722,6 +831,24 @@ extern "C" tq_status tq_attend_workspace_bytes(const tq_attend_args* a, size_t* 
     if (s != TQ_OK) return s;
     *bytes = plan.workspace_bytes;
     return TQ_OK;
+}
+
+extern "C" tq_status tq_attend_qjl_workspace_bytes(const tq_attend_args* a, size_t* bytes) {
+    clear_error();
+    if (!bytes) return fail(TQ_ERR_INVALID_ARG, "tq_attend_qjl_workspace_bytes: bytes is NULL");
+    *bytes = 0;
+    AttendPlan plan;
+    tq_status s = plan_attend(a, &plan, false, kAttendCtasPerSm, true);
+    if (s != TQ_OK) return s;
+    *bytes = plan.workspace_bytes;
+    return TQ_OK;
+}
+
+extern "C" tq_status tq_attend_decode_qjl(const tq_codec* c, const tq_attend_args* a, const tq_qjl_keys* keys,
+                                          void* stream) {
+    clear_error();
+    if (!keys) return fail(TQ_ERR_INVALID_ARG, "tq_attend_decode_qjl: keys is NULL");
+    return attend_decode_impl("tq_attend_decode_qjl", c, a, nullptr, stream, keys);
 }
 
 extern "C" tq_status tq_attend_window_workspace_bytes(const tq_attend_args* a, const tq_attend_window* w, size_t* bytes) {

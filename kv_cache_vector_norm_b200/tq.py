@@ -44,6 +44,11 @@ class AttendWindow(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("lens", ctypes.c_void_p), ("max_len", ctypes.c_int)]
 
 
+class QjlKeys(ctypes.Structure):
+    """Mirror of tq_qjl_keys."""
+    _fields_ = [("signs", ctypes.c_void_p), ("rho", ctypes.c_void_p)]
+
+
 SIGNATURES = {
     "tq_last_error": (ctypes.c_char_p, []),
     "tq_version": (ctypes.c_int, []),
@@ -76,6 +81,16 @@ SIGNATURES = {
     "tq_attend_decode_window": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs),
                                                ctypes.POINTER(AttendWindow), ctypes.c_void_p]),
     "tq_read_device_flag": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), ctypes.c_int]),
+    "tq_codec_create_qjl": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_uint64, ctypes.c_int,
+                                           ctypes.POINTER(ctypes.c_void_p)]),
+    "tq_codec_qjl_bits": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)]),
+    "tq_make_qjl_matrix": (ctypes.c_int, [ctypes.c_int, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]),
+    "tq_attend_qjl_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(AttendArgs), ctypes.POINTER(ctypes.c_size_t)]),
+    "tq_attend_decode_qjl": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs), ctypes.POINTER(QjlKeys),
+                                            ctypes.c_void_p]),
+    "tq_encode_k_qjl": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 
@@ -200,6 +215,52 @@ class Codec:
         _check("tq_decode_k", LIB.tq_decode_k(self._h, _ptr(packed), _ptr(norms), n, _ptr(out), dt,
                                               _stream(packed.device)))
         return out
+
+
+def make_qjl_matrix(d: int, seed: int = 0):
+    """(S fp64 [d, d], fp16(S) as float16 [d, d]) of a QJL codec, built by the library on the host."""
+    s = np.empty((d, d), dtype=np.float64)
+    s16 = np.empty((d, d), dtype=np.uint16)
+    _check("tq_make_qjl_matrix", LIB.tq_make_qjl_matrix(d, seed, s.ctypes.data, s16.ctypes.data))
+    return s, s16.view(np.float16)
+
+
+class QjlCodec(Codec):
+    """A QJL key codec: the MSE stage at bits - 1 (an ordinary Codec of bits - 1 for encode_k / decode_k /
+    attend_decode) plus the seeded Gaussian sketch S of the residual."""
+
+    def __init__(self, d: int, bits: int, seed: int = 0, rotation: str = "haar"):
+        h = ctypes.c_void_p()
+        _check("tq_codec_create_qjl", LIB.tq_codec_create_qjl(d, bits, seed, ROTATIONS[rotation], ctypes.byref(h)))
+        self._h = h
+        self.d, self.bits, self.seed, self.rotation = d, bits - 1, seed, rotation
+        self.qjl_bits = bits
+        self.row_bytes = d * (bits - 1) // 8
+
+    def encode_k_qjl(self, x: torch.Tensor, slot_mapping: torch.Tensor | None = None,
+                     packed: torch.Tensor | None = None, norms: torch.Tensor | None = None,
+                     signs: torch.Tensor | None = None, rho: torch.Tensor | None = None):
+        """x: [N, d] fp16.  Returns (packed u8 [rows, d*(bits-1)/8], norms f32 [rows], signs u8 [rows, d/8],
+        rho f32 [rows])."""
+        _need_cuda(x, "x", torch.float16)
+        if x.dim() != 2 or x.shape[1] != self.d or x.stride(1) != 1:
+            raise ValueError(f"x must be [N, {self.d}] with unit column stride")
+        n = x.shape[0]
+        if packed is None:
+            packed = torch.empty((n, self.row_bytes), dtype=torch.uint8, device=x.device)
+        rows = packed.shape[0]
+        if norms is None:
+            norms = torch.empty((rows,), dtype=torch.float32, device=x.device)
+        if signs is None:
+            signs = torch.empty((rows, self.d // 8), dtype=torch.uint8, device=x.device)
+        if rho is None:
+            rho = torch.empty((rows,), dtype=torch.float32, device=x.device)
+        if slot_mapping is not None:
+            _need_cuda(slot_mapping, "slot_mapping", torch.int64)
+        _check("tq_encode_k_qjl", LIB.tq_encode_k_qjl(self._h, _ptr(x), n, x.stride(0), _ptr(slot_mapping),
+                                                      _ptr(packed), _ptr(norms), _ptr(signs), _ptr(rho),
+                                                      _stream(x.device)))
+        return packed, norms, signs, rho
 
 
 # ---------------------------------------------------------------------------------- value codec
@@ -359,6 +420,32 @@ def attend_scores(codec: Codec, q: torch.Tensor, cache: Cache, *, num_kv_heads: 
     a = _attend_args(codec, q, cache, out=None, workspace=workspace, **kw)
     _check("tq_attend_scores", LIB.tq_attend_scores(codec.handle, ctypes.byref(a), scores.data_ptr(), _stream(q.device)))
     return scores
+
+
+def attend_decode_qjl(codec: "QjlCodec", q: torch.Tensor, cache: Cache, signs: torch.Tensor, rho: torch.Tensor, *,
+                      num_kv_heads: int, v_bits: int, v_group: int = 32, max_seq_len: int | None = None,
+                      block_table: torch.Tensor | None = None, seq_lens: torch.Tensor | None = None,
+                      scale: float = 0.0, out: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Decode attention over QJL residual keys: cache holds the MSE stage (codes at bits - 1, norms) and the
+    values; signs [rows, d/8] u8 and rho [rows] f32 the residual sketch.  Returns out [B, H_q, d] f32."""
+    _need_cuda(q, "q", torch.float16)
+    _need_cuda(signs, "signs", torch.uint8)
+    _need_cuda(rho, "rho", torch.float32)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    kw = dict(num_kv_heads=num_kv_heads, v_bits=v_bits, v_group=v_group, max_seq_len=max_seq_len,
+              block_table=block_table, seq_lens=seq_lens, scale=scale)
+    if workspace is None:
+        a0 = _attend_args(codec, q, cache, out=None, workspace=None, **kw)
+        nb = ctypes.c_size_t()
+        _check("tq_attend_qjl_workspace_bytes", LIB.tq_attend_qjl_workspace_bytes(ctypes.byref(a0), ctypes.byref(nb)))
+        workspace = torch.empty(max(16, nb.value), dtype=torch.uint8, device=q.device)
+    a = _attend_args(codec, q, cache, out=out, workspace=workspace, **kw)
+    keys = QjlKeys(signs.data_ptr(), rho.data_ptr())
+    _check("tq_attend_decode_qjl", LIB.tq_attend_decode_qjl(codec.handle, ctypes.byref(a), ctypes.byref(keys),
+                                                            _stream(q.device)))
+    return out
 
 
 ATTEND_SCRATCH_BYTES = 4 << 20

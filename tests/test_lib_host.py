@@ -125,3 +125,11 @@ def test_codec_create_without_device_reports_cuda_error():
     h = ctypes.c_void_p()
     assert tq.LIB.tq_codec_create(128, 4, 0, ctypes.byref(h)) == tq.TQ_ERR_CUDA
     assert h.value is None
+
+
+@pytest.mark.parametrize("d", [8, 64, 128, 256])
+def test_qjl_matrix_matches_oracle(d):
+    for seed in (0, 77):
+        s, s16 = tq.make_qjl_matrix(d, seed)
+        assert np.max(np.abs(s - o.qjl_matrix(d, seed))) < 1e-12      # libm last-ulp differences only
+        assert np.array_equal(s16.astype(np.float64), o.operational_qjl_matrix(d, seed))
