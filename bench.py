@@ -63,11 +63,18 @@ WORKLOADS = {
 
 def algorithmic_bytes(w):
     """Bytes per unit of each launch: per vector for the codec calls (the appended token counts its key and
-    value), per (token, kv head) for attention."""
+    value), per (token, kv head) for attention.  With QJL keys of k_bits total bits the key is the MSE stage at
+    k_bits - 1 plus d/8 bytes of signs and a 4-byte residual norm; its decode reads the MSE stage only."""
     d, kb, vb, g = w["d"], w["k_bits"], w["v_bits"], w["v_group"]
-    k = 2 * d + d * kb // 8 + 4
     v = 2 * d + (d * vb + 7) // 8 + 4 * (d // g)
-    att = (d * kb // 8 + 4) + ((d * vb + 7) // 8 + 4 * (d // g))
+    vrow = (d * vb + 7) // 8 + 4 * (d // g)
+    if w.get("qjl"):
+        mse = d * (kb - 1) // 8 + 4
+        k_enc = 2 * d + mse + d // 8 + 4
+        return {"encode_k": k_enc, "decode_k": 2 * d + mse, "encode_v": v, "decode_v": v, "append": k_enc + v,
+                "attend": mse + d // 8 + 4 + vrow}
+    k = 2 * d + d * kb // 8 + 4
+    att = (d * kb // 8 + 4) + vrow
     return {"encode_k": k, "decode_k": k, "encode_v": v, "decode_v": v, "append": k + v, "attend": att}
 
 
@@ -241,7 +248,9 @@ def build_workload(w, dev, seed, rotation):
     k = synth.kv_tensor(seed, synth.STREAM_K, b, hkv, t, d, device=dev, scales=ks).view(n_in, d)
     v = synth.kv_tensor(seed, synth.STREAM_V, b, hkv, t, d, device=dev, scales=vs).view(n_in, d) if has_v else None
     q = synth.normal_fp16(seed, synth.STREAM_Q, (b, hq, d), device=dev) if has_v else None
-    codec = tq.Codec(d, kb, 0, rotation=rotation)
+    qjl = bool(w.get("qjl"))
+    codec = tq.QjlCodec(d, kb, 0, rotation=rotation) if qjl else tq.Codec(d, kb, 0, rotation=rotation)
+    kbm = kb - 1 if qjl else kb                           # bits of the stored codes
     slots = table = lens = k_new = v_new = new_slots = None
     if kind == "paged":
         per_seq = t // 16 + 1                             # room for the appended token
@@ -253,8 +262,10 @@ def build_workload(w, dev, seed, rotation):
         lens = torch.full((b,), t + 1, dtype=torch.int32, device=dev)
     else:
         n_pool = n_in
-    kp = torch.zeros(n_pool, d * kb // 8, dtype=torch.uint8, device=dev)
+    kp = torch.zeros(n_pool, d * kbm // 8, dtype=torch.uint8, device=dev)
     kn = torch.zeros(n_pool, dtype=torch.float32, device=dev)
+    ksg = torch.zeros(n_pool, d // 8, dtype=torch.uint8, device=dev) if qjl else None
+    krho = torch.zeros(n_pool, dtype=torch.float32, device=dev) if qjl else None
     kdec = torch.empty(n_pool, d, dtype=torch.float16, device=dev)
     vd = vsc = vz = vdec = out = cache = ws = akw = None
     if has_v:
@@ -271,9 +282,20 @@ def build_workload(w, dev, seed, rotation):
             akw = dict(num_kv_heads=hkv, v_bits=vb, v_group=vg, max_seq_len=t, block_table=None, seq_lens=None,
                        scale=0.0)
         ws = tq.attend_workspace(codec, q, cache, **akw)
+        if qjl:
+            a0 = tq._attend_args(codec, q, cache, out=None, workspace=None, **akw)
+            import ctypes
+            nb = ctypes.c_size_t()
+            tq.LIB.tq_attend_qjl_workspace_bytes(ctypes.byref(a0), ctypes.byref(nb))
+            ws = torch.empty(max(16, nb.value), dtype=torch.uint8, device=dev)
 
     def enc_k(r0, r1):
-        if slots is None:
+        if qjl:
+            if slots is None:
+                codec.encode_k_qjl(k[r0:r1], packed=kp[r0:r1], norms=kn[r0:r1], signs=ksg[r0:r1], rho=krho[r0:r1])
+            else:
+                codec.encode_k_qjl(k[r0:r1], slot_mapping=slots[r0:r1], packed=kp, norms=kn, signs=ksg, rho=krho)
+        elif slots is None:
             codec.encode_k(k[r0:r1], packed=kp[r0:r1], norms=kn[r0:r1])
         else:
             codec.encode_k(k[r0:r1], slot_mapping=slots[r0:r1], packed=kp, norms=kn)
@@ -291,11 +313,17 @@ def build_workload(w, dev, seed, rotation):
         tq.decode_v(vd[r0:r1], vsc[r0:r1], vz[r0:r1], d, vb, vg, out=vdec[r0:r1])
 
     def append():
-        codec.encode_k(k_new, slot_mapping=new_slots, packed=kp, norms=kn)
+        if qjl:
+            codec.encode_k_qjl(k_new, slot_mapping=new_slots, packed=kp, norms=kn, signs=ksg, rho=krho)
+        else:
+            codec.encode_k(k_new, slot_mapping=new_slots, packed=kp, norms=kn)
         tq.encode_v(v_new, vb, vg, slot_mapping=new_slots, data=vd, scales=vsc, zeros=vz)
 
     def attend():
-        tq.attend_decode(codec, q, cache, out=out, workspace=ws, **akw)
+        if qjl:
+            tq.attend_decode_qjl(codec, q, cache, ksg, krho, out=out, workspace=ws, **akw)
+        else:
+            tq.attend_decode(codec, q, cache, out=out, workspace=ws, **akw)
 
     kernels = [("encode_k", lambda: enc_k(0, n_in))]
     if has_v:
@@ -310,8 +338,9 @@ def build_workload(w, dev, seed, rotation):
     att_tokens = (t + 1) if kind == "paged" else t
     # launches per call: one for each codec call; attention = query preparation + split kernel (+ the split
     # merge when the workspace holds split-K partials beyond the query fragments)
-    qfrag_bytes = b * hkv * ((d // 16) * 32 + 2) * 16
-    per_call = {"append": 2, "attend": (3 if ws.numel() > qfrag_bytes else 2) if has_v else 0}
+    qfrag_bytes = b * hkv * ((d // 16) * 32 + 2) * 16 * (2 if qjl else 1)
+    per_call = {"append": 3 if qjl else 2, "attend": (3 if ws.numel() > qfrag_bytes else 2) if has_v else 0,
+                "encode_k": 2 if qjl else 1}
     return dict(kind=kind, n_in=n_in, n_pool=n_pool, att_units=b * hkv * att_tokens, kernels=kernels,
                 per_call=per_call, enc_k=enc_k, enc_v=enc_v, dec_k=dec_k, dec_v=dec_v, append=append, attend=attend,
                 k=k, v=v, q=q, k_new=k_new, v_new=v_new, kdec=kdec, vdec=vdec, out=out, has_v=has_v,
@@ -611,19 +640,32 @@ def oracle_sample(w, tokens, seed=0, head=0):
     k = synth.kv_rows(seed, synth.STREAM_K, shape, rows, scales=ks).numpy()
     v = synth.kv_rows(seed, synth.STREAM_V, shape, rows, scales=vs).numpy() if has_v else None
     q = synth.normal_fp16(seed, synth.STREAM_Q, (1, g, d)).numpy()
+    qjl = bool(w.get("qjl"))
+    kbm = kb - 1 if qjl else kb
     pi = o.operational_rotation(d, 0)
-    c, t = o.operational_codebook(d, kb)
+    c, t = o.operational_codebook(d, kbm)
+    s_op = o.operational_qjl_matrix(d, 0) if qjl else None
     layout = "token" if vg == d else "group"
     t0 = time.perf_counter()
-    idx, nrm, _ = o.encode_k(k, pi, t)
-    packed = o.pack_lsb(idx, kb)
+    if qjl:
+        idx, nrm, _, sbits, rho, _ = o.encode_k_qjl(k, pi, c, t, s_op)
+        signs = o.pack_lsb(sbits.astype(np.int64), 1)
+    else:
+        idx, nrm, _ = o.encode_k(k, pi, t)
+    packed = o.pack_lsb(idx, kbm)
     nrm32 = nrm.astype(np.float32)
-    kidx = o.unpack_lsb(packed, kb, d)
+    kidx = o.unpack_lsb(packed, kbm, d)
     o.decode_k(kidx, nrm32.astype(np.float64), pi, c)
     if has_v:
         data, s16, z16, _ = o.encode_v(v, vb, 32, layout)
         vhat = o.decode_v(data, s16, z16, vb, d, 32, layout)
-        o.attend(q, kidx[None, None], nrm32.astype(np.float64)[None, None], vhat[None, None], pi, c)
+        n64 = nrm32.astype(np.float64)[None, None]
+        if qjl:
+            bits = o.unpack_lsb(signs, 1, d).astype(bool)
+            o.attend_qjl(q, kidx[None, None], n64, bits[None, None], rho.astype(np.float32).astype(np.float64)[None, None],
+                         vhat[None, None], pi, c, s_op)
+        else:
+            o.attend(q, kidx[None, None], n64, vhat[None, None], pi, c)
     return time.perf_counter() - t0
 
 
@@ -753,12 +795,16 @@ def main():
     ap.add_argument("--sweep-rows", type=int, default=1 << 24)
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="row chunks of the end-to-end pass (host copies overlap the kernels across chunks)")
+    ap.add_argument("--qjl", action="store_true",
+                    help="QJL residual keys of the workload's key bits (MSE stage at bits - 1 + sign sketch)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the workload's cache length (a multiple of 16; profiling aid for small captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = dict(WORKLOADS[args.workload])
+    if args.qjl:
+        w["qjl"] = True
     if args.tokens > 0:
         if args.tokens % 16:
             ap.error("--tokens must be a multiple of 16")
@@ -770,6 +816,7 @@ def main():
     config = {"workload": args.workload, "description": w["desc"], "batch": w["batch"], "kv_heads": w["kv_heads"],
               "q_heads": w["q_heads"], "tokens": w["tokens"], "head_dim": w["d"], "k_bits": w["k_bits"],
               "v_bits": w["v_bits"], "v_group": w["v_group"], "rotation": args.rotation, "window": args.window,
+              "qjl": bool(w.get("qjl")),
               "vector": "one (token, kv head) key/value pair through encode + decode + attention",
               "l2": "flushed by a 256 MiB write before every kernel launch (outside the timed interval)",
               "e2e": f"pinned host buffers, {max(1, args.e2e_chunks)} row chunks pipelined over host-to-device, kernel "

@@ -424,6 +424,25 @@ tq_status tq_attend_decode_qjl(const tq_codec* codec, const tq_attend_args* args
  */
 tq_status tq_read_device_flag(int* flag_out, int clear);
 
+/*
+ * tq_stream_status -- wait for the work queued on `stream` (that stream only; other streams keep running) and
+ * report whether any kernel's bounded wait has expired: TQ_ERR_DEVICE_FLAG (with the flag in tq_last_error)
+ * if the device's error flag is set, else TQ_OK.  clear != 0 resets the flag after reading it.  A kernel
+ * whose wait expired has stopped its roles, let every copy and tensor-core operation it issued complete,
+ * released its tensor memory and returned, so the context stays usable; its outputs are incomplete.
+ */
+tq_status tq_stream_status(void* stream, int clear);
+
+/*
+ * tq_debug_encode_k_stalled -- a test of the bounded-wait path: tq_encode_k on n contiguous rows (row stride d)
+ * with the first 128-row tile's copy withheld in every CTA and every wait limited to wait_limit_cycles
+ * (1000 .. 2^31).  Nothing waits on a copy or an MMA that was issued and is still in flight: the waits on
+ * the withheld tile run out, the kernel raises the device flag, drains what it issued, frees its tensor memory
+ * and returns.  Follow with tq_stream_status to read the result.  The outputs are not meaningful.
+ */
+tq_status tq_debug_encode_k_stalled(const tq_codec* codec, const void* x, int64_t n, uint8_t* packed, float* norms,
+                                    long long wait_limit_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

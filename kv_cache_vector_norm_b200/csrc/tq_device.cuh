@@ -58,13 +58,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait until the phase of `bar` with the given parity has completed.  Gives up after
 // kWaitLimitCycles, raises the device flag and sets *abort (a shared-memory flag every role polls),
 // returning false.  Also returns false at once if *abort is already set.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          long long limit = kWaitLimitCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long start = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - start > kWaitLimitCycles) {
+        if (clock64() - start > limit) {
             *abort = 1;
             raise_flag(kFlagWaitTimeout);
             return false;
@@ -74,12 +75,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 
 // Bounded wait that ignores the abort flag: used to drain copies or MMAs still in flight before a CTA
 // releases shared or tensor memory, on the normal and the abort path alike.
-__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, long long limit = kWaitLimitCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long start = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (clock64() - start > kWaitLimitCycles) {
+        if (clock64() - start > limit) {
             raise_flag(kFlagWaitTimeout);
             return false;
         }

@@ -292,7 +292,8 @@ namespace {
 
 template <int D, int BITS>
 tq_status launch_encode_k(const tq_codec* c, const void* x, int64_t n, int64_t stride, const int64_t* slots,
-                          uint8_t* packed, float* norms, cudaStream_t st) {
+                          uint8_t* packed, float* norms, cudaStream_t st, long long wait_limit = kWaitLimitCycles,
+                          int withhold_first_tile = 0) {
     static std::atomic<uint64_t> mask{0};
     constexpr uint32_t smem = enc_smem_bytes<D, BITS>();
     auto kern = encode_k_kernel<D, BITS>;
@@ -302,7 +303,8 @@ tq_status launch_encode_k(const tq_codec* c, const void* x, int64_t n, int64_t s
     if (s != TQ_OK) return s;
     const int64_t tiles = (n + 127) / 128;
     const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-    kern<<<grid, EncCfg<D>::kThreads, smem, st>>>(tx, c->tmap_pi, c->enc_lut, n, slots, packed, norms);
+    kern<<<grid, EncCfg<D>::kThreads, smem, st>>>(tx, c->tmap_pi, c->enc_lut, n, slots, packed, norms, wait_limit,
+                                                  withhold_first_tile);
     TQ_CUDA(cudaGetLastError(), "tq_encode_k: launch");
     return TQ_OK;
 }
@@ -377,8 +379,9 @@ tq_status launch_qjl_residual(const tq_codec* c, const void* x, int64_t n, int64
     constexpr uint32_t smem = qjl_smem_bytes<D, KB>();
     auto kern = qjl_residual_kernel<D, KB>;
     TQ_CUDA(allow_smem(kern, smem, mask), "tq_encode_k_qjl: cudaFuncSetAttribute");
-    const int64_t grid = (n + 16 * kQjlWarps - 1) / (16 * kQjlWarps);
-    kern<<<static_cast<unsigned>(grid), 32 * kQjlWarps, smem, st>>>(static_cast<const __half*>(x), n, stride, slots,
+    constexpr int W = qjl_warps<D>();
+    const int64_t grid = (n + 16 * W - 1) / (16 * W);
+    kern<<<static_cast<unsigned>(grid), 32 * W, smem, st>>>(static_cast<const __half*>(x), n, stride, slots,
                                                                      packed, norms, c->pair_lut, c->pi_op_t, c->s_op,
                                                                      signs, rho);
     TQ_CUDA(cudaGetLastError(), "tq_encode_k_qjl: residual launch");
@@ -923,6 +926,37 @@ extern "C" tq_status tq_attend_decode_noalloc(const tq_codec* c, const tq_attend
 }
 
 // --------------------------------------------------------------------------------------- diagnostics
+
+extern "C" tq_status tq_stream_status(void* stream, int clear) {
+    clear_error();
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned v = 0;
+    TQ_CUDA(cudaMemcpyFromSymbolAsync(&v, g_error_flag, sizeof(v), 0, cudaMemcpyDeviceToHost, st),
+            "tq_stream_status: read");
+    TQ_CUDA(cudaStreamSynchronize(st), "tq_stream_status: cudaStreamSynchronize");
+    if (v && clear) {
+        const unsigned z = 0;
+        TQ_CUDA(cudaMemcpyToSymbolAsync(g_error_flag, &z, sizeof(z), 0, cudaMemcpyHostToDevice, st),
+                "tq_stream_status: clear");
+        TQ_CUDA(cudaStreamSynchronize(st), "tq_stream_status: cudaStreamSynchronize");
+    }
+    if (v) return fail(TQ_ERR_DEVICE_FLAG, "a kernel's bounded wait expired (device flag 0x%x)", v);
+    return TQ_OK;
+}
+
+extern "C" tq_status tq_debug_encode_k_stalled(const tq_codec* c, const void* x, int64_t n, uint8_t* packed,
+                                               float* norms, long long wait_limit_cycles, void* stream) {
+    clear_error();
+    if (!c) return fail(TQ_ERR_INVALID_ARG, "tq_debug_encode_k_stalled: codec is NULL");
+    if (n < 1 || n > (1ll << 31) - 256) return fail(TQ_ERR_INVALID_ARG, "tq_debug_encode_k_stalled: n=%lld", (long long)n);
+    if (wait_limit_cycles < 1000 || wait_limit_cycles > kWaitLimitCycles)
+        return fail(TQ_ERR_INVALID_ARG, "tq_debug_encode_k_stalled: wait_limit_cycles=%lld outside [1000, %lld]",
+                    wait_limit_cycles, static_cast<long long>(kWaitLimitCycles));
+    if (!x || !packed || !norms || !aligned(x, 16) || !aligned(packed, 16) || !aligned(norms, 4))
+        return fail(TQ_ERR_INVALID_ARG, "tq_debug_encode_k_stalled: x, packed and norms must be non-NULL and aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TQ_DISPATCH_DB(c->d, c->bits, launch_encode_k, c, x, n, c->d, nullptr, packed, norms, st, wait_limit_cycles, 1);
+}
 
 extern "C" tq_status tq_read_device_flag(int* flag_out, int clear) {
     clear_error();

@@ -85,6 +85,9 @@ SIGNATURES = {
                                            ctypes.POINTER(ctypes.c_void_p)]),
     "tq_codec_qjl_bits": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)]),
     "tq_make_qjl_matrix": (ctypes.c_int, [ctypes.c_int, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]),
+    "tq_stream_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int]),
+    "tq_debug_encode_k_stalled": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p]),
     "tq_attend_qjl_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(AttendArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "tq_attend_decode_qjl": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(AttendArgs), ctypes.POINTER(QjlKeys),
                                             ctypes.c_void_p]),
@@ -467,6 +470,16 @@ def attend_decode_noalloc(codec: Codec, q: torch.Tensor, cache: Cache, *, num_kv
                      workspace=None)
     _check("tq_attend_decode_noalloc", LIB.tq_attend_decode_noalloc(codec.handle, ctypes.byref(a), _stream(q.device)))
     return out
+
+
+def stream_status(device=None, clear: bool = True) -> int:
+    """tq_stream_status on the current stream of `device`: the status code (0 or TQ_ERR_DEVICE_FLAG); raises on
+    any other error."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = LIB.tq_stream_status(_stream(dev), 1 if clear else 0)
+    if st not in (TQ_OK, TQ_ERR_DEVICE_FLAG):
+        _check("tq_stream_status", st)
+    return st
 
 
 def read_device_flag(clear: bool = True) -> int:
