@@ -26,9 +26,11 @@ constexpr int kGridCells = 256;
 constexpr float kCodeMagic = 12582912.0f;                   // 1.5 * 2^23
 constexpr uint32_t kCodeMagicBits = 0x4B400000u;
 
-// RN(x / L) for x >= 0 and L in {3, 7, 15, 255}: q = RN(x RN(1/L)), then one FMA correction with the exact
-// residual x - q L.  Checked exhaustively against IEEE division for every non-negative finite fp32 x and each
-// of the four L (all 2^31 - 2^23 values, on the host with hardware FMA).
+// RN(x / L) for x >= 0 and L in {3, 7, 15, 255}: q = RN(x RN(1/L)), then one correction step with the exact
+// residual x - q L computed by an FMA -- the quotient correction of Markstein's method (P. Markstein, "IA-64
+// and Elementary Functions", 2000; the residual of a product is exact under an FMA), applied once to a constant
+// divisor.  Checked exhaustively against IEEE division for every non-negative finite fp32 x and each of the
+// four L (all 2^31 - 2^23 values, on the host with hardware FMA).
 template <int L>
 __device__ __forceinline__ float div_by_levels(float x) {
     constexpr float y = 1.0f / static_cast<float>(L);

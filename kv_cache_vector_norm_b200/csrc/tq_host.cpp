@@ -219,8 +219,64 @@ void host_codebook(int d, int bits, double* levels) {
         }
         c[i] = 0.5 * (lo + hi);
     }
-    // Lloyd iteration on the positive half: boundaries = midpoints, levels = cell centroids
-    for (int it = 0; it < 200000; ++it) {
+    // Newton's method on the Lloyd fixed point c = g(c), g_i the centroid of cell i = [t_i, t_{i+1}] with
+    // t_i = (c_{i-1} + c_i) / 2 (t_0 = 0, t_half = 1).  A centroid moves with its two boundaries,
+    //   dg_i/dt_i = f(t_i) (g_i - t_i) / P_i,   dg_i/dt_{i+1} = f(t_{i+1}) (t_{i+1} - g_i) / P_i   (P_i the mass),
+    // and each boundary with its two levels (1/2 each), so J = dg/dc is tridiagonal and each step solves
+    // (J - I) dc = c - g(c) by the Thomas algorithm.  The plain iteration below converges linearly with a rate
+    // near 1 - O(1 / half^2) (minutes at 8 bits); Newton's converges quadratically to the same fixed point.
+    // A step that would break the ordering 0 < c_0 < ... < c_{half-1} < 1 is halved.
+    bool newton_converged = false;
+    {
+        std::vector<double> g(half), lo_d(half), di(half), up(half), r(half), cp(half), dp(half), nc(half);
+        double prev = INFINITY;
+        for (int it = 0; it < 60; ++it) {
+            t[0] = 0.0;
+            t[half] = 1.0;
+            for (int i = 1; i < half; ++i) t[i] = 0.5 * (c[i - 1] + c[i]);
+            double rmax = 0.0, cmax = 0.0;
+            for (int i = 0; i < half; ++i) {
+                const double mass = s.moment(t[i], t[i + 1], 0, spread);
+                g[i] = s.m1(t[i], t[i + 1]) / mass;
+                const double a_lo = (i > 0) ? s.f(t[i]) * (g[i] - t[i]) / mass : 0.0;
+                const double a_hi = (i < half - 1) ? s.f(t[i + 1]) * (t[i + 1] - g[i]) / mass : 0.0;
+                lo_d[i] = 0.5 * a_lo;
+                up[i] = 0.5 * a_hi;
+                di[i] = 0.5 * (a_lo + a_hi) - 1.0;
+                r[i] = c[i] - g[i];
+                rmax = std::fmax(rmax, std::fabs(r[i]));
+                cmax = std::fmax(cmax, std::fabs(c[i]));
+            }
+            // converged to the quadrature's noise floor (about 1e-15 relative): a further step cannot reduce it
+            if (rmax <= 1e-13 * cmax) newton_converged = true;
+            if (rmax <= 2e-16 * cmax || (newton_converged && rmax > 0.25 * prev)) break;
+            prev = rmax;
+            // Thomas algorithm for the tridiagonal system (lo_d, di, up) dc = r
+            cp[0] = up[0] / di[0];
+            dp[0] = r[0] / di[0];
+            for (int i = 1; i < half; ++i) {
+                const double m = di[i] - lo_d[i] * cp[i - 1];
+                cp[i] = up[i] / m;
+                dp[i] = (r[i] - lo_d[i] * dp[i - 1]) / m;
+            }
+            for (int i = half - 2; i >= 0; --i) dp[i] -= cp[i] * dp[i + 1];
+            double lambda = 1.0;
+            for (int tries = 0; tries < 40; ++tries, lambda *= 0.5) {
+                bool ordered = true;
+                for (int i = 0; i < half; ++i) {
+                    nc[i] = c[i] + lambda * dp[i];
+                    if (nc[i] <= (i ? nc[i - 1] : 0.0) || nc[i] >= 1.0) ordered = false;
+                }
+                if (ordered) break;
+            }
+            c.swap(nc);
+        }
+    }
+    // Lloyd iteration on the positive half: boundaries = midpoints, levels = cell centroids.  After Newton's
+    // solution it only polishes (at most 1000 steps, as the 2e-16 stop can lie below the quadrature's noise);
+    // it is also the fallback, with the full iteration budget, if Newton's did not converge
+    const int lloyd_iters = newton_converged ? 1000 : 200000;
+    for (int it = 0; it < lloyd_iters; ++it) {
         t[0] = 0.0;
         t[half] = 1.0;
         for (int i = 1; i < half; ++i) t[i] = 0.5 * (c[i - 1] + c[i]);

@@ -303,13 +303,14 @@ def boundaries_of(c: np.ndarray) -> np.ndarray:
     return 0.5 * (c[:-1] + c[1:])
 
 
-def operational_codebook(d: int, bits: int):
+def operational_codebook(d: int, bits: int, levels: np.ndarray | None = None):
     """(c_op, t): c_op = fp16(c*) as fp64 values; t = the midpoints of c_op, which are exact in fp32.
 
     Reading: the kernels compare rotated coordinates with fp32 boundaries and gather fp16 levels, so
     the operational codebook is c* rounded once to fp16; the oracle consumes the same values.
+    ``levels`` may pass c* when it is already at hand (the 7- and 8-bit fixed points take minutes).
     """
-    c_op = to_fp16_values(sphere_codebook(d, bits))
+    c_op = to_fp16_values(sphere_codebook(d, bits) if levels is None else np.asarray(levels, dtype=np.float64))
     t = boundaries_of(c_op)
     if not np.array_equal(t.astype(np.float32).astype(np.float64), t):
         raise AssertionError("boundary midpoints of fp16 levels are expected to be exact in fp32")

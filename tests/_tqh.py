@@ -9,11 +9,27 @@ Rules (the tolerances of the parity contract):
   GPU's own indices.
 """
 import functools
+import json
+import os
 
 import numpy as np
 import torch
 
 from oracle import tq_oracle as o
+
+_GOLDEN_CB = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "sphere_codebooks_b7_b8.json")
+
+
+@functools.lru_cache(maxsize=None)
+def sphere_codebook(d: int, bits: int) -> np.ndarray:
+    """The oracle's c* (sphere_codebook); the 7- and 8-bit ones at d = 64, 128, 256 come from the file
+    tests/golden/make_sphere_codebooks.py wrote with the oracle (their plain iteration takes minutes)."""
+    if bits >= 7:
+        with open(_GOLDEN_CB) as f:
+            book = json.load(f)["codebooks"].get(f"{d}/{bits}")
+        if book is not None:
+            return np.array([float.fromhex(h) for h in book])
+    return o.sphere_codebook(d, bits)
 
 BAND = 1e-5
 FLIP_LIMIT = 1e-4
@@ -24,7 +40,7 @@ L2_RTOL = 1e-3
 @functools.lru_cache(maxsize=None)
 def params(d: int, bits: int, seed: int, rotation: str = "haar"):
     pi_op = o.operational_rotation(d, seed, rotation)
-    c_op, t = o.operational_codebook(d, bits)
+    c_op, t = o.operational_codebook(d, bits, levels=sphere_codebook(d, bits))
     return pi_op, c_op, t
 
 

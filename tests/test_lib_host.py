@@ -11,6 +11,7 @@ import torch
 
 from kv_cache_vector_norm_b200 import tq
 from oracle import tq_oracle as o
+from _tqh import sphere_codebook
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -133,3 +134,17 @@ def test_qjl_matrix_matches_oracle(d):
         s, s16 = tq.make_qjl_matrix(d, seed)
         assert np.max(np.abs(s - o.qjl_matrix(d, seed))) < 1e-12      # libm last-ulp differences only
         assert np.array_equal(s16.astype(np.float64), o.operational_qjl_matrix(d, seed))
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("bits", [5, 6, 7, 8])
+def test_high_width_codebook_matches_oracle(d, bits):
+    # the library solves the Lloyd fixed point by Newton's method; the oracle by the plain iteration (its 7- and
+    # 8-bit fixed points are the stored ones): same levels, the same fp16 operational levels and boundaries
+    cb = tq.build_codebook(d, bits)
+    c = sphere_codebook(d, bits)
+    assert np.max(np.abs(cb["centroids"] - c)) < 1e-12 * np.max(np.abs(c))
+    c_op, t = o.operational_codebook(d, bits, levels=c)
+    assert np.array_equal(cb["centroids_f16"].astype(np.float64), c_op)
+    assert np.array_equal(cb["boundaries"].astype(np.float64), t)
+    assert abs(cb["distortion"] - o.sphere_distortion(d, c_op, t)) < 1e-10

@@ -11,11 +11,14 @@ import pytest
 from scipy import integrate, special
 
 from oracle import tq_oracle as o
+from _tqh import sphere_codebook
+
+STORED = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "sphere_codebooks_b7_b8.json")))
 
 GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "pages_figures.json")))
 
 
-@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6])
 def test_d3_is_uniform_quantizer(bits):
     # On S^2 one coordinate is uniform on [-1, 1] (Archimedes), so Lloyd-Max is the uniform quantizer.
     c = o.sphere_codebook(3, bits)
@@ -53,9 +56,9 @@ def test_large_d_limit_is_gaussian(bits):
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_codebook_invariants_and_bounds(d, bits):
-    c = o.sphere_codebook(d, bits)
+    c = sphere_codebook(d, bits)
     assert np.all(np.diff(c) > 0)
     assert np.array_equal(c, -c[::-1])
     dist = o.SphereMarginal(d)
@@ -110,14 +113,14 @@ def test_sphere_marginal_matches_uniform_unit_vectors(d):
     assert ks < 1.95 / math.sqrt(n)      # 0.1% critical value
 
 
-@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_monte_carlo_distortion_of_unit_vectors(bits):
     # E ||y - Q(y)||^2 over uniform unit vectors y in R^128 equals D(b, 128).
     d, n = 128, 20000
     rng = np.random.default_rng(100 + bits)
     v = rng.standard_normal((n, d))
     y = v / np.linalg.norm(v, axis=1, keepdims=True)
-    c = o.sphere_codebook(d, bits)
+    c = sphere_codebook(d, bits)
     q = c[o.nearest_index(y, o.boundaries_of(c))]
     err = np.sum((y - q) ** 2, axis=1)
     D = o.sphere_distortion(d, c)
@@ -125,13 +128,47 @@ def test_monte_carlo_distortion_of_unit_vectors(bits):
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_operational_codebook(d, bits):
-    c = o.sphere_codebook(d, bits)
-    c_op, t = o.operational_codebook(d, bits)
+    c = sphere_codebook(d, bits)
+    c_op, t = o.operational_codebook(d, bits, levels=c)
     assert np.array_equal(c_op, c.astype(np.float16).astype(np.float64))
     assert np.array_equal(t.astype(np.float32).astype(np.float64), t)
     d_star = o.sphere_distortion(d, c)
     d_op = o.sphere_distortion(d, c_op, t)
     # fp16 rounding moves D only at second order
     assert 0.0 <= d_op - d_star < 1e-3 * d_star
+
+
+@pytest.mark.parametrize("key", sorted(STORED["codebooks"]))
+def test_stored_high_width_codebooks_are_fixed_points_of_the_lloyd_step(key):
+    # the 7- and 8-bit levels the tests read: ascending, symmetric, and each level the conditional mean of its
+    # nearest-neighbour cell under the sphere marginal (one step of the oracle's own iteration moves none of them)
+    d, bits = (int(v) for v in key.split("/"))
+    c = np.array([float.fromhex(h) for h in STORED["codebooks"][key]])
+    assert len(c) == 1 << bits and np.all(np.diff(c) > 0) and np.array_equal(c, -c[::-1])
+    dist = o.SphereMarginal(d)
+    pos = c[len(c) // 2:]
+    t = np.concatenate(([0.0], 0.5 * (pos[:-1] + pos[1:]), [1.0]))
+    g = dist.first_moment(t[:-1], t[1:]) / dist.mass(t[:-1], t[1:])
+    assert np.max(np.abs(g - pos)) <= 1e-13 * pos[-1]
+    lo, hi = o.distortion_bounds(bits)
+    assert lo <= o.sphere_distortion(d, c) <= hi
+
+
+def test_a_stored_codebook_is_the_oracles_own():
+    # the file is the oracle's output: recompute one of its entries (d = 64, 7 bits, about 15 s) and compare
+    c = np.array([float.fromhex(h) for h in STORED["codebooks"]["64/7"]])
+    assert np.array_equal(o.sphere_codebook(64, 7), c)
+
+
+@pytest.mark.parametrize("bits", [5, 6, 7, 8])
+def test_high_width_distortion_approaches_the_gaussian_limit(bits):
+    # D(b, d) grows with d toward the Gaussian quantizer's distortion (d -> infinity); the ordering holds at
+    # every width and the d = 256 value is within a few percent of the limit
+    g, _ = o.lloyd_max(o.GaussianMarginal(), bits) if bits <= 6 else (None, None)
+    ds = [o.sphere_distortion(d, sphere_codebook(d, bits)) for d in (64, 128, 256)]
+    assert ds[0] < ds[1] < ds[2]
+    if g is not None:
+        dg = o.distortion(o.GaussianMarginal(), g)
+        assert ds[2] < dg < ds[2] * 1.03

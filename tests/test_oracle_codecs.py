@@ -10,6 +10,7 @@ import numpy as np
 import pytest
 
 from oracle import tq_oracle as o
+from _tqh import sphere_codebook
 
 GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "pages_figures.json")))
 
@@ -17,7 +18,7 @@ GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "pages
 # ------------------------------------------------------------------------------------ key codec
 
 @pytest.mark.parametrize("d", [3, 4, 8])
-@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6])
 def test_boundary_count_is_brute_force_argmin(d, bits):
     rng = np.random.default_rng(d * 10 + bits)
     x16 = rng.standard_normal((1000, d)).astype(np.float16)
@@ -49,11 +50,11 @@ def test_pack_3bit_worked_example():
     assert list(o.pack_lsb(np.array([[5, 3, 7, 1, 0, 6, 2, 4]]), 3)[0]) == [0xDD, 0x03, 0x8B]
 
 
-@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_zero_vector(bits):
     d = 128
     pi = o.operational_rotation(d, 0)
-    c, t = o.operational_codebook(d, bits)
+    c, t = o.operational_codebook(d, bits, levels=sphere_codebook(d, bits))
     idx, n, _ = o.encode_k(np.zeros((2, d), np.float16), pi, t)
     assert np.all(idx == (1 << (bits - 1)) - 1) and np.all(n == 0.0)
     assert np.all(o.decode_k(idx, n, pi, c) == 0.0)
@@ -71,7 +72,7 @@ def test_power_of_two_scaling_invariance():
     assert np.mean(i1 != i2) < 1e-4 and np.allclose(n2, 4 * n1, rtol=0, atol=0)
 
 
-@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_measured_mse_matches_distortion(bits):
     # Workload of the K-only round trip: 4096 fp16 N(0,1) vectors, head_dim 128, seeded rotation.
     d, n = 128, 4096
@@ -79,7 +80,7 @@ def test_measured_mse_matches_distortion(bits):
     x16 = rng.standard_normal((n, d)).astype(np.float16)
     x = x16.astype(np.float64)
     pi = o.operational_rotation(d, 0)
-    c, t = o.operational_codebook(d, bits)
+    c, t = o.operational_codebook(d, bits, levels=sphere_codebook(d, bits))
     idx, norms, _ = o.encode_k(x16, pi, t)
     xh = o.decode_k(idx, norms, pi, c)
     rel = np.sum((xh - x) ** 2, axis=1) / np.sum(x * x, axis=1)
