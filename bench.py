@@ -547,9 +547,9 @@ def e2e_pass(args, wl, world, dev):
 # ----------------------------------------------------------------------------- bit-width sweep
 
 def sweep_arm(args):
-    """Encode and decode throughput of every key width (1..4 bits) and value width (2/3/4/8 bits, group 32
-    and one group per token) on 2^24 fp16 N(0,1) vectors of d = 128, each launch with a cold L2, plus the
-    measured key distortion mean ||x_hat - x||^2 / ||x||^2 against the codebook's D(b, d)."""
+    """Encode and decode throughput of every key width (1..8 bits; --sweep-key-bits) and value width (2/3/4/8
+    bits, group 32 and one group per token) on 2^24 fp16 N(0,1) vectors of d = 128, each launch with a cold L2,
+    plus the measured key distortion mean ||x_hat - x||^2 / ||x||^2 against the codebook's D(b, d)."""
     import torch
     from kv_cache_vector_norm_b200 import synth, tq
 
@@ -580,7 +580,7 @@ def sweep_arm(args):
                 "GBps": gbps, "frac_of_hbm": gbps / hbm, "bytes_per_vector": bpv}
 
     rows = []
-    for kb in (1, 2, 3, 4):
+    for kb in args.sweep_key_bits:
         codec = tq.Codec(d, kb, 0)
         kp = torch.empty(n, d * kb // 8, dtype=torch.uint8, device=dev)
         kn = torch.empty(n, dtype=torch.float32, device=dev)
@@ -793,6 +793,8 @@ def main():
                     help="bit-width sweep instead of the step: encode/decode of every key and value width on "
                          "--sweep-rows vectors (one JSON line of per-kernel rows)")
     ap.add_argument("--sweep-rows", type=int, default=1 << 24)
+    ap.add_argument("--sweep-key-bits", type=lambda v: [int(x) for x in v.split(",")], default=[1, 2, 3, 4, 5, 6, 7, 8],
+                    help="key widths of the sweep (comma-separated)")
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="row chunks of the end-to-end pass (host copies overlap the kernels across chunks)")
     ap.add_argument("--qjl", action="store_true",

@@ -53,6 +53,11 @@ struct AttendParams {
     float s_row_bound;                               // max over rows of ||S_op row||
 };
 
+// Entries of the key table: a pair of codes -> half2 of codebook values up to 4 bits; from 5 bits (whose
+// 2^(2 bits) pairs would not fit) one code -> its fp16 value in the low half, and a half2 takes two lookups.
+template <int KB>
+__host__ __device__ constexpr int key_table_entries() { return KB > 4 ? (1 << KB) : (1 << (2 * KB)); }
+
 constexpr int kWinMax = 256;                         // largest window per (sequence, kv head)
 constexpr int kWinChunk = 32;                        // window tokens staged in shared memory at a time
 
@@ -74,7 +79,7 @@ struct AttCfg {
     static constexpr int kTileTok = kWarps * kChunkTok;
     // stages of the copy ring (a power of two): 4; 2 with the 32 KB table of 4-bit keys, which keeps four CTAs
     // per SM resident (two 64-token stages of four CTAs still hold ~60 KB per SM in flight)
-    static constexpr int kStages = ((1 << (2 * KB)) * 128 > 8192) ? 2 : 4;
+    static constexpr int kStages = (key_table_entries<KB>() * 128 > 8192) ? 2 : 4;
     static constexpr int kKRow = D * KB / 8;
     static constexpr int kVRow = D * VB / 8;
     static constexpr int kVGroups = D / VG;
@@ -99,7 +104,7 @@ struct AttCfg {
     static constexpr bool kQInRegs = false;
     // key table: a pair of codes (2 KB bits, first code in the low bits) -> half2 of codebook values, with one
     // copy per shared-memory bank (entry e of lane l at byte 128 e + 4 l), so lookups never conflict
-    static constexpr int kPairs = 1 << (2 * KB);
+    static constexpr int kPairs = key_table_entries<KB>();
     static constexpr int kLutBytes = kPairs * 128;
     // shared memory: stages | q fragments (d = 256) | key table (aligned to its size at run time) |
     // per-warp zero sums | barriers
@@ -247,6 +252,25 @@ __device__ __forceinline__ int64_t attend_seq_len(const AttendParams& p, int b) 
     const int64_t cap = p.block_table ? static_cast<int64_t>(p.max_blocks) * 16 : p.max_seq_len;
     const int64_t t = p.seq_lens ? static_cast<int64_t>(p.seq_lens[b]) : cap;
     return t < 0 ? 0 : (t > cap ? cap : t);
+}
+
+// The score B register of code positions j, j + 1 of the lane's key quarter w (j even): the table entry of the
+// pair, or at 5..8 bits the two single entries merged (first code in the low half).  lane_addr: this lane's copy
+// of the table; ALIGNED: the table starts on a multiple of its size, so an address is an OR of field and lane
+// bits, else a sum.
+template <int KB, bool ALIGNED, int NW>
+__device__ __forceinline__ uint32_t key_b_reg(const uint32_t (&w)[NW], int j, uint32_t lane_addr) {
+    if constexpr (KB > 4) {
+        constexpr uint32_t kMask = ((1u << KB) - 1u) << 7;
+        const uint32_t e0 = window_shr(w, j * KB - 7) & kMask, e1 = window_shr(w, (j + 1) * KB - 7) & kMask;
+        const uint32_t v0 = ALIGNED ? lds_u32(lane_addr | e0) : lds_u32(lane_addr + e0);
+        const uint32_t v1 = ALIGNED ? lds_u32(lane_addr | e1) : lds_u32(lane_addr + e1);
+        return __byte_perm(v0, v1, 0x5410);
+    } else {
+        constexpr uint32_t kMask = ((1u << (2 * KB)) - 1u) << 7;
+        const uint32_t e = window_shr(w, j * KB - 7) & kMask;
+        return ALIGNED ? lds_u32(lane_addr | e) : lds_u32(lane_addr + e);
+    }
 }
 
 // Query preparation: the rotated query q_rot[g] = Pi_op q[g] of each of the group's heads, scaled by softmax
@@ -583,7 +607,6 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG, QJL>::kThreads, AttCfg<D
             for (int ks = 0; ks < KS; ++ks) qa[ks] = __ldcg(qf + ks * 32 + lane);
         }
         const uint32_t lane_addr = lut_addr + 4u * lane;
-        constexpr uint32_t kFieldMask = static_cast<uint32_t>(C::kPairs - 1) << 7;
         float o[MT][4];
 #pragma unroll
         for (int m = 0; m < MT; ++m) o[m][0] = o[m][1] = o[m][2] = o[m][3] = 0.f;
@@ -642,13 +665,9 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG, QJL>::kThreads, AttCfg<D
                     if constexpr (C::kQInRegs) a = qa[ks]; else a = s_qf[ks * 32 + lane];
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
-                        const uint32_t e0 = window_shr(w[nt], 4 * ks * KB - 7) & kFieldMask;
-                        const uint32_t e1 = window_shr(w[nt], (4 * ks + 2) * KB - 7) & kFieldMask;
-                        if constexpr (C::kLutAligned) {
-                            mma_f16(sc[nt], a, lds_u32(lane_addr | e0), lds_u32(lane_addr | e1));
-                        } else {
-                            mma_f16(sc[nt], a, lds_u32(lane_addr + e0), lds_u32(lane_addr + e1));
-                        }
+                        // code pairs (4ks, 4ks+1) and (4ks+2, 4ks+3) of the lane's quarter
+                        mma_f16(sc[nt], a, key_b_reg<KB, C::kLutAligned>(w[nt], 4 * ks, lane_addr),
+                                key_b_reg<KB, C::kLutAligned>(w[nt], 4 * ks + 2, lane_addr));
                     }
                 }
                 // ---- logits (log2 domain) of head gid for tokens t0, t0+1, t0+8, t0+9
@@ -883,7 +902,7 @@ __global__ void __launch_bounds__(128) attend_scores_kernel(const AttendParams p
     constexpr int kKRow = D * KB / 8;
     constexpr int kQuarterHalves = D * KB / 4 / 16;
     constexpr int kQuarterWords = (kQuarterHalves + 1) / 2 + 1;
-    constexpr int kPairs = 1 << (2 * KB);
+    constexpr int kPairs = key_table_entries<KB>();
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t lut_addr = (smem_u32(smem) + kPairs * 128 - 1) & ~static_cast<uint32_t>(kPairs * 128 - 1);
     uint32_t* lut = reinterpret_cast<uint32_t*>(smem + (lut_addr - smem_u32(smem)));
@@ -923,16 +942,14 @@ __global__ void __launch_bounds__(128) attend_scores_kernel(const AttendParams p
         }
     }
     const uint32_t lane_addr = lut_addr + 4u * lane;
-    constexpr uint32_t kFieldMask = static_cast<uint32_t>(kPairs - 1) << 7;
     float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
         const uint4 a = __ldcg(qf + ks * 32 + lane);
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-            const uint32_t e0 = window_shr(w[nt], 4 * ks * KB - 7) & kFieldMask;
-            const uint32_t e1 = window_shr(w[nt], (4 * ks + 2) * KB - 7) & kFieldMask;
-            mma_f16(sc[nt], a, lds_u32(lane_addr | e0), lds_u32(lane_addr | e1));
+            mma_f16(sc[nt], a, key_b_reg<KB, true>(w[nt], 4 * ks, lane_addr),
+                    key_b_reg<KB, true>(w[nt], 4 * ks + 2, lane_addr));
         }
     }
     // C columns 2 tig, 2 tig + 1 of n-tile nt are tokens 8 nt + 2 tig (+1), whose norms sit in lanes 4 (2 tig + k)

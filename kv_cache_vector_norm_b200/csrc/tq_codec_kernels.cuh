@@ -388,13 +388,17 @@ struct EncLayout {
     using C = KeyCfg<D>;
     static constexpr int kRowBytes = D * BITS / 8;
     static constexpr int kPkBytes = C::kEncStaged ? 128 * kRowBytes : 0;   // one staged packed tile
+    // input stages: wider packed tiles (5..8 bits) leave room for three at d = 128
+    static constexpr int kStages = (D == 128 && BITS > 4) ? 3 : C::kEncStages;
+    // search table: the 256-cell grid up to 4 bits; from 5 bits the 2^bits boundary slots of a binary search
+    static constexpr int kLutEntries = (BITS > 4) ? (1 << BITS) : C::kLutEntries;
     static constexpr uint32_t kPi = 0;
     static constexpr uint32_t kX = kPi + C::kPiBytes;
-    static constexpr uint32_t kLut = kX + C::kEncStages * C::kTileBytes;
-    static constexpr uint32_t kPk = kLut + C::kLutEntries * 128;            // entry e of lane l at 128 e + 4 l
+    static constexpr uint32_t kLut = kX + kStages * C::kTileBytes;
+    static constexpr uint32_t kPk = kLut + kLutEntries * 128;               // entry e of lane l at 128 e + 4 l
     static constexpr uint32_t kNorm = kPk + 2 * kPkBytes;                   // [stage][128] {norm, 1/(norm+1e-8)}
-    static constexpr uint32_t kBar = kNorm + C::kEncStages * 128 * 8;
-    static constexpr int kBars = 4 * C::kEncStages + 10;
+    static constexpr uint32_t kBar = kNorm + kStages * 128 * 8;
+    static constexpr int kBars = 4 * kStages + 10;
     static constexpr uint32_t kMisc = kBar + 8 * kBars;
     static constexpr uint32_t kBytes = kMisc + 16 + 1024;                  // + alignment slack
     static_assert(kBytes <= 227 * 1024, "encode layout exceeds the shared memory of one CTA");
@@ -414,7 +418,7 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
     using C = KeyCfg<D>;
     using E = EncCfg<D>;
     using Lo = EncLayout<D, BITS>;
-    constexpr int S = C::kEncStages;
+    constexpr int S = Lo::kStages;
     constexpr int kRowBytes = Lo::kRowBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);   // stays a shared-space pointer
@@ -456,7 +460,7 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
-    fill_replicated(reinterpret_cast<uint32_t*>(smem + Lo::kLut), lut_g, C::kLutEntries);
+    fill_replicated(reinterpret_cast<uint32_t*>(smem + Lo::kLut), lut_g, Lo::kLutEntries);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -596,13 +600,27 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                     const uint32_t cell[2] = {__float_as_uint(g2.x), __float_as_uint(g2.y)};
 #pragma unroll
                     for (int e2 = 0; e2 < 2; ++e2) {
+                        if constexpr (BITS > 4) {
+                            // 5..8 bits: branch-free binary search over the ascending boundaries (slot 2^bits - 1
+                            // holds +inf); index = #{t_i < y}, a tie staying below, as with the grid
+                            uint32_t idx = 0;
+#pragma unroll
+                            for (int step = 1 << (BITS - 1); step >= 1; step >>= 1) {
+                                const float tb = __uint_as_float(lds_u32(lut_lane + ((idx + step - 1) << 7)));
+                                idx = (tb < yv[e2]) ? idx + step : idx;
+                            }
+                            add_field<BITS>(w, 2 * j2 + e2, idx);
+                            continue;
+                        }
                         const uint32_t e = lds_u32(lut_lane + ((cell[e2] & (C::kLutEntries - 1)) << 7));
                         // the entry read as a float is the cell's boundary moved by at most 15 ulps (its low 4 bits
                         // hold the count; the boundary's own low bits are zero), or +inf / a NaN when it has none.
                         // The sign of (boundary - y) is set exactly when y lies above the boundary (ties stay below);
                         // +inf - y is +inf and NaN - y the canonical, positive NaN.
-                        const uint32_t above = __float_as_uint(__fsub_rn(__uint_as_float(e), yv[e2])) >> 31;
-                        add_field<BITS>(w, 2 * j2 + e2, (e & 15u) + above);
+                        // index = count + (sign bit of the difference): the high word of diff * 2 is that bit,
+                        // so one multiply-high with the count as addend gives the index
+                        const uint32_t diff = __float_as_uint(__fsub_rn(__uint_as_float(e), yv[e2]));
+                        add_field<BITS>(w, 2 * j2 + e2, __umulhi(diff, 2u) + (e & 15u));
                     }
                 }
                 const int boff = (c0 + k * 32) * BITS / 8;
@@ -665,7 +683,10 @@ struct DecLayout {
     static constexpr int kInBufs = (D == 256) ? 1 : ((D == 128 && BITS == 4) ? 3 : 4);
     // code-pair table: one copy per shared-memory bank (entry e of lane l at 128 e + 4 l) where it fits
     static constexpr bool kReplPairs = (D <= 128);
-    static constexpr int kPairBytes = (1 << (2 * BITS)) * (kReplPairs ? 128 : 4);
+    // up to 4 bits the table maps a pair of codes to a half2 of levels; from 5 bits (2^(2 bits) pairs would not
+    // fit) it maps one code to its fp16 level (low half) and a half2 takes two lookups
+    static constexpr int kEntries = (BITS > 4) ? (1 << BITS) : (1 << (2 * BITS));
+    static constexpr int kPairBytes = kEntries * (kReplPairs ? 128 : 4);
     // d <= 128: the A tile (the looked-up codebook values) is built in tensor memory with tcgen05.st and the MMA
     // reads it from there, which takes its writes and the tensor core's reads off shared memory; d = 256 keeps
     // it in shared memory (its two accumulators fill the 512 TMEM columns)
@@ -682,7 +703,7 @@ struct DecLayout {
     static constexpr uint32_t kPatchBytes = 32 * 64;
     static constexpr int kBars = 2 * C::kDecBufs + 2 * kInBufs + 8;
     static constexpr uint32_t kTailBytes = E::kEpiWarps * kPatchBufs * kPatchBytes + 8 * kBars + 16 + 1024;
-    static constexpr bool kAlignPairs = kReplPairs &&
+    static constexpr bool kAlignPairs = kReplPairs && BITS <= 4 &&
         (((kPair + 2 * kPairBytes + 511) & ~511u) + kTailBytes <= 227 * 1024);
     static constexpr uint32_t kPairRegion = kAlignPairs ? 2 * kPairBytes : kPairBytes;
     // per-warp output patches: 32 rows x 64 bytes, 64B-swizzled, the source of one tensor store each
@@ -710,7 +731,7 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
     constexpr int NI = Lo::kInBufs;
     constexpr int kRowBytes = Lo::kRowBytes;
     constexpr int kPartWords = E::kCols * BITS / 32;   // 32-bit words of this warp's columns of a packed row
-    constexpr int kPairs = 1 << (2 * BITS);
+    constexpr int kPairs = Lo::kEntries;
     constexpr int kOutBytes = OUT_F32 ? 4 : 2;
     constexpr int kPasses = 32 * kOutBytes / 64;   // 64-byte row segments of one 32-column chunk
     extern __shared__ uint8_t smem_raw[];
@@ -860,7 +881,14 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
             if (lane == 0) mbar_arrive(b_inempty + 8 * ib);
             // one half2 of codebook values per code pair (two consecutive columns of the row)
             auto pair_value = [&](int c, int p) -> uint32_t {
-                if constexpr (Lo::kAlignPairs) {
+                if constexpr (BITS > 4) {
+                    // two single-code lookups, merged into one half2 (first column in the low half)
+                    const uint32_t i0 = get_bits<BITS>(w, (c * 8 + 2 * p) * BITS);
+                    const uint32_t i1 = get_bits<BITS>(w, (c * 8 + 2 * p + 1) * BITS);
+                    const uint32_t v0 = Lo::kReplPairs ? lds_u32(pair_lane + i0 * 128u) : s_pair[i0];
+                    const uint32_t v1 = Lo::kReplPairs ? lds_u32(pair_lane + i1 * 128u) : s_pair[i1];
+                    return __byte_perm(v0, v1, 0x5410);
+                } else if constexpr (Lo::kAlignPairs) {
                     const uint32_t x = bits_shr(w, (c * 8 + 2 * p) * BITS - 7);
                     return lds_u32((x & (static_cast<uint32_t>(kPairs - 1) << 7)) | pair_lane);
                 } else {

@@ -161,7 +161,11 @@ extern "C" tq_status tq_codec_create_ex(int d, int k_bits, uint64_t seed, int ro
     if (!out) return fail(TQ_ERR_INVALID_ARG, "tq_codec_create: out is NULL");
     *out = nullptr;
     if (!supported_d(d)) return fail(TQ_ERR_UNSUPPORTED, "tq_codec_create: d=%d (supported: 64, 128, 256)", d);
-    if (k_bits < 1 || k_bits > 4) return fail(TQ_ERR_UNSUPPORTED, "tq_codec_create: k_bits=%d (supported: 1..4)", k_bits);
+    if (k_bits < 1 || k_bits > 8) return fail(TQ_ERR_UNSUPPORTED, "tq_codec_create: k_bits=%d (supported: 1..8)", k_bits);
+    if (k_bits > 4 && d > 128)
+        return fail(TQ_ERR_UNSUPPORTED,
+                    "tq_codec_create: k_bits=%d needs d <= 128 (at d=256 the key decoder's shared memory holds no wider "
+                    "rows)", k_bits);
     if (rotation != TQ_ROT_HAAR && rotation != TQ_ROT_HADAMARD)
         return fail(TQ_ERR_INVALID_ARG, "tq_codec_create: rotation=%d (TQ_ROT_HAAR or TQ_ROT_HADAMARD)", rotation);
     const size_t dd = static_cast<size_t>(d) * d;
@@ -179,10 +183,23 @@ extern "C" tq_status tq_codec_create_ex(int d, int k_bits, uint64_t seed, int ro
     tq_status st = tq_build_codebook(d, k_bits, nullptr, c16.data(), t.data(), nullptr);
     if (st != TQ_OK) return st;
     std::vector<uint32_t> lut;
-    if ((st = build_grid_lut(k_bits, t.data(), lut)) != TQ_OK) return st;
-    std::vector<uint32_t> pairs(1u << (2 * k_bits));
-    for (uint32_t key = 0; key < pairs.size(); ++key)
-        pairs[key] = static_cast<uint32_t>(c16[key & (k - 1)]) | (static_cast<uint32_t>(c16[key >> k_bits]) << 16);
+    std::vector<uint32_t> pairs;
+    if (k_bits <= 4) {
+        // search grid and code-pair table (a pair of codes -> half2 of levels, the first code in the low half)
+        if ((st = build_grid_lut(k_bits, t.data(), lut)) != TQ_OK) return st;
+        pairs.resize(1u << (2 * k_bits));
+        for (uint32_t key = 0; key < pairs.size(); ++key)
+            pairs[key] = static_cast<uint32_t>(c16[key & (k - 1)]) | (static_cast<uint32_t>(c16[key >> k_bits]) << 16);
+    } else {
+        // 5..8 bits: the ascending boundaries of the encoder's binary search (the last slot +inf) and a
+        // single-code table (code -> its fp16 level in the low half)
+        lut.resize(k);
+        for (int i = 0; i < k - 1; ++i) std::memcpy(&lut[i], &t[i], 4);
+        const float inf = INFINITY;
+        std::memcpy(&lut[k - 1], &inf, 4);
+        pairs.resize(k);
+        for (int i = 0; i < k; ++i) pairs[i] = c16[i];
+    }
 
     tq_codec* c = new tq_codec();
     c->d = d;
@@ -195,12 +212,12 @@ extern "C" tq_status tq_codec_create_ex(int d, int k_bits, uint64_t seed, int ro
         return s;
     };
     if (cudaMalloc(&c->pi_op, dd * 2) != cudaSuccess || cudaMalloc(&c->pi_op_t, dd * 2) != cudaSuccess ||
-        cudaMalloc(&c->enc_lut, kGridCells * sizeof(uint32_t)) != cudaSuccess ||
+        cudaMalloc(&c->enc_lut, lut.size() * sizeof(uint32_t)) != cudaSuccess ||
         cudaMalloc(&c->pair_lut, pairs.size() * 4) != cudaSuccess)
         return cleanup(fail(TQ_ERR_CUDA, "tq_codec_create: cudaMalloc failed"));
     if (cudaMemcpy(c->pi_op, pi16.data(), dd * 2, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(c->pi_op_t, pit16.data(), dd * 2, cudaMemcpyHostToDevice) != cudaSuccess ||
-        cudaMemcpy(c->enc_lut, lut.data(), kGridCells * sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->enc_lut, lut.data(), lut.size() * sizeof(uint32_t), cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(c->pair_lut, pairs.data(), pairs.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
         return cleanup(fail(TQ_ERR_CUDA, "tq_codec_create: cudaMemcpy failed"));
     if ((st = make_tmap_f16(&c->tmap_pi, c->pi_op, d, d, d, d)) != TQ_OK) return cleanup(st);
@@ -346,6 +363,14 @@ tq_status launch_decode_k(const tq_codec* c, const uint8_t* packed, const float*
         case 2562: return FN<256, 2>(__VA_ARGS__);                                                    \
         case 2563: return FN<256, 3>(__VA_ARGS__);                                                    \
         case 2564: return FN<256, 4>(__VA_ARGS__);                                                    \
+        case 645: return FN<64, 5>(__VA_ARGS__);                                                      \
+        case 646: return FN<64, 6>(__VA_ARGS__);                                                      \
+        case 647: return FN<64, 7>(__VA_ARGS__);                                                      \
+        case 648: return FN<64, 8>(__VA_ARGS__);                                                      \
+        case 1285: return FN<128, 5>(__VA_ARGS__);                                                    \
+        case 1286: return FN<128, 6>(__VA_ARGS__);                                                    \
+        case 1287: return FN<128, 7>(__VA_ARGS__);                                                    \
+        case 1288: return FN<128, 8>(__VA_ARGS__);                                                    \
         default: return fail(TQ_ERR_UNSUPPORTED, "unsupported d=%d bits=%d", (d), (bits));            \
     }
 
@@ -375,6 +400,9 @@ namespace {
 template <int D, int KB>
 tq_status launch_qjl_residual(const tq_codec* c, const void* x, int64_t n, int64_t stride, const int64_t* slots,
                               const uint8_t* packed, const float* norms, uint8_t* signs, float* rho, cudaStream_t st) {
+    if constexpr (KB > 4) {
+        return fail(TQ_ERR_UNSUPPORTED, "tq_encode_k_qjl: an MSE stage of %d bits (QJL codecs have 1..4)", KB);
+    } else {
     static std::atomic<uint64_t> mask{0};
     constexpr uint32_t smem = qjl_smem_bytes<D, KB>();
     auto kern = qjl_residual_kernel<D, KB>;
@@ -386,6 +414,7 @@ tq_status launch_qjl_residual(const tq_codec* c, const void* x, int64_t n, int64
                                                                      signs, rho);
     TQ_CUDA(cudaGetLastError(), "tq_encode_k_qjl: residual launch");
     return TQ_OK;
+    }
 }
 
 }  // namespace
@@ -676,6 +705,15 @@ template <int D, int KB>
 tq_status attend_v(const tq_codec* c, const tq_attend_args* a, const tq_attend_window* win, const tq_qjl_keys* qjl,
                    const AttendPlan& plan, cudaStream_t st) {
     const bool tok = a->v_group == D;
+    if constexpr (KB > 4) {
+        // keys of 5..8 bits (e.g. protected layers): values of 2, 4 or 8 bits in groups of 32
+        if (!qjl && !tok && a->v_bits == 2) return launch_attend<D, KB, 2, 32>(c, a, win, qjl, plan, st);
+        if (!qjl && !tok && a->v_bits == 4) return launch_attend<D, KB, 4, 32>(c, a, win, qjl, plan, st);
+        if (!qjl && !tok && a->v_bits == 8) return launch_attend<D, KB, 8, 32>(c, a, win, qjl, plan, st);
+        return fail(TQ_ERR_UNSUPPORTED,
+                    "tq_attend_decode: keys of %d bits take values of 2, 4 or 8 bits in groups of 32 (v_bits=%d "
+                    "v_group=%d)", KB, a->v_bits, a->v_group);
+    }
     if (qjl) {
         // QJL residual keys: values of 2 or 4 bits in groups of 32
         if (!tok && a->v_bits == 2) return launch_attend<D, KB, 2, 32, true>(c, a, win, qjl, plan, st);
@@ -748,6 +786,14 @@ tq_status attend_decode_impl(const char* fn, const tq_codec* c, const tq_attend_
         case 2562: return attend_v<256, 2>(c, a, win, qjl, plan, st);
         case 2563: return attend_v<256, 3>(c, a, win, qjl, plan, st);
         case 2564: return attend_v<256, 4>(c, a, win, qjl, plan, st);
+        case 645: return attend_v<64, 5>(c, a, win, qjl, plan, st);
+        case 646: return attend_v<64, 6>(c, a, win, qjl, plan, st);
+        case 647: return attend_v<64, 7>(c, a, win, qjl, plan, st);
+        case 648: return attend_v<64, 8>(c, a, win, qjl, plan, st);
+        case 1285: return attend_v<128, 5>(c, a, win, qjl, plan, st);
+        case 1286: return attend_v<128, 6>(c, a, win, qjl, plan, st);
+        case 1287: return attend_v<128, 7>(c, a, win, qjl, plan, st);
+        case 1288: return attend_v<128, 8>(c, a, win, qjl, plan, st);
         default: return fail(TQ_ERR_UNSUPPORTED, "%s: d=%d bits=%d", fn, c->d, c->bits);
     }
 }
@@ -761,7 +807,7 @@ tq_status launch_scores(const tq_codec* c, const tq_attend_args* a, const Attend
                         int64_t score_len, cudaStream_t st) {
     static std::atomic<uint64_t> mask{0};
     auto kern = attend_scores_kernel<D, KB>;
-    const uint32_t smem = 2u * (1u << (2 * KB)) * 128u;
+    const uint32_t smem = 2u * static_cast<uint32_t>(key_table_entries<KB>()) * 128u;
     TQ_CUDA(allow_smem(kern, smem, mask), "tq_attend_scores: cudaFuncSetAttribute");
     AttendParams p = {};
     p.batch = a->batch;
