@@ -561,23 +561,30 @@ def sweep_arm(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     hbm, peak_src = peaks()
 
-    def timeit(fn):
-        ms = []
-        for i in range(args.warmup + args.steps):
-            flush.fill_(1)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            if i >= args.warmup:
-                ms.append((e0, e1))
-        torch.cuda.synchronize()
-        return statistics.median(a.elapsed_time(b) for a, b in ms)
+    all_reasons = set()
 
-    def entry(kind, bits, layout, bpv, ms):
+    def timeit(fn):
+        # returns (median ms, clocks seen while those launches ran)
+        ms = []
+        sampler = ClockSampler(0)
+        with sampler:
+            for i in range(args.warmup + args.steps):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                if i >= args.warmup:
+                    ms.append((e0, e1))
+            torch.cuda.synchronize()
+        all_reasons.update(sampler.reasons)
+        return statistics.median(a.elapsed_time(b) for a, b in ms), sampler.summary()
+
+    def entry(kind, bits, layout, bpv, timed):
+        ms, clk = timed
         gbps = bpv * n / (ms / 1e3) / 1e9
         return {"kernel": kind, "bits": bits, "layout": layout, "us": ms * 1e3, "Mvectors_s": n / (ms / 1e3) / 1e6,
-                "GBps": gbps, "frac_of_hbm": gbps / hbm, "bytes_per_vector": bpv}
+                "GBps": gbps, "frac_of_hbm": gbps / hbm, "bytes_per_vector": bpv, "sm_mhz": clk["sm_mhz"]}
 
     rows = []
     for kb in args.sweep_key_bits:
@@ -613,7 +620,9 @@ def sweep_arm(args):
         raise RuntimeError("a kernel raised the device error flag during the sweep")
     print(json.dumps({"mode": "bit-width sweep", "vectors": n, "head_dim": d, "data": "synthetic fp16 N(0,1), seed 0",
                       "l2": "flushed by a 256 MiB write before every launch", "steps": args.steps,
-                      "hbm_peak_GBps": hbm, "peak_source": peak_src, "rows": rows}))
+                      "hbm_peak_GBps": hbm, "peak_source": peak_src,
+                      "clocks": {"sm_max_mhz": ClockSampler(0).max_mhz, "reasons": sorted(all_reasons)},
+                      "rows": rows}))
 
 
 # ------------------------------------------------------------------------------------- CPU (oracle)

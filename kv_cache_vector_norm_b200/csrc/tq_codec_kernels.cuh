@@ -680,7 +680,8 @@ struct DecLayout {
     static constexpr int kRowBytes = D * BITS / 8;
     static constexpr int kInBytes = 128 * kRowBytes + 128 * 4;            // packed rows + norms
     // staging buffers for the packed rows: the producer runs up to kInBufs - 1 tiles ahead of the builders
-    static constexpr int kInBufs = (D == 256) ? 1 : ((D == 128 && BITS == 4) ? 3 : 4);
+    // (a buffer is released once its tile's A values are stored; measured best: 6 up to 3 bits, else 4)
+    static constexpr int kInBufs = (D == 256) ? 1 : (BITS <= 3 ? 6 : 4);
     // code-pair table: one copy per shared-memory bank (entry e of lane l at 128 e + 4 l) where it fits
     static constexpr bool kReplPairs = (D <= 128);
     // up to 4 bits the table maps a pair of codes to a half2 of levels; from 5 bits (2^(2 bits) pairs would not
@@ -788,6 +789,8 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
     // a tile's packed rows and norms go through the staging buffer when both copies are 16-byte multiples
     auto tile_rows = [&](int64_t tile) -> int64_t { return (n - tile * 128 < 128) ? n - tile * 128 : 128; };
     auto bulk_ok = [&](int64_t rows) -> bool { return ((rows * kRowBytes) % 16 == 0) && ((rows * 4) % 16 == 0); };
+    // 0 at run time (the host rejects n < 0) but unknown to the compiler: ties a load to a later use (below)
+    const uint32_t opaque_zero = static_cast<uint32_t>(static_cast<uint64_t>(n) >> 63);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -862,23 +865,22 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
             uint32_t w[kPartWords + 1];
             w[kPartWords] = 0u;
             if (r < rows) {
+                auto& wp = *reinterpret_cast<uint32_t(*)[kPartWords]>(w);
                 if (bulk_ok(rows)) {
-                    const uint8_t* src = s_in + ib * Lo::kInBytes + r * kRowBytes + c0 * BITS / 8;
-#pragma unroll
-                    for (int i = 0; i < kPartWords; ++i) w[i] = reinterpret_cast<const uint32_t*>(src)[i];
                     nrm_next = reinterpret_cast<const float*>(s_in + ib * Lo::kInBytes + 128 * kRowBytes)[r];
+                    load_words<kPartWords>(s_in + ib * Lo::kInBytes + r * kRowBytes + c0 * BITS / 8, wp);
+                    // the norm is used only a tile later: make the lookups (and so the A store that precedes the
+                    // release of this buffer) depend on its load as well
+                    w[0] |= __float_as_uint(nrm_next) & opaque_zero;
                 } else {
-                    load_words<kPartWords>(packed + row * kRowBytes + c0 * BITS / 8,
-                                           *reinterpret_cast<uint32_t(*)[kPartWords]>(w));
                     nrm_next = norms[row];
+                    load_words<kPartWords>(packed + row * kRowBytes + c0 * BITS / 8, wp);   // ragged tail
                 }
             } else {
 #pragma unroll
                 for (int i = 0; i < kPartWords; ++i) w[i] = 0u;
                 nrm_next = 0.f;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b_inempty + 8 * ib);
             // one half2 of codebook values per code pair (two consecutive columns of the row)
             auto pair_value = [&](int c, int p) -> uint32_t {
                 if constexpr (BITS > 4) {
@@ -924,8 +926,15 @@ __global__ void __launch_bounds__(DecCfg<D>::kThreads, 1)
                 }
                 fence_proxy_async_smem();
             }
+            // The staging buffer is released only now: the A values just stored were looked up from every word
+            // (and the norm) this warp read from it, so those reads have completed. Releasing it straight after
+            // issuing the loads let the next bulk copy into the buffer overwrite words that a bank-conflicted
+            // shared load (128-byte rows at 8 bits: all 32 lanes in one bank) was still reading.
             __syncwarp();
-            if (lane == 0) mbar_arrive(b_afull + 8 * b);
+            if (lane == 0) {
+                mbar_arrive(b_inempty + 8 * ib);
+                mbar_arrive(b_afull + 8 * b);
+            }
             return true;
         };
 

@@ -317,6 +317,8 @@ __device__ __forceinline__ void store_words(uint8_t* dst, const uint32_t (&w)[NW
     }
 }
 
+// Load NW words with the widest vector loads NW allows: 16-byte loads when NW % 4 == 0 and 8-byte loads when
+// NW is even, so `src` must be aligned to 16 or 8 bytes in those cases (4 otherwise).
 template <int NW>
 __device__ __forceinline__ void load_words(const uint8_t* src, uint32_t (&w)[NW]) {
     if constexpr (NW % 4 == 0) {
@@ -325,9 +327,12 @@ __device__ __forceinline__ void load_words(const uint8_t* src, uint32_t (&w)[NW]
             uint4 v = *reinterpret_cast<const uint4*>(src + 4 * i);
             w[i] = v.x; w[i + 1] = v.y; w[i + 2] = v.z; w[i + 3] = v.w;
         }
-    } else if constexpr (NW == 2) {
-        uint2 v = *reinterpret_cast<const uint2*>(src);
-        w[0] = v.x; w[1] = v.y;
+    } else if constexpr (NW % 2 == 0) {
+#pragma unroll
+        for (int i = 0; i < NW; i += 2) {
+            uint2 v = *reinterpret_cast<const uint2*>(src + 4 * i);
+            w[i] = v.x; w[i + 1] = v.y;
+        }
     } else {
 #pragma unroll
         for (int i = 0; i < NW; ++i) w[i] = reinterpret_cast<const uint32_t*>(src)[i];

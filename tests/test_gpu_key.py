@@ -122,6 +122,32 @@ def test_key_full_size_sampled():
     assert tq.read_device_flag() == 0
 
 
+_DB_ALL = [(d, b) for d in (64, 128, 256) for b in range(1, 9) if b <= 4 or d <= 128]
+
+
+@pytest.mark.parametrize("d,bits", _DB_ALL)
+def test_key_decode_many_tiles_per_cta(d, bits):
+    """Six 128-row tiles per CTA plus a ragged tail, decoded right after a decode of random codes of the same
+    shape: a staging buffer refilled before every read of it had completed, or stale shared memory left by the
+    previous launch, shows up as wrong rows.  Every row is checked against the oracle's decode of the GPU's
+    own indices and norms."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    n = sms * 128 * 6 + 77
+    cd = codec(d, bits)
+    pi, c, t = params(d, bits, 0)
+    x = synth.normal_fp16(900 + bits, synth.STREAM_K, (n, d), device=DEV)
+    packed, norms = cd.encode_k(x)
+    noise = torch.randint(0, 256, tuple(packed.shape), dtype=torch.uint8,
+                          generator=torch.Generator().manual_seed(bits)).to(DEV)
+    cd.decode_k(noise, norms, out_dtype=torch.float32)
+    for out_dtype in (torch.float32, torch.float16):
+        out = to_np(cd.decode_k(packed, norms, out_dtype=out_dtype)).astype(np.float64)
+        ref = o.decode_k(o.unpack_lsb(to_np(packed), bits, d), to_np(norms).astype(np.float64), pi, c)
+        err = np.linalg.norm(out - ref, axis=1)
+        bad = np.nonzero(err > L2_RTOL * np.linalg.norm(ref, axis=1))[0]
+        assert bad.size == 0, f"{bad.size} rows off, first {bad[:8].tolist()}"
+
+
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("bits", [2, 4])
 def test_key_codec_parity_hadamard_rotation(d, bits):
