@@ -77,9 +77,12 @@ struct AttCfg {
     static constexpr int kThreads = 32 * (kWarps + 1);
     static constexpr int kChunkTok = 16;             // tokens per chunk (= one paged block)
     static constexpr int kTileTok = kWarps * kChunkTok;
-    // stages of the copy ring (a power of two): 4; 2 with the 32 KB table of 4-bit keys, which keeps four CTAs
-    // per SM resident (two 64-token stages of four CTAs still hold ~60 KB per SM in flight)
-    static constexpr int kStages = (key_table_entries<KB>() * 128 > 8192) ? 2 : 4;
+    // stages of the copy ring (a power of two): 4; 2 with the 32 KB table of 4-bit keys above d = 64, which keeps
+    // four CTAs per SM resident (two 64-token stages of four CTAs still hold ~60 KB per SM in flight)
+    static constexpr int kStages = (key_table_entries<KB>() * 128 > 8192 && D > 64) ? 2 : 4;
+    // paged blocks of d = 64 are copied by the producer warp's lanes with cp.async, larger ones by bulk copies
+    // from one lane (measured on the 64 x 4096-token paged cache: d = 64 99 vs 106 us, d = 128 162 vs 140 us)
+    static constexpr bool kPagedCpAsync = (D == 64);
     static constexpr int kKRow = D * KB / 8;
     static constexpr int kVRow = D * VB / 8;
     static constexpr int kVGroups = D / VG;
@@ -518,7 +521,8 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG, QJL>::kThreads, AttCfg<D
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(b_full + 8 * s, 1);
+            // one expect-tx arrival by lane 0, or one cp.async arrival per lane of the producer warp (paged)
+            mbar_init(b_full + 8 * s, (p.block_table && C::kPagedCpAsync) ? 32 : 1);
             mbar_init(b_empty + 8 * s, C::kWarps);
         }
         *abort_flag = 0;
@@ -529,18 +533,18 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG, QJL>::kThreads, AttCfg<D
     __syncthreads();
 
     if (warp == C::kWarps) {
-        // ------------------------------------------------------------------ bulk-copy producer
-        if (lane == 0) {
-            for (int64_t ti = 0; ti < ntiles; ++ti) {
-                const int s = static_cast<int>(ti % S);
-                if (!mbar_wait(b_empty + 8 * s, static_cast<uint32_t>((ti / S) & 1) ^ 1u, abort_flag)) break;
-                const int64_t c0 = c_begin + ti * C::kWarps;
-                const int nc = static_cast<int>((c_end - c0 < C::kWarps) ? c_end - c0 : C::kWarps);
-                mbar_arrive_expect_tx(b_full + 8 * s, nc * (C::kStageBytes / C::kWarps));
-                uint8_t* st = smem + s * C::kStageBytes;
-                const uint32_t bar = b_full + 8 * s;
-                if (!p.block_table) {
-                    // the tile's chunks are consecutive rows of the pool: one copy per array
+        // ------------------------------------------------------------------ copy producer
+        if (!p.block_table) {
+            // contiguous cache: a stage's chunks are consecutive rows of the pool, one bulk copy per array (lane 0)
+            if (lane == 0) {
+                for (int64_t ti = 0; ti < ntiles; ++ti) {
+                    const int s = static_cast<int>(ti % S);
+                    if (!mbar_wait(b_empty + 8 * s, static_cast<uint32_t>((ti / S) & 1) ^ 1u, abort_flag)) break;
+                    const int64_t c0 = c_begin + ti * C::kWarps;
+                    const int nc = static_cast<int>((c_end - c0 < C::kWarps) ? c_end - c0 : C::kWarps);
+                    uint8_t* st = smem + s * C::kStageBytes;
+                    const uint32_t bar = b_full + 8 * s;
+                    mbar_arrive_expect_tx(bar, nc * (C::kStageBytes / C::kWarps));
                     const int64_t row0 = (static_cast<int64_t>(b) * p.num_kv_heads + h) * p.max_seq_len + c0 * 16;
                     const int rows = nc * 16;
                     bulk_load(smem_u32(st + C::kKOff), p.k_packed + row0 * C::kKRow, rows * C::kKRow, bar);
@@ -552,26 +556,94 @@ __global__ void __launch_bounds__(AttCfg<D, KB, VB, VG, QJL>::kThreads, AttCfg<D
                         bulk_load(smem_u32(st + C::kSgOff), p.k_signs + row0 * C::kSgRow, rows * C::kSgRow, bar);
                         bulk_load(smem_u32(st + C::kRhoOff), p.k_rho + row0, rows * 4, bar);
                     }
-                } else {
-                    for (int c = 0; c < nc; ++c) {
-                        const int64_t blk = p.block_table[static_cast<int64_t>(b) * p.max_blocks + c0 + c];
-                        const int64_t row0 = (blk * p.num_kv_heads + h) * 16;
-                        bulk_load(smem_u32(st + C::kKOff + c * 16 * C::kKRow), p.k_packed + row0 * C::kKRow,
-                                  16 * C::kKRow, bar);
-                        bulk_load(smem_u32(st + C::kNOff + c * 64), p.k_norms + row0, 64, bar);
-                        bulk_load(smem_u32(st + C::kVOff + c * 16 * C::kVRow), p.v_data + row0 * C::kVRow,
-                                  16 * C::kVRow, bar);
-                        bulk_load(smem_u32(st + C::kSOff + c * 32 * G8), p.v_scales + row0 * G8, 32 * G8, bar);
-                        bulk_load(smem_u32(st + C::kZOff + c * 32 * G8), p.v_zeros + row0 * G8, 32 * G8, bar);
-                        if constexpr (QJL) {
-                            bulk_load(smem_u32(st + C::kSgOff + c * 16 * C::kSgRow), p.k_signs + row0 * C::kSgRow,
-                                      16 * C::kSgRow, bar);
-                            bulk_load(smem_u32(st + C::kRhoOff + c * 64), p.k_rho + row0, 64, bar);
-                        }
+                }
+                for (int64_t ti = (ntiles > S ? ntiles - S : 0); ti < ntiles; ++ti)
+                    mbar_wait_drain(b_full + 8 * static_cast<int>(ti % S), static_cast<uint32_t>((ti / S) & 1));
+            }
+        } else if constexpr (C::kPagedCpAsync) {
+            // paged cache, d = 64: every 16-token block is a separate small piece of each array, and a run of
+            // small bulk copies from one thread is serial, so the whole warp copies a stage in 16-byte cp.async
+            // pieces and each lane arrives on the stage's barrier once its pieces have landed.  The block indices
+            // of 32 chunks are read at once (one per lane), a period ahead of their use.
+            static_assert(32 % C::kWarps == 0, "a stage's chunks lie in one 32-chunk period of block indices");
+            const int32_t* bt = p.block_table + static_cast<int64_t>(b) * p.max_blocks;
+            auto block_at = [&](int64_t rel) -> int32_t {      // block index of the split's chunk rel (0 past the end)
+                return (c_begin + rel < c_end) ? __ldg(bt + c_begin + rel) : 0;
+            };
+            int32_t blk_cur = block_at(lane), blk_next = block_at(32 + lane);
+            for (int64_t ti = 0; ti < ntiles; ++ti) {
+                const int s = static_cast<int>(ti % S);
+                const int64_t rel0 = ti * C::kWarps;            // the stage's first chunk, split-relative
+                if (ti > 0 && (rel0 & 31) == 0) {
+                    blk_cur = blk_next;
+                    blk_next = block_at(rel0 + 32 + lane);
+                }
+                const bool ok =
+                    (lane != 0) || mbar_wait(b_empty + 8 * s, static_cast<uint32_t>((ti / S) & 1) ^ 1u, abort_flag);
+                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+                const int64_t c0 = c_begin + rel0;
+                const int nc = static_cast<int>((c_end - c0 < C::kWarps) ? c_end - c0 : C::kWarps);
+                const uint32_t st_addr = smem_u32(smem + s * C::kStageBytes);
+                int32_t blks[C::kWarps];
+#pragma unroll
+                for (int c = 0; c < C::kWarps; ++c)
+                    blks[c] = __shfl_sync(0xffffffffu, blk_cur, static_cast<int>(rel0 & 31) + c);
+                auto blk_of = [&](int c) -> int32_t {
+                    int32_t v = blks[0];
+#pragma unroll
+                    for (int k = 1; k < C::kWarps; ++k) v = (c == k) ? blks[k] : v;
+                    return v;
+                };
+                // an array of R-byte rows holds a block as 16 R contiguous bytes: R pieces of 16 bytes
+                auto copy_array = [&](uint32_t off, const void* base, int R) {
+                    for (int i = lane; i < nc * R; i += 32) {
+                        const int c = i / R, piece = i - c * R;
+                        const int64_t row0 = (static_cast<int64_t>(blk_of(c)) * p.num_kv_heads + h) * 16;
+                        cp_async16(st_addr + off + static_cast<uint32_t>(c * 16 * R + piece * 16),
+                                   static_cast<const uint8_t*>(base) + row0 * R + piece * 16);
+                    }
+                };
+                copy_array(C::kKOff, p.k_packed, C::kKRow);
+                copy_array(C::kNOff, p.k_norms, 4);
+                copy_array(C::kVOff, p.v_data, C::kVRow);
+                copy_array(C::kSOff, p.v_scales, 2 * G8);
+                copy_array(C::kZOff, p.v_zeros, 2 * G8);
+                if constexpr (QJL) {
+                    copy_array(C::kSgOff, p.k_signs, C::kSgRow);
+                    copy_array(C::kRhoOff, p.k_rho, 4);
+                }
+                cp_async_arrive_noinc(b_full + 8 * s);
+            }
+            if (lane == 0)
+                for (int64_t ti = (ntiles > S ? ntiles - S : 0); ti < ntiles; ++ti)
+                    mbar_wait_drain(b_full + 8 * static_cast<int>(ti % S), static_cast<uint32_t>((ti / S) & 1));
+        } else if (lane == 0) {
+            // paged cache, larger blocks: one bulk copy per array and block, from lane 0
+            for (int64_t ti = 0; ti < ntiles; ++ti) {
+                const int s = static_cast<int>(ti % S);
+                if (!mbar_wait(b_empty + 8 * s, static_cast<uint32_t>((ti / S) & 1) ^ 1u, abort_flag)) break;
+                const int64_t c0 = c_begin + ti * C::kWarps;
+                const int nc = static_cast<int>((c_end - c0 < C::kWarps) ? c_end - c0 : C::kWarps);
+                uint8_t* st = smem + s * C::kStageBytes;
+                const uint32_t bar = b_full + 8 * s;
+                mbar_arrive_expect_tx(bar, nc * (C::kStageBytes / C::kWarps));
+                for (int c = 0; c < nc; ++c) {
+                    const int64_t blk = p.block_table[static_cast<int64_t>(b) * p.max_blocks + c0 + c];
+                    const int64_t row0 = (blk * p.num_kv_heads + h) * 16;
+                    bulk_load(smem_u32(st + C::kKOff + c * 16 * C::kKRow), p.k_packed + row0 * C::kKRow,
+                              16 * C::kKRow, bar);
+                    bulk_load(smem_u32(st + C::kNOff + c * 64), p.k_norms + row0, 64, bar);
+                    bulk_load(smem_u32(st + C::kVOff + c * 16 * C::kVRow), p.v_data + row0 * C::kVRow,
+                              16 * C::kVRow, bar);
+                    bulk_load(smem_u32(st + C::kSOff + c * 32 * G8), p.v_scales + row0 * G8, 32 * G8, bar);
+                    bulk_load(smem_u32(st + C::kZOff + c * 32 * G8), p.v_zeros + row0 * G8, 32 * G8, bar);
+                    if constexpr (QJL) {
+                        bulk_load(smem_u32(st + C::kSgOff + c * 16 * C::kSgRow), p.k_signs + row0 * C::kSgRow,
+                                  16 * C::kSgRow, bar);
+                        bulk_load(smem_u32(st + C::kRhoOff + c * 64), p.k_rho + row0, 64, bar);
                     }
                 }
             }
-            // drain: the last issued stages have landed before the CTA may reuse or leave them
             for (int64_t ti = (ntiles > S ? ntiles - S : 0); ti < ntiles; ++ti)
                 mbar_wait_drain(b_full + 8 * static_cast<int>(ti % S), static_cast<uint32_t>((ti / S) & 1));
         }
