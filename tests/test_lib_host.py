@@ -118,7 +118,11 @@ def test_argument_errors_are_reported():
     assert nb.value == 3 * 2 * (128 // 16 * 32 + 2) * 16                   # only the prepared query fragments
     assert tq.LIB.tq_attend_decode(None, ctypes.byref(a), None) == tq.TQ_ERR_INVALID_ARG
     assert tq.LIB.tq_codec_create(96, 4, 0, ctypes.byref(ctypes.c_void_p())) == tq.TQ_ERR_UNSUPPORTED
-    assert tq.LIB.tq_codec_create(128, 5, 0, ctypes.byref(ctypes.c_void_p())) == tq.TQ_ERR_UNSUPPORTED
+    # key widths 1..8; from 5 bits only at d <= 128
+    assert tq.LIB.tq_codec_create(256, 5, 0, ctypes.byref(ctypes.c_void_p())) == tq.TQ_ERR_UNSUPPORTED
+    assert b"d <= 128" in tq.LIB.tq_last_error()
+    assert tq.LIB.tq_codec_create(128, 9, 0, ctypes.byref(ctypes.c_void_p())) == tq.TQ_ERR_UNSUPPORTED
+    assert tq.LIB.tq_codec_create(128, 0, 0, ctypes.byref(ctypes.c_void_p())) == tq.TQ_ERR_UNSUPPORTED
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
