@@ -7,7 +7,8 @@ namespace tq {
 namespace dev {
 
 // Grid of the key encoder's nearest-level search (built on the host, see tq_lib.cu build_grid_lut):
-// kGridCells cells of width 1 / kGridRes, cell = rint(kGridRes * y + kGridOffset).
+// kGridCells cells of width 1 / kGridRes; u = kGridRes * y + kGridOffset is rounded to a multiple of 2^-7 and
+// the cell is its integer part.
 constexpr int kGridRes = 64;
 constexpr int kGridOffset = 128;
 constexpr int kGridCells = 256;
@@ -361,11 +362,12 @@ struct KeyCfg {
     static constexpr uint32_t kIdesc = idesc_f16_f32(128, D);
 };
 
-// Encode-side search: y maps to grid cell rint(64 y + 128) (an exact FMA into the 1.5*2^23 magic range);
-// the cell's entry holds the count L of boundaries below the cell and the one boundary B that may fall
-// inside it (+inf if none): index = L + (y > B).
+// Encode-side search: one FMA g = 64 y + (1.5 * 2^16 + 128) rounds u = 64 y + 128 to a multiple of 2^-7 (the
+// float's ulp in [2^16, 2^17)), so bits 7..14 of g hold the cell (the integer part of the rounded u) already
+// shifted into place for a table entry of 128 bytes; the cell's entry holds the count L of boundaries below the
+// cell and the one boundary B that may fall inside it (+inf if none): index = L + (y > B).
 constexpr float kGridScale = static_cast<float>(kGridRes);
-constexpr float kGridMagic = 12582912.0f + kGridOffset;   // 1.5 * 2^23 + 128
+constexpr float kGridMagic = 98304.0f + kGridOffset;   // 1.5 * 2^16 + 128
 
 
 
@@ -388,14 +390,17 @@ struct EncLayout {
     using C = KeyCfg<D>;
     static constexpr int kRowBytes = D * BITS / 8;
     static constexpr int kPkBytes = C::kEncStaged ? 128 * kRowBytes : 0;   // one staged packed tile
-    // input stages: wider packed tiles (5..8 bits) leave room for three at d = 128
-    static constexpr int kStages = (D == 128 && BITS > 4) ? 3 : C::kEncStages;
+    // input stages: three at d = 128 (room for the aligned grid table, or for the wider tables of 5..8 bits)
+    static constexpr int kStages = (D == 128) ? 3 : C::kEncStages;
     // search table: the 256-cell grid up to 4 bits; from 5 bits the 2^bits boundary slots of a binary search
     static constexpr int kLutEntries = (BITS > 4) ? (1 << BITS) : C::kLutEntries;
     static constexpr uint32_t kPi = 0;
     static constexpr uint32_t kX = kPi + C::kPiBytes;
     static constexpr uint32_t kLut = kX + kStages * C::kTileBytes;
-    static constexpr uint32_t kPk = kLut + kLutEntries * 128;               // entry e of lane l at 128 e + 4 l
+    // entry e of lane l at 128 e + 4 l; up to d = 128 the 32 KB grid table starts on a multiple of its size
+    // (slack reserved), so an entry's address is (the cell bits of g, already at bits 7..14) | lane bits: one LOP3
+    static constexpr bool kAlignLut = (BITS <= 4 && D <= 128);
+    static constexpr uint32_t kPk = kLut + kLutEntries * 128 * (kAlignLut ? 2 : 1);
     static constexpr uint32_t kNorm = kPk + 2 * kPkBytes;                   // [stage][128] {norm, 1/(norm+1e-8)}
     static constexpr uint32_t kBar = kNorm + kStages * 128 * 8;
     static constexpr int kBars = 4 * kStages + 10;
@@ -424,7 +429,6 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);   // stays a shared-space pointer
     uint8_t* s_pi = smem + Lo::kPi;
     uint8_t* s_x = smem + Lo::kX;
-    const uint32_t* s_lut = reinterpret_cast<const uint32_t*>(smem + Lo::kLut);
     uint8_t* s_pk = smem + Lo::kPk;
     float2* s_norm = reinterpret_cast<float2*>(smem + Lo::kNorm);
     const uint32_t bar0 = smem_u32(smem + Lo::kBar);
@@ -460,7 +464,8 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
-    fill_replicated(reinterpret_cast<uint32_t*>(smem + Lo::kLut), lut_g, Lo::kLutEntries);
+    const uint32_t lut_base = Lo::kAlignLut ? (smem_u32(smem + Lo::kLut) + 32767u) & ~32767u : smem_u32(smem + Lo::kLut);
+    fill_replicated(reinterpret_cast<uint32_t*>(smem + (lut_base - smem_u32(smem))), lut_g, Lo::kLutEntries);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -559,7 +564,7 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         const int c0 = (ew >> 2) * E::kCols;                  // first column of this warp
         const int r = quarter * 32 + lane;
         const bool issuer = (ew == 0 && lane == 0);           // issues the bulk stores of staged tiles
-        const uint32_t lut_lane = smem_u32(s_lut) + 4u * lane; // this lane's copy of the grid table (its own bank)
+        const uint32_t lut_lane = lut_base + 4u * lane;        // this lane's copy of the search table (its own bank)
         int li = 0;
         for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
             const int s = li % S, a = li & 1, pb = li & 1;
@@ -612,7 +617,8 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                             add_field<BITS>(w, 2 * j2 + e2, idx);
                             continue;
                         }
-                        const uint32_t e = lds_u32(lut_lane + ((cell[e2] & (C::kLutEntries - 1)) << 7));
+                        const uint32_t cb = cell[e2] & static_cast<uint32_t>((C::kLutEntries - 1) << 7);
+                        const uint32_t e = lds_u32(Lo::kAlignLut ? (cb | lut_lane) : (lut_lane + cb));
                         // the entry read as a float is the cell's boundary moved by at most 15 ulps (its low 4 bits
                         // hold the count; the boundary's own low bits are zero), or +inf / a NaN when it has none.
                         // The sign of (boundary - y) is set exactly when y lies above the boundary (ties stay below);

@@ -127,16 +127,19 @@ struct tq_codec {
 
 namespace {
 
-// Grid table of the encode search (see encode_k_kernel): cell c holds the y with rint(64 y + 128) = c, so the
-// 256 cells cover y in [-2, 2) (|y| <= ||Pi_op|| < 1.01).  Entry = bits of the one boundary inside the cell
-// (+inf if none) OR the count of boundaries below the cell; the boundaries, midpoints of fp16 levels, have at
-// least 4 zero low bits in fp32 (checked), and no cell holds two of them for any supported d and bits
-// (checked: the closest pair, d = 256 at 4 bits, is 0.016 apart, above the 1/64 cell width).
+// Grid table of the encode search (see encode_k_kernel): cell c holds the y whose u = 64 y + 128, rounded to a
+// multiple of 2^-7, has integer part c, so the 256 cells cover y in [-2, 2) (|y| <= ||Pi_op|| < 1.01).  Each
+// cell is taken as the closed range u in [c - 1/128, c + 1], wider than the values that can reach it: a
+// boundary below it is below every y in the cell, and one inside it is decided by y > B.  Entry = bits of the
+// one boundary inside the cell (+inf if none) OR the count of boundaries below the cell; the boundaries,
+// midpoints of fp16 levels, have at least 4 zero low bits in fp32 (checked), and no cell holds two of them for
+// any supported d and bits (checked: the closest pair, d = 256 at 4 bits, is 0.016 apart, above the widened
+// cell's 0.01575).
 tq_status build_grid_lut(int bits, const float* t, std::vector<uint32_t>& lut) {
     const int nb = (1 << bits) - 1;
     lut.assign(kGridCells, 0);
     for (int c = 0; c < kGridCells; ++c) {
-        const double lo = (c - kGridOffset - 0.5) / kGridRes, hi = (c - kGridOffset + 0.5) / kGridRes;
+        const double lo = (c - kGridOffset - 1.0 / 128) / kGridRes, hi = (c + 1.0 - kGridOffset) / kGridRes;
         uint32_t below = 0;
         int inside = 0;
         float b = INFINITY;
