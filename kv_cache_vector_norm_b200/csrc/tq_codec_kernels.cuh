@@ -12,6 +12,10 @@ namespace dev {
 constexpr int kGridRes = 64;
 constexpr int kGridOffset = 128;
 constexpr int kGridCells = 256;
+// Keys of 5..8 bits: a 1024-cell grid of 8-byte entries (boundary, count below), built by tq_lib.cu
+// build_wide_grid; cell = bits 3..12 of fma(sat(fma(y, s, 0.5)), 1023.75, 1.5 * 2^20)
+constexpr int kWideCells = 1024;
+constexpr int kWideWords = 2 * kWideCells + 4;           // the entries, then s (padded to 16 bytes)
 
 // ------------------------------------------------------------------------------------ value codec
 // "KV Cache API", values.py quantize_values / dequantize_values.  The lanes of one scale group reduce
@@ -392,15 +396,17 @@ struct EncLayout {
     static constexpr int kPkBytes = C::kEncStaged ? 128 * kRowBytes : 0;   // one staged packed tile
     // input stages: three at d = 128 (room for the aligned grid table, or for the wider tables of 5..8 bits)
     static constexpr int kStages = (D == 128) ? 3 : C::kEncStages;
-    // search table: the 256-cell grid up to 4 bits; from 5 bits the 2^bits boundary slots of a binary search
-    static constexpr int kLutEntries = (BITS > 4) ? (1 << BITS) : C::kLutEntries;
+    // search table: the 256-cell grid up to 4 bits, replicated once per bank; from 5 bits the 1024-cell grid of
+    // 8-byte entries (one copy, 8 KB)
+    static constexpr int kLutEntries = C::kLutEntries;
     static constexpr uint32_t kPi = 0;
     static constexpr uint32_t kX = kPi + C::kPiBytes;
     static constexpr uint32_t kLut = kX + kStages * C::kTileBytes;
     // entry e of lane l at 128 e + 4 l; up to d = 128 the 32 KB grid table starts on a multiple of its size
     // (slack reserved), so an entry's address is (the cell bits of g, already at bits 7..14) | lane bits: one LOP3
     static constexpr bool kAlignLut = (BITS <= 4 && D <= 128);
-    static constexpr uint32_t kPk = kLut + kLutEntries * 128 * (kAlignLut ? 2 : 1);
+    static constexpr uint32_t kLutBytes = (BITS > 4) ? kWideWords * 4 : kLutEntries * 128 * (kAlignLut ? 2 : 1);
+    static constexpr uint32_t kPk = kLut + kLutBytes;
     static constexpr uint32_t kNorm = kPk + 2 * kPkBytes;                   // [stage][128] {norm, 1/(norm+1e-8)}
     static constexpr uint32_t kBar = kNorm + kStages * 128 * 8;
     static constexpr int kBars = 4 * kStages + 10;
@@ -465,7 +471,12 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         tmem_relinquish();
     }
     const uint32_t lut_base = Lo::kAlignLut ? (smem_u32(smem + Lo::kLut) + 32767u) & ~32767u : smem_u32(smem + Lo::kLut);
-    fill_replicated(reinterpret_cast<uint32_t*>(smem + (lut_base - smem_u32(smem))), lut_g, Lo::kLutEntries);
+    if constexpr (BITS > 4) {
+        uint32_t* tab = reinterpret_cast<uint32_t*>(smem + Lo::kLut);
+        for (int i = threadIdx.x; i < kWideWords; i += blockDim.x) tab[i] = __ldg(lut_g + i);
+    } else {
+        fill_replicated(reinterpret_cast<uint32_t*>(smem + (lut_base - smem_u32(smem))), lut_g, Lo::kLutEntries);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -565,6 +576,8 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         const int r = quarter * 32 + lane;
         const bool issuer = (ew == 0 && lane == 0);           // issues the bulk stores of staged tiles
         const uint32_t lut_lane = lut_base + 4u * lane;        // this lane's copy of the search table (its own bank)
+        // 5..8 bits: the wide grid's scale s (after the table's entries)
+        const float wide_s = (BITS > 4) ? __uint_as_float(lds_u32(lut_base + 8u * kWideCells)) : 0.f;
         int li = 0;
         for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
             const int s = li % S, a = li & 1, pb = li & 1;
@@ -606,15 +619,14 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
 #pragma unroll
                     for (int e2 = 0; e2 < 2; ++e2) {
                         if constexpr (BITS > 4) {
-                            // 5..8 bits: branch-free binary search over the ascending boundaries (slot 2^bits - 1
-                            // holds +inf); index = #{t_i < y}, a tie staying below, as with the grid
-                            uint32_t idx = 0;
-#pragma unroll
-                            for (int step = 1 << (BITS - 1); step >= 1; step >>= 1) {
-                                const float tb = __uint_as_float(lds_u32(lut_lane + ((idx + step - 1) << 7)));
-                                idx = (tb < yv[e2]) ? idx + step : idx;
-                            }
-                            add_field<BITS>(w, 2 * j2 + e2, idx);
+                            // 5..8 bits: the 1024-cell grid (cell = bits 3..12 of the second FMA, so the offset
+                            // of its 8-byte entry is one LOP3); index = count below + (y > boundary in the cell),
+                            // a tie staying below, as with the 256-cell grid
+                            const float u = __saturatef(fmaf(yv[e2], wide_s, 0.5f));
+                            const float g = fmaf(u, 1023.75f, 1572864.0f);
+                            const uint2 ent = lds_u64(lut_base + (__float_as_uint(g) & ((kWideCells - 1u) << 3)));
+                            const uint32_t diff = __float_as_uint(__fsub_rn(__uint_as_float(ent.x), yv[e2]));
+                            add_field<BITS>(w, 2 * j2 + e2, __umulhi(diff, 2u) + ent.y);
                             continue;
                         }
                         const uint32_t cb = cell[e2] & static_cast<uint32_t>((C::kLutEntries - 1) << 7);

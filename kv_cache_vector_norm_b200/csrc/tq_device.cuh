@@ -255,6 +255,13 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
     return v;
 }
 
+// Two 32-bit words from an 8-byte aligned shared-space address (same ordering rule as lds_u32).
+__device__ __forceinline__ uint2 lds_u64(uint32_t addr) {
+    uint2 v;
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
 // Add value v (< 2^BITS) into field j of the zero-initialised bitstream `w` (fields do not overlap, so this is
 // the same as OR-ing it in, as a shift-add).
 template <int BITS, int NW>

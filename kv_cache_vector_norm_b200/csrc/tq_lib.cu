@@ -157,6 +157,46 @@ tq_status build_grid_lut(int bits, const float* t, std::vector<uint32_t>& lut) {
     return TQ_OK;
 }
 
+// Grid of the encode search for 5..8 bits (see encode_k_kernel): cell(y) = bits 3..12 of
+// fma(sat(fma(y, s, 0.5)), 1023.75, 1.5 * 2^20) with s = 0.499 / max|t|, a monotone map of y onto 1024 cells
+// that the device computes with the same two fp32 FMAs.  Every boundary must land in a cell of its own; then for
+// y in cell c the boundaries of lower cells are below y, those of higher cells above it, and the one in c (if
+// any) is decided by y > B.  Entry c = {bits of the boundary in c (+inf if none), boundaries in lower cells};
+// word 2 * kWideCells holds s.
+uint32_t wide_cell(float y, float s) {
+    float u = std::fmaf(y, s, 0.5f);
+    u = (u > 0.f) ? ((u < 1.f) ? u : 1.f) : 0.f;               // saturate; NaN -> 0
+    const float g = std::fmaf(u, 1023.75f, 1572864.0f);           // ulp 2^-3: the cell at bits 3..12
+    uint32_t b;
+    std::memcpy(&b, &g, 4);
+    return (b >> 3) & (kWideCells - 1);
+}
+
+tq_status build_wide_grid(int bits, const float* t, std::vector<uint32_t>& lut) {
+    const int nb = (1 << bits) - 1;
+    float tmax = 0.f;
+    for (int i = 0; i < nb; ++i) tmax = std::fmax(tmax, std::fabs(t[i]));
+    const float s = static_cast<float>(0.499 / tmax);
+    lut.assign(2 * kWideCells + 4, 0);
+    const float inf = INFINITY;
+    uint32_t inf_bits;
+    std::memcpy(&inf_bits, &inf, 4);
+    for (int c = 0; c < kWideCells; ++c) lut[2 * c] = inf_bits;
+    int prev = -1;
+    for (int i = 0; i < nb; ++i) {
+        const int c = static_cast<int>(wide_cell(t[i], s));
+        if (c <= prev) return fail(TQ_ERR_UNSUPPORTED, "codebook boundaries closer than the wide search grid (bits=%d)", bits);
+        std::memcpy(&lut[2 * c], &t[i], 4);
+        prev = c;
+    }
+    for (int c = 0, below = 0, i = 0; c < kWideCells; ++c) {
+        while (i < nb && static_cast<int>(wide_cell(t[i], s)) < c) { ++i; ++below; }
+        lut[2 * c + 1] = static_cast<uint32_t>(below);
+    }
+    std::memcpy(&lut[2 * kWideCells], &s, 4);
+    return TQ_OK;
+}
+
 }  // namespace
 
 extern "C" tq_status tq_codec_create_ex(int d, int k_bits, uint64_t seed, int rotation, tq_codec** out) {
@@ -194,12 +234,8 @@ extern "C" tq_status tq_codec_create_ex(int d, int k_bits, uint64_t seed, int ro
         for (uint32_t key = 0; key < pairs.size(); ++key)
             pairs[key] = static_cast<uint32_t>(c16[key & (k - 1)]) | (static_cast<uint32_t>(c16[key >> k_bits]) << 16);
     } else {
-        // 5..8 bits: the ascending boundaries of the encoder's binary search (the last slot +inf) and a
-        // single-code table (code -> its fp16 level in the low half)
-        lut.resize(k);
-        for (int i = 0; i < k - 1; ++i) std::memcpy(&lut[i], &t[i], 4);
-        const float inf = INFINITY;
-        std::memcpy(&lut[k - 1], &inf, 4);
+        // 5..8 bits: the 1024-cell search grid and a single-code table (code -> its fp16 level in the low half)
+        if ((st = build_wide_grid(k_bits, t.data(), lut)) != TQ_OK) return st;
         pairs.resize(k);
         for (int i = 0; i < k; ++i) pairs[i] = c16[i];
     }
