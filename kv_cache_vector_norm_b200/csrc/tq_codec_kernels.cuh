@@ -13,9 +13,12 @@ constexpr int kGridRes = 64;
 constexpr int kGridOffset = 128;
 constexpr int kGridCells = 256;
 // Keys of 5..8 bits: a 1024-cell grid of 8-byte entries (boundary, count below), built by tq_lib.cu
-// build_wide_grid; cell = bits 3..12 of fma(sat(fma(y, s, 0.5)), 1023.75, 1.5 * 2^20)
+// build_wide_grid; cell = bits 5..14 of fma(sat(fma(y, s, 0.5)), 1023.75, 1.5 * 2^18).  Each entry is stored
+// kWideCopies times side by side and lane l reads copy l % kWideCopies, which spreads a warp's lookups of nearby
+// cells over more banks.
 constexpr int kWideCells = 1024;
-constexpr int kWideWords = 2 * kWideCells + 4;           // the entries, then s (padded to 16 bytes)
+constexpr int kWideCopies = 4;
+constexpr int kWideWords = 2 * kWideCells * kWideCopies + 4;   // the entries, then s (padded to 16 bytes)
 
 // ------------------------------------------------------------------------------------ value codec
 // "KV Cache API", values.py quantize_values / dequantize_values.  The lanes of one scale group reduce
@@ -576,8 +579,9 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         const int r = quarter * 32 + lane;
         const bool issuer = (ew == 0 && lane == 0);           // issues the bulk stores of staged tiles
         const uint32_t lut_lane = lut_base + 4u * lane;        // this lane's copy of the search table (its own bank)
-        // 5..8 bits: the wide grid's scale s (after the table's entries)
-        const float wide_s = (BITS > 4) ? __uint_as_float(lds_u32(lut_base + 8u * kWideCells)) : 0.f;
+        // 5..8 bits: the wide grid's scale s (after the table's entries) and this lane's copy of the entries
+        const float wide_s = (BITS > 4) ? __uint_as_float(lds_u32(lut_base + 8u * kWideCells * kWideCopies)) : 0.f;
+        const uint32_t wide_lane = lut_base + 8u * static_cast<uint32_t>(lane % kWideCopies);
         int li = 0;
         for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
             const int s = li % S, a = li & 1, pb = li & 1;
@@ -619,12 +623,13 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
 #pragma unroll
                     for (int e2 = 0; e2 < 2; ++e2) {
                         if constexpr (BITS > 4) {
-                            // 5..8 bits: the 1024-cell grid (cell = bits 3..12 of the second FMA, so the offset
-                            // of its 8-byte entry is one LOP3); index = count below + (y > boundary in the cell),
-                            // a tie staying below, as with the 256-cell grid
+                            // 5..8 bits: the 1024-cell grid (cell = bits 5..14 of the second FMA, so the offset of
+                            // its group of kWideCopies 8-byte entries is one LOP3); index = count below + (y >
+                            // boundary in the cell), a tie staying below, as with the 256-cell grid
+                            static_assert(kWideCopies * 8 == 32, "the cell bits give the entry group's byte offset");
                             const float u = __saturatef(fmaf(yv[e2], wide_s, 0.5f));
-                            const float g = fmaf(u, 1023.75f, 1572864.0f);
-                            const uint2 ent = lds_u64(lut_base + (__float_as_uint(g) & ((kWideCells - 1u) << 3)));
+                            const float g = fmaf(u, 1023.75f, 393216.0f);
+                            const uint2 ent = lds_u64(wide_lane + (__float_as_uint(g) & ((kWideCells - 1u) << 5)));
                             const uint32_t diff = __float_as_uint(__fsub_rn(__uint_as_float(ent.x), yv[e2]));
                             add_field<BITS>(w, 2 * j2 + e2, __umulhi(diff, 2u) + ent.y);
                             continue;

@@ -157,19 +157,20 @@ tq_status build_grid_lut(int bits, const float* t, std::vector<uint32_t>& lut) {
     return TQ_OK;
 }
 
-// Grid of the encode search for 5..8 bits (see encode_k_kernel): cell(y) = bits 3..12 of
-// fma(sat(fma(y, s, 0.5)), 1023.75, 1.5 * 2^20) with s = 0.499 / max|t|, a monotone map of y onto 1024 cells
+// Grid of the encode search for 5..8 bits (see encode_k_kernel): cell(y) = bits 5..14 of
+// fma(sat(fma(y, s, 0.5)), 1023.75, 1.5 * 2^18) with s = 0.499 / max|t|, a monotone map of y onto 1024 cells
 // that the device computes with the same two fp32 FMAs.  Every boundary must land in a cell of its own; then for
 // y in cell c the boundaries of lower cells are below y, those of higher cells above it, and the one in c (if
-// any) is decided by y > B.  Entry c = {bits of the boundary in c (+inf if none), boundaries in lower cells};
-// word 2 * kWideCells holds s.
+// any) is decided by y > B.  Entry c = {bits of the boundary in c (+inf if none), boundaries in lower cells},
+// stored kWideCopies times side by side (copy r of entry c at 8-byte slot kWideCopies c + r, so lanes reading
+// different copies of nearby entries use different banks); the word after the entries holds s.
 uint32_t wide_cell(float y, float s) {
     float u = std::fmaf(y, s, 0.5f);
     u = (u > 0.f) ? ((u < 1.f) ? u : 1.f) : 0.f;               // saturate; NaN -> 0
-    const float g = std::fmaf(u, 1023.75f, 1572864.0f);           // ulp 2^-3: the cell at bits 3..12
+    const float g = std::fmaf(u, 1023.75f, 393216.0f);            // 1.5 * 2^18, ulp 2^-5: the cell at bits 5..14
     uint32_t b;
     std::memcpy(&b, &g, 4);
-    return (b >> 3) & (kWideCells - 1);
+    return (b >> 5) & (kWideCells - 1);
 }
 
 tq_status build_wide_grid(int bits, const float* t, std::vector<uint32_t>& lut) {
@@ -177,23 +178,29 @@ tq_status build_wide_grid(int bits, const float* t, std::vector<uint32_t>& lut) 
     float tmax = 0.f;
     for (int i = 0; i < nb; ++i) tmax = std::fmax(tmax, std::fabs(t[i]));
     const float s = static_cast<float>(0.499 / tmax);
-    lut.assign(2 * kWideCells + 4, 0);
+    std::vector<uint32_t> bnd(kWideCells), cnt(kWideCells);
     const float inf = INFINITY;
     uint32_t inf_bits;
     std::memcpy(&inf_bits, &inf, 4);
-    for (int c = 0; c < kWideCells; ++c) lut[2 * c] = inf_bits;
+    for (int c = 0; c < kWideCells; ++c) bnd[c] = inf_bits;
     int prev = -1;
     for (int i = 0; i < nb; ++i) {
         const int c = static_cast<int>(wide_cell(t[i], s));
         if (c <= prev) return fail(TQ_ERR_UNSUPPORTED, "codebook boundaries closer than the wide search grid (bits=%d)", bits);
-        std::memcpy(&lut[2 * c], &t[i], 4);
+        std::memcpy(&bnd[c], &t[i], 4);
         prev = c;
     }
     for (int c = 0, below = 0, i = 0; c < kWideCells; ++c) {
         while (i < nb && static_cast<int>(wide_cell(t[i], s)) < c) { ++i; ++below; }
-        lut[2 * c + 1] = static_cast<uint32_t>(below);
+        cnt[c] = static_cast<uint32_t>(below);
     }
-    std::memcpy(&lut[2 * kWideCells], &s, 4);
+    lut.assign(2 * kWideCells * kWideCopies + 4, 0);
+    for (int c = 0; c < kWideCells; ++c)
+        for (int r = 0; r < kWideCopies; ++r) {
+            lut[2 * (kWideCopies * c + r)] = bnd[c];
+            lut[2 * (kWideCopies * c + r) + 1] = cnt[c];
+        }
+    std::memcpy(&lut[2 * kWideCells * kWideCopies], &s, 4);
     return TQ_OK;
 }
 
