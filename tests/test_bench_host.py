@@ -26,7 +26,7 @@ def test_chunk_bounds_cover_the_rows_in_whole_tiles(n, chunks):
         assert all((x * row_bytes) % 16 == 0 for x in b[:-1])
 
 
-def test_paged_workload_bytes_match_the_survey_figures():
+def test_paged_workload_bytes_per_vector_are_the_layout_sums():
     bench = _bench()
     # high-concurrency paged cache, K 4-bit / V 4-bit group 32: per vector K 164 / 644 B, V 168 / 672 B;
     # attention 76 / 292 B per (token, kv head) at head_dim 64 / 256
