@@ -559,11 +559,10 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                 }
                 const float nrm = sqrtf(((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
                 s_norm[s * 128 + r] = make_float2(nrm, 1.0f / (nrm + 1e-8f));
+                // with a slot mapping the epilogue stores the norm (it loads the row's slot anyway, a tile ahead of
+                // its use); a load of the slot here would stall the norm warps on a global round trip every tile
                 const int64_t row = tile * 128 + r;
-                if (row < n) {
-                    const int64_t orow = slots ? slots[row] : row;
-                    if (orow >= 0) norms[orow] = nrm;
-                }
+                if (row < n && !slots) norms[row] = nrm;
             }
             __syncwarp();
             if (lane == 0) {
@@ -586,7 +585,8 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
             const int s = li % S, a = li & 1, pb = li & 1;
             if (!mbar_wait(b_nrdy + 8 * s, (li / S) & 1, abort_flag, wait_limit)) break;
-            const float inv = s_norm[s * 128 + r].y;
+            const float2 nrm_inv = s_norm[s * 128 + r];
+            const float inv = nrm_inv.y;
             __syncwarp();
             if (lane == 0) mbar_arrive(b_nfree + 8 * s);
             const int64_t row = tile * 128 + r;
@@ -654,6 +654,7 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                     store_words<BITS>(packed + orow * kRowBytes + boff, w);
                 }
             }
+            if (slots && c0 == 0 && orow >= 0) norms[orow] = nrm_inv.x;
             if (staged) {
                 // make this warp's rows visible to the bulk copy engine, then hand the tile to the issuer
                 fence_proxy_async_smem();
