@@ -585,10 +585,11 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
         for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
             const int s = li % S, a = li & 1, pb = li & 1;
             if (!mbar_wait(b_nrdy + 8 * s, (li / S) & 1, abort_flag, wait_limit)) break;
-            const float2 nrm_inv = s_norm[s * 128 + r];
-            const float inv = nrm_inv.y;
+            const float inv = s_norm[s * 128 + r].y;
             __syncwarp();
-            if (lane == 0) mbar_arrive(b_nfree + 8 * s);
+            // with a slot mapping the norm entry is read again (and stored) at the end of the tile, so the stage's
+            // norms are released there
+            if (lane == 0 && !slots) mbar_arrive(b_nfree + 8 * s);
             const int64_t row = tile * 128 + r;
             int64_t orow = -1;
             if (!staged && row < n) orow = slots ? slots[row] : row;
@@ -654,7 +655,11 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                     store_words<BITS>(packed + orow * kRowBytes + boff, w);
                 }
             }
-            if (slots && c0 == 0 && orow >= 0) norms[orow] = nrm_inv.x;
+            if (slots) {
+                if (c0 == 0 && orow >= 0) norms[orow] = s_norm[s * 128 + r].x;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_nfree + 8 * s);
+            }
             if (staged) {
                 // make this warp's rows visible to the bulk copy engine, then hand the tile to the issuer
                 fence_proxy_async_smem();
