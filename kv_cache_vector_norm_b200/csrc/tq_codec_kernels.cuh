@@ -423,7 +423,7 @@ __host__ __device__ constexpr uint32_t enc_smem_bytes() {
     return EncLayout<D, BITS>::kBytes;
 }
 
-template <int D, int BITS>
+template <int D, int BITS, bool SLOTS>
 __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
     encode_k_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_pi,
                     const uint32_t* __restrict__ lut_g, int64_t n, const int64_t* __restrict__ slots,
@@ -449,7 +449,8 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t num_tiles = (n + 127) / 128;
-    const bool staged = C::kEncStaged && (slots == nullptr);
+    // SLOTS: this instantiation writes rows through the slot mapping (the host passes slots != nullptr)
+    constexpr bool staged = C::kEncStaged && !SLOTS;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -562,7 +563,7 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                 // with a slot mapping the epilogue stores the norm (it loads the row's slot anyway, a tile ahead of
                 // its use); a load of the slot here would stall the norm warps on a global round trip every tile
                 const int64_t row = tile * 128 + r;
-                if (row < n && !slots) norms[row] = nrm;
+                if (!SLOTS && row < n) norms[row] = nrm;
             }
             __syncwarp();
             if (lane == 0) {
@@ -589,10 +590,10 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
             __syncwarp();
             // with a slot mapping the norm entry is read again (and stored) at the end of the tile, so the stage's
             // norms are released there
-            if (lane == 0 && !slots) mbar_arrive(b_nfree + 8 * s);
+            if (!SLOTS && lane == 0) mbar_arrive(b_nfree + 8 * s);
             const int64_t row = tile * 128 + r;
             int64_t orow = -1;
-            if (!staged && row < n) orow = slots ? slots[row] : row;
+            if (!staged && row < n) orow = SLOTS ? slots[row] : row;
 
             if (!mbar_wait(b_accfull + 8 * a, (li >> 1) & 1, abort_flag, wait_limit)) break;
             tc_fence_after();
@@ -655,7 +656,7 @@ __global__ void __launch_bounds__(EncCfg<D>::kThreads, 1)
                     store_words<BITS>(packed + orow * kRowBytes + boff, w);
                 }
             }
-            if (slots) {
+            if constexpr (SLOTS) {
                 if (c0 == 0 && orow >= 0) norms[orow] = s_norm[s * 128 + r].x;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(b_nfree + 8 * s);

@@ -357,10 +357,11 @@ template <int D, int BITS>
 tq_status launch_encode_k(const tq_codec* c, const void* x, int64_t n, int64_t stride, const int64_t* slots,
                           uint8_t* packed, float* norms, cudaStream_t st, long long wait_limit = kWaitLimitCycles,
                           int withhold_first_tile = 0) {
-    static std::atomic<uint64_t> mask{0};
+    // separate instantiations with and without a slot mapping, so the contiguous one carries none of its code
+    static std::atomic<uint64_t> mask_rows{0}, mask_slots{0};
     constexpr uint32_t smem = enc_smem_bytes<D, BITS>();
-    auto kern = encode_k_kernel<D, BITS>;
-    TQ_CUDA(allow_smem(kern, smem, mask), "tq_encode_k: cudaFuncSetAttribute");
+    auto kern = slots ? encode_k_kernel<D, BITS, true> : encode_k_kernel<D, BITS, false>;
+    TQ_CUDA(allow_smem(kern, smem, slots ? mask_slots : mask_rows), "tq_encode_k: cudaFuncSetAttribute");
     CUtensorMap tx;
     tq_status s = make_tmap_f16(&tx, x, static_cast<uint64_t>(n), D, static_cast<uint64_t>(stride), 128);
     if (s != TQ_OK) return s;
